@@ -1,0 +1,368 @@
+/*
+ * ss_oracle.c -- plain CPU oracle of the Mamba selective scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * CPU-baseline leg of the benchmark load this file.  The product path (the
+ * CUDA library) never calls it and shares no code with it.
+ *
+ * What it computes follows the equations of "Understanding Mamba and Selective
+ * State Space Models (SSMs)" (bqwf.cn deep-dive article):
+ *   - §2.1   classic SSM, y_n = C h_n + D x_n (skip term D);
+ *   - §2.2, first cut: the selective recurrence h_n = exp(Δ_n A) h_{n-1} + Δ_n B_n x_n;
+ *   - §2.2, second cut: the recurrent scan, state starting at zero;
+ *   - §2.2, closing tip: Δ goes through softplus, log(1 + exp(x));
+ *   - §3.1 (end): the readout against C_n;
+ *   - §4.3: A = -exp(A_log), a diagonal matrix, so every state index n
+ *     evolves on its own.
+ * The optional silu(z) output gate and the bias added to Δ before the softplus
+ * are not on the pages; they follow the benchmark spec of the path
+ * (y = (C_t·h_t + D u_t) * z σ(z), Δ = softplus(Δ_raw + bias)).
+ *
+ * Readings taken where the pages are garbled or silent (each is listed in the
+ * design notes):
+ *   - decay = exp(Δ·A) with A as given (negative); the pseudocode's
+ *     "exp(-Δ·A)" assumes a positive magnitude for A;
+ *   - the readout is the dot product Σ_n C_n h_n (the "⊙" of §3.1 would
+ *     leave an N-vector per channel, contradicting y_n = C h_n of §2.1);
+ *   - B̄ = Δ·B (as written), h_{-1} = 0;
+ *   - D is one constant per channel;
+ *   - softplus(x) = x for x > 20, else log1p(exp(x)).
+ *
+ * Layouts (row-major, no padding):
+ *   u, delta, z, y : [batch, L, d]       (token-major, channels contiguous)
+ *   B, C           : [batch, L, N]       (one group shared by all channels)
+ *   A              : [d, N]
+ *   D, delta_bias  : [d]
+ *   last_state     : [batch, d, N]
+ * Inputs come in as double; callers pass the exact values the GPU consumed
+ * (bf16 or fp32 values widen to double without rounding).
+ *
+ * Two arithmetic modes:
+ *   *_f64 : everything in double (the reference truth);
+ *   *_f32 : state and all arithmetic in float, libm float functions.
+ *
+ * Nothing here is blocked, fused or reordered: each channel runs the
+ * recurrence step by step in time order, exactly as the equations read.
+ * The only parallelism is an OpenMP loop over independent (batch, channel)
+ * pairs.
+ *
+ * Parity pins (tests/test_oracle_pins.py): closed form at L = 1, LTI
+ * reduction to a direct convolution, linearity in u, chunked = sequential,
+ * causality, channel independence, limiting cases, a hand-derived worked
+ * example, and step-by-step decode equivalence.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ---------------------------------------------------------------------------
+ * Test-only planted mistakes.  0 (the default) is the oracle as specified;
+ * a nonzero value switches on ONE deliberate error so that a test can show
+ * that the pins catch it.  Never set outside tests.
+ *   1: decay exp(-Δ·A) (the pseudocode's sign taken literally)
+ *   2: skip term D dropped
+ *   3: B and C swapped
+ *   4: Δ bias ignored
+ *   5: softplus skipped (Δ = Δ_raw + bias)
+ *   6: readout taken before the state update (uses h_{t-1})
+ *   7: gate σ(z) instead of z·σ(z)
+ *   8: Δ missing from the input term (h = Ā h + B u)
+ *   9: A read transposed (A[n*d + ch] instead of A[ch*N + n])
+ * ------------------------------------------------------------------------- */
+static int g_mutation = 0;
+void ss_oracle_set_mutation(int m) { g_mutation = m; }
+int ss_oracle_get_mutation(void) { return g_mutation; }
+
+int ss_oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void ss_oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* softplus in double: log(1 + e^x), with the identity branch above 20
+ * (there log1p(e^x) - x < 2.1e-9, below the precision either side keeps). */
+static double softplus_d(double x)
+{
+    return x > 20.0 ? x : log1p(exp(x));
+}
+
+static float softplus_f(float x)
+{
+    return x > 20.0f ? x : log1pf(expf(x));
+}
+
+static double a_at_d(const double* A, int64_t ch, int64_t n, int64_t d, int64_t N)
+{
+    if (g_mutation == 9) return A[n * d + ch];
+    return A[ch * N + n];
+}
+
+/* Δ for one element, double. */
+static double delta_d(double raw, const double* bias, int64_t ch, int softplus)
+{
+    double x = raw;
+    if (bias && g_mutation != 4) x += bias[ch];
+    if (softplus && g_mutation != 5) return softplus_d(x);
+    return x;
+}
+
+static float delta_f(float raw, const double* bias, int64_t ch, int softplus)
+{
+    float x = raw;
+    if (bias && g_mutation != 4) x += (float)bias[ch];
+    if (softplus && g_mutation != 5) return softplus_f(x);
+    return x;
+}
+
+static double gate_d(double zv)
+{
+    double sig = 1.0 / (1.0 + exp(-zv));
+    return g_mutation == 7 ? sig : zv * sig;
+}
+
+static float gate_f(float zv)
+{
+    float sig = 1.0f / (1.0f + expf(-zv));
+    return g_mutation == 7 ? sig : zv * sig;
+}
+
+/* ---------------------------------------------------------------------------
+ * Forward scan, double precision.
+ * For every (b, ch): h = 0; for t in 0..L-1:
+ *   Δ  = softplus(Δ_raw + bias)
+ *   h_n = exp(Δ A_n) h_n + Δ B_n u          (n = 0..N-1)
+ *   y  = (Σ_n C_n h_n + D u) · z σ(z)
+ * and last_state = h after the final step.
+ * The state lives in a stack array, so N <= 256 is required.
+ * Returns 0, or -1 for unsupported sizes.
+ * ------------------------------------------------------------------------- */
+int ss_oracle_fwd_f64(const double* u, const double* delta, const double* delta_bias,
+                      const double* A, const double* B, const double* C,
+                      const double* D, const double* z, double* y, double* last_state,
+                      int64_t batch, int64_t L, int64_t d, int64_t N, int softplus)
+{
+    if (N < 1 || N > 256 || batch < 0 || L < 0 || d < 0) return -1;
+    const double* Bsel = (g_mutation == 3) ? C : B;
+    const double* Csel = (g_mutation == 3) ? B : C;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t ch = 0; ch < d; ++ch) {
+            double h[256];
+            for (int64_t n = 0; n < N; ++n) h[n] = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t i = (b * L + t) * d + ch;      /* [b, t, ch] */
+                const int64_t bc = (b * L + t) * N;          /* [b, t, 0]  */
+                const double dt = delta_d(delta[i], delta_bias, ch, softplus);
+                const double uv = u[i];
+                double acc = 0.0;
+                if (g_mutation == 6)
+                    for (int64_t n = 0; n < N; ++n) acc += Csel[bc + n] * h[n];
+                for (int64_t n = 0; n < N; ++n) {
+                    const double an = a_at_d(A, ch, n, d, N);
+                    const double decay = (g_mutation == 1) ? exp(-dt * an) : exp(dt * an);
+                    const double input = (g_mutation == 8) ? Bsel[bc + n] * uv
+                                                            : dt * Bsel[bc + n] * uv;
+                    h[n] = decay * h[n] + input;
+                }
+                if (g_mutation != 6)
+                    for (int64_t n = 0; n < N; ++n) acc += Csel[bc + n] * h[n];
+                double yv = acc;
+                if (D && g_mutation != 2) yv += D[ch] * uv;
+                if (z) yv *= gate_d(z[i]);
+                y[i] = yv;
+            }
+            if (last_state)
+                for (int64_t n = 0; n < N; ++n) last_state[(b * d + ch) * N + n] = h[n];
+        }
+    }
+    return 0;
+}
+
+/* Forward scan with the state and every operation in float (the fp32-state
+ * oracle).  Same loop as ss_oracle_fwd_f64; outputs widened to double. */
+int ss_oracle_fwd_f32(const double* u, const double* delta, const double* delta_bias,
+                      const double* A, const double* B, const double* C,
+                      const double* D, const double* z, double* y, double* last_state,
+                      int64_t batch, int64_t L, int64_t d, int64_t N, int softplus)
+{
+    if (N < 1 || N > 256 || batch < 0 || L < 0 || d < 0) return -1;
+    const double* Bsel = (g_mutation == 3) ? C : B;
+    const double* Csel = (g_mutation == 3) ? B : C;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t ch = 0; ch < d; ++ch) {
+            float h[256];
+            for (int64_t n = 0; n < N; ++n) h[n] = 0.0f;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t i = (b * L + t) * d + ch;
+                const int64_t bc = (b * L + t) * N;
+                const float dt = delta_f((float)delta[i], delta_bias, ch, softplus);
+                const float uv = (float)u[i];
+                float acc = 0.0f;
+                if (g_mutation == 6)
+                    for (int64_t n = 0; n < N; ++n) acc += (float)Csel[bc + n] * h[n];
+                for (int64_t n = 0; n < N; ++n) {
+                    const float an = (float)a_at_d(A, ch, n, d, N);
+                    const float decay = (g_mutation == 1) ? expf(-dt * an) : expf(dt * an);
+                    const float input = (g_mutation == 8) ? (float)Bsel[bc + n] * uv
+                                                           : dt * (float)Bsel[bc + n] * uv;
+                    h[n] = decay * h[n] + input;
+                }
+                if (g_mutation != 6)
+                    for (int64_t n = 0; n < N; ++n) acc += (float)Csel[bc + n] * h[n];
+                float yv = acc;
+                if (D && g_mutation != 2) yv += (float)D[ch] * uv;
+                if (z) yv *= gate_f((float)z[i]);
+                y[i] = (double)yv;
+            }
+            if (last_state)
+                for (int64_t n = 0; n < N; ++n)
+                    last_state[(b * d + ch) * N + n] = (double)h[n];
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * One decode step (the streaming "step" of the tutorial pages: one token in,
+ * state carried), double precision.  state [batch, d, N] is read and
+ * overwritten; u, delta, z, y are [batch, d]; B, C are [batch, N].
+ * The arithmetic is the body of the forward loop for a single t.
+ * ------------------------------------------------------------------------- */
+int ss_oracle_step_f64(double* state, const double* u, const double* delta,
+                       const double* delta_bias, const double* A, const double* B,
+                       const double* C, const double* D, const double* z, double* y,
+                       int64_t batch, int64_t d, int64_t N, int softplus)
+{
+    if (N < 1 || batch < 0 || d < 0) return -1;
+#pragma omp parallel for collapse(2)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t ch = 0; ch < d; ++ch) {
+            const int64_t i = b * d + ch;
+            const double dt = delta_d(delta[i], delta_bias, ch, softplus);
+            const double uv = u[i];
+            double* h = state + i * N;
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                const double an = a_at_d(A, ch, n, d, N);
+                h[n] = exp(dt * an) * h[n] + dt * B[b * N + n] * uv;
+                acc += C[b * N + n] * h[n];
+            }
+            double yv = acc;
+            if (D) yv += D[ch] * uv;
+            if (z) yv *= gate_d(z[i]);
+            y[i] = yv;
+        }
+    }
+    return 0;
+}
+
+/* Decode step with a float state and float arithmetic. */
+int ss_oracle_step_f32(double* state, const double* u, const double* delta,
+                       const double* delta_bias, const double* A, const double* B,
+                       const double* C, const double* D, const double* z, double* y,
+                       int64_t batch, int64_t d, int64_t N, int softplus)
+{
+    if (N < 1 || batch < 0 || d < 0) return -1;
+#pragma omp parallel for collapse(2)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t ch = 0; ch < d; ++ch) {
+            const int64_t i = b * d + ch;
+            const float dt = delta_f((float)delta[i], delta_bias, ch, softplus);
+            const float uv = (float)u[i];
+            double* h = state + i * N;
+            float acc = 0.0f;
+            for (int64_t n = 0; n < N; ++n) {
+                const float an = (float)a_at_d(A, ch, n, d, N);
+                const float hn = expf(dt * an) * (float)h[n] + dt * (float)B[b * N + n] * uv;
+                h[n] = (double)hn;
+                acc += (float)C[b * N + n] * hn;
+            }
+            float yv = acc;
+            if (D) yv += (float)D[ch] * uv;
+            if (z) yv *= gate_f((float)z[i]);
+            y[i] = (double)yv;
+        }
+    }
+    return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Chunked forward scan, double precision: the time-parallel re-association
+ * that a GPU uses, written out plainly so that "chunked = sequential" can be
+ * checked on the CPU.
+ *
+ * The recurrence h_t = a_t ⊙ h_{t-1} + b_t is linear, so a chunk of steps acts
+ * on its entry state as h_end = P ⊙ h_entry + h_loc, where P = Π a_t over the
+ * chunk and h_loc is the chunk's end state when entered from zero.  Pairs
+ * compose by (P, h) ∘ (P', h') = (P·P', P'·h + h').  The "hardware-aware
+ * parallel algorithm" of the Mamba tutorial (discosf.com, §2.3) and the
+ * single-launch scan of the deep-dive article (§2.2, second cut) rely on
+ * exactly this associativity.
+ *
+ * Steps, per (b, ch):
+ *   1. every chunk is scanned from a zero state, giving y_loc, P, h_loc;
+ *   2. entry states are combined left to right: h0[0] = 0,
+ *      h0[c+1] = P[c] ⊙ h0[c] + h_loc[c];
+ *   3. each output gets the entry state's contribution:
+ *      y_t = (y_loc,t + Σ_n C_t,n · Π_{s<=t in chunk} a_s,n · h0_n + D u_t) · gate.
+ * The prefix product in step 3 is accumulated step by step.  The gate and
+ * the D term are applied once, after the correction.
+ * ------------------------------------------------------------------------- */
+int ss_oracle_fwd_chunked_f64(const double* u, const double* delta, const double* delta_bias,
+                              const double* A, const double* B, const double* C,
+                              const double* D, const double* z, double* y, double* last_state,
+                              int64_t batch, int64_t L, int64_t d, int64_t N, int softplus,
+                              int64_t chunk)
+{
+    if (N < 1 || N > 256 || chunk < 1 || batch < 0 || L < 0 || d < 0) return -1;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t ch = 0; ch < d; ++ch) {
+            double h0[256];                      /* entry state of the current chunk */
+            for (int64_t n = 0; n < N; ++n) h0[n] = 0.0;
+            for (int64_t c0 = 0; c0 < L; c0 += chunk) {
+                const int64_t c1 = (c0 + chunk < L) ? c0 + chunk : L;
+                double hl[256], P[256];
+                for (int64_t n = 0; n < N; ++n) { hl[n] = 0.0; P[n] = 1.0; }
+                for (int64_t t = c0; t < c1; ++t) {
+                    const int64_t i = (b * L + t) * d + ch;
+                    const int64_t bc = (b * L + t) * N;
+                    const double dt = delta_d(delta[i], delta_bias, ch, softplus);
+                    const double uv = u[i];
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) {
+                        const double a = exp(dt * a_at_d(A, ch, n, d, N));
+                        hl[n] = a * hl[n] + dt * B[bc + n] * uv;  /* local state  */
+                        P[n] *= a;                                /* prefix decay */
+                        acc += C[bc + n] * (hl[n] + P[n] * h0[n]);
+                    }
+                    double yv = acc;
+                    if (D) yv += D[ch] * uv;
+                    if (z) yv *= gate_d(z[i]);
+                    y[i] = yv;
+                }
+                /* combine: entry state of the next chunk */
+                for (int64_t n = 0; n < N; ++n) h0[n] = P[n] * h0[n] + hl[n];
+            }
+            if (last_state)
+                for (int64_t n = 0; n < N; ++n) last_state[(b * d + ch) * N + n] = h0[n];
+        }
+    }
+    return 0;
+}

@@ -1,0 +1,144 @@
+"""Seeded random draws for the selective-scan workloads (torch generators).
+
+Every tensor is drawn from a torch.Generator seeded from (seed, tensor tag),
+so the same call on the same device type gives the same values.  Large
+workloads are drawn directly on the GPU in slices (no host staging); the CPU
+oracle then receives the exact values of a sample of channels copied back.
+"""
+import math
+
+import numpy as np
+import torch
+
+_TAGS = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "bias": 6, "D": 7, "A": 8, "state": 9}
+_SLICE = 1 << 26  # elements drawn per slice when filling a large tensor
+
+
+def _gen(device, seed, tag):
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 1000003 + _TAGS[tag])
+    return g
+
+
+def _normal(shape, std, dtype, device, seed, tag):
+    """N(0, std^2) rounded once to dtype, drawn in fp32 slices."""
+    g = _gen(device, seed, tag)
+    out = torch.empty(shape, dtype=dtype, device=device)
+    flat = out.view(-1)
+    n = flat.numel()
+    for s in range(0, n, _SLICE):
+        e = min(n, s + _SLICE)
+        tmp = torch.randn(e - s, generator=g, device=device, dtype=torch.float32)
+        if std != 1.0:
+            tmp.mul_(std)
+        flat[s:e].copy_(tmp)
+    return out
+
+
+def _torch_dtype(name):
+    return {"fp32": torch.float32, "bf16": torch.bfloat16}[name]
+
+
+def delta_bias_init(d, seed, device="cpu", lo=1e-3, hi=1e-1):
+    """bias = softplus^-1(Δ0) with Δ0 log-uniform in [lo, hi]; fp32 [d]."""
+    g = _gen(device, seed, "bias")
+    r = torch.rand(d, generator=g, device=device, dtype=torch.float64)
+    d0 = torch.exp(math.log(lo) + r * (math.log(hi) - math.log(lo)))
+    return torch.log(torch.expm1(d0)).to(torch.float32)
+
+
+def structured_A(d, N, device="cpu"):
+    """A[d, n] = -(n + 1), fp32 [d, N]."""
+    return (-(torch.arange(N, dtype=torch.float32, device=device) + 1.0)).repeat(d, 1).contiguous()
+
+
+def general_A(d, N, seed, device="cpu"):
+    """A[d, n] = -(n + 1) * (1 + 0.25 * U[0,1)): negative, but off the
+    a_d * (n + 1) ladder, so the general-A code path is exercised."""
+    g = _gen(device, seed, "A")
+    r = torch.rand(d, N, generator=g, device=device, dtype=torch.float32)
+    return (structured_A(d, N, device) * (1.0 + 0.25 * r)).contiguous()
+
+
+def fwd_inputs(batch, seqlen, d_inner, d_state=16, dtype="bf16", seed=0, device="cpu",
+               gate=True, D_kind="ones", bias=True, A_kind="structured", delta_std=0.5):
+    """Inputs of one ss_fwd call as a dict of torch tensors on `device`.
+
+    u, delta, z : [batch, seqlen, d_inner] in `dtype`
+    B, C        : [batch, seqlen, d_state] in `dtype`
+    A           : [d_inner, d_state] fp32; D, delta_bias : [d_inner] fp32
+    """
+    dt = _torch_dtype(dtype)
+    shp = (batch, seqlen, d_inner)
+    out = {
+        "u": _normal(shp, 1.0, dt, device, seed, "u"),
+        "delta": _normal(shp, delta_std, dt, device, seed, "delta"),
+        "z": _normal(shp, 1.0, dt, device, seed, "z") if gate else None,
+        "B": _normal((batch, seqlen, d_state), 1.0, dt, device, seed, "B"),
+        "C": _normal((batch, seqlen, d_state), 1.0, dt, device, seed, "C"),
+    }
+    out["A"] = (structured_A(d_inner, d_state, device) if A_kind == "structured"
+                else general_A(d_inner, d_state, seed, device))
+    if D_kind == "ones":
+        out["D"] = torch.ones(d_inner, dtype=torch.float32, device=device)
+    elif D_kind == "normal":
+        out["D"] = _normal((d_inner,), 1.0, torch.float32, device, seed, "D")
+    else:
+        out["D"] = None
+    out["delta_bias"] = delta_bias_init(d_inner, seed, "cpu").to(device) if bias else None
+    return out
+
+
+def step_inputs(batch, d_inner, d_state=16, dtype="bf16", seed=0, device="cpu", gate=True,
+                bias=True, A_kind="structured"):
+    """One decode step's inputs: u, delta, z [batch, d_inner]; B, C [batch, d_state];
+    A, D, delta_bias as in fwd_inputs; state [batch, d_inner, d_state] fp32 ~ N(0, 1)."""
+    dt = _torch_dtype(dtype)
+    out = {
+        "u": _normal((batch, d_inner), 1.0, dt, device, seed, "u"),
+        "delta": _normal((batch, d_inner), 0.5, dt, device, seed, "delta"),
+        "z": _normal((batch, d_inner), 1.0, dt, device, seed, "z") if gate else None,
+        "B": _normal((batch, d_state), 1.0, dt, device, seed, "B"),
+        "C": _normal((batch, d_state), 1.0, dt, device, seed, "C"),
+        "state": _normal((batch, d_inner, d_state), 1.0, torch.float32, device, seed, "state"),
+    }
+    out["A"] = (structured_A(d_inner, d_state, device) if A_kind == "structured"
+                else general_A(d_inner, d_state, seed, device))
+    out["D"] = torch.ones(d_inner, dtype=torch.float32, device=device)
+    out["delta_bias"] = delta_bias_init(d_inner, seed, "cpu").to(device) if bias else None
+    return out
+
+
+def step_sequence_inputs(steps, batch, d_inner, d_state=16, dtype="bf16", seed=0,
+                         device="cpu", gate=True):
+    """Per-step inputs for `steps` successive decode steps, stacked on a leading
+    axis: u, delta, z [steps, batch, d_inner]; B, C [steps, batch, d_state]."""
+    dt = _torch_dtype(dtype)
+    return {
+        "u": _normal((steps, batch, d_inner), 1.0, dt, device, seed, "u"),
+        "delta": _normal((steps, batch, d_inner), 0.5, dt, device, seed, "delta"),
+        "z": _normal((steps, batch, d_inner), 1.0, dt, device, seed, "z") if gate else None,
+        "B": _normal((steps, batch, d_state), 1.0, dt, device, seed, "B"),
+        "C": _normal((steps, batch, d_state), 1.0, dt, device, seed, "C"),
+    }
+
+
+def to_f64(t):
+    """Exact float64 numpy copy of a tensor (None passes through)."""
+    if t is None:
+        return None
+    return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def sample_channels(batch, d_inner, count, seed):
+    """A seeded sample of distinct (b, channel) pairs, always including the
+    first and last channel of the first and last batch entry."""
+    rng = np.random.default_rng(seed + 777)
+    total = batch * d_inner
+    count = min(count, total)
+    picks = set([0, total - 1, d_inner - 1, (batch - 1) * d_inner])
+    picks = set(p for p in picks if 0 <= p < total)
+    while len(picks) < count:
+        picks.add(int(rng.integers(0, total)))
+    flat = sorted(picks)[:max(count, len(picks))]
+    return [(p // d_inner, p % d_inner) for p in flat]
