@@ -1,0 +1,465 @@
+#!/usr/bin/env python
+"""Benchmark of the selective-scan forward pass (and the decode step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload mamba2p8b] [--no-extras] [--no-cpu-baseline]
+
+One step = one ss_fwd call over the whole workload (Δ softplus, discretise,
+recurrence, readout + skip, gate, final state: every step of the path), with
+inputs resident in HBM.  The default workload is the Mamba-2.8B-shaped layer
+(batch 4, L 8192, d_inner 5120, N 16, bf16 I/O, fp32 state).  Its inputs
+(1.34 GB) are larger than the 126 MB L2, so no flush is needed between steps.
+
+Metric: effective HBM bandwidth = compulsory bytes of the step / step time
+(u, Δ_raw, z read and y written once each, B, C, A, D, bias read, final state
+written), in GB/s.  Under torchrun every rank runs its own copy of the
+workload (independent problems, no data-path collective: weak scaling); the
+value is all ranks' bytes over the slowest rank's time.
+
+Rank 0 prints ONE JSON line.  `--impl reference` times the CPU oracle (the
+plain sequential loop the GPU path is checked against) on a bounded sample of
+the same workload instead.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "selective-scan fwd effective HBM GB/s (% of B200 peak); decode steps/s"
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["selective_state_space_37_b200/csrc/fwd.cuh",
+                  "selective_state_space_37_b200/csrc/common.cuh",
+                  "selective_state_space_37_b200/csrc/selscan.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mamba2p8b")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch from the committed ncu summary, when it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"ss_fwd_kernel_{workload}.md")
+    try:
+        src, val = None, None
+        with open(path) as f:
+            for line in f:
+                if line.startswith("source_sha:"):
+                    src = line.split(":", 1)[1].strip()
+                if line.startswith("dram_bytes_per_launch:"):
+                    val = float(line.split(":", 1)[1].strip())
+        if src == kernel_source_hash() and val:
+            return val
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons via NVML in a background thread."""
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.002):
+        self.ok = False
+        self.samples = []
+        self.reasons = set()
+        self.period = period
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._stop = threading.Event()
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------- our arm
+def fwd_call(ss, inp, y, st, ws, stream):
+    return ss.ss_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"], z=inp["z"],
+                     delta_bias=inp["delta_bias"], y=y, last_state=st, workspace=ws, stream=stream)
+
+
+def time_fwd(ss, torch, cfg, device, steps, warmup, seed_offset=0, dist=None, clocks=None):
+    from ss_inputs import fwd_inputs
+    inp = fwd_inputs(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.d_state, cfg.dtype,
+                     cfg.seed + seed_offset, device, gate=cfg.gate, D_kind=cfg.D_kind)
+    y = torch.empty_like(inp["u"])
+    st = torch.empty((cfg.batch, cfg.d_inner, cfg.d_state), dtype=torch.float32, device=device)
+    nbytes = ss.fwd_workspace_bytes(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.dtype == "bf16")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        fwd_call(ss, inp, y, st, ws, stream)
+    torch.cuda.synchronize(device)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    ctx = clocks if clocks is not None else _Null()
+    with ctx:
+        e0.record(stream)
+        for _ in range(steps):
+            fwd_call(ss, inp, y, st, ws, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1)
+    status = ss.ss_check(ws, stream=stream)
+    if status != 0:
+        raise RuntimeError(f"device status {ss.status_string(status)}")
+    return ms, inp, y, st, ws
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def time_e2e(ss, torch, cfg, device, inp, steps):
+    """Public API with host buffers: pinned host inputs -> device, ss_fwd,
+    y -> pinned host, all inside the timed region, every step."""
+    names = ["u", "delta", "z", "B", "C"]
+    host = {k: torch.empty(inp[k].shape, dtype=inp[k].dtype, pin_memory=True) for k in names}
+    for k in names:
+        host[k].copy_(inp[k])
+    dev = {k: torch.empty_like(inp[k]) for k in names}
+    y_dev = torch.empty_like(inp["u"])
+    y_host = torch.empty(inp["u"].shape, dtype=inp["u"].dtype, pin_memory=True)
+    nbytes = ss.fwd_workspace_bytes(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.dtype == "bf16")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    h2d = sum(host[k].numel() * host[k].element_size() for k in names)
+    d2h = y_host.numel() * y_host.element_size()
+
+    def one():
+        for k in names:
+            dev[k].copy_(host[k], non_blocking=True)
+        ss.ss_fwd(dev["u"], dev["delta"], inp["A"], dev["B"], dev["C"], D=inp["D"], z=dev["z"],
+                  delta_bias=inp["delta_bias"], y=y_dev, last_state=None, return_last_state=False,
+                  workspace=ws, stream=stream)
+        y_host.copy_(y_dev, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    return ms, h2d, d2h
+
+
+def time_decode(ss, torch, device, steps_total=1000, reps=3):
+    """The decode workload: 1000 successive ss_step calls captured in one CUDA
+    graph, replayed `reps` times after warm-up; returns (ms per step, bytes per step)."""
+    from ss_inputs import CONFIGS, step_inputs, step_sequence_inputs
+    c = CONFIGS["decode"]
+    base = step_inputs(c.batch, c.d_inner, c.d_state, c.dtype, c.seed, device, gate=c.gate)
+    seq = step_sequence_inputs(steps_total, c.batch, c.d_inner, c.d_state, c.dtype, c.seed + 1,
+                               device, gate=c.gate)
+    y = torch.empty((c.batch, c.d_inner), dtype=torch.bfloat16, device=device)
+    state = base["state"]
+
+    def run_all():
+        for t in range(steps_total):
+            ss.ss_step(state, seq["u"][t], seq["delta"][t], base["A"], seq["B"][t], seq["C"][t],
+                       D=base["D"], z=seq["z"][t], delta_bias=base["delta_bias"], y=y)
+
+    s = torch.cuda.Stream(device)
+    s.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(s):
+        run_all()
+    torch.cuda.current_stream(device).wait_stream(s)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run_all()
+    g.replay()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / (reps * steps_total)
+    del g
+    return ms, c.compulsory_bytes_per_step()
+
+
+def cpu_baseline(cfg, budget_s=10.0):
+    """The oracle (fp32 state, as it stands) on a bounded sample of the
+    workload: the first k channels of batch entry 0 over the full sequence."""
+    import numpy as np
+
+    import oracle
+    from ss_inputs import fwd_inputs, to_f64
+    cores = oracle.max_threads()
+    L = cfg.seqlen
+
+    def run(k):
+        inp = fwd_inputs(1, L, k, cfg.d_state, cfg.dtype, cfg.seed, "cpu", gate=cfg.gate,
+                         D_kind=cfg.D_kind)
+        args = [to_f64(inp[n]) for n in ("u", "delta", "A", "B", "C")]
+        t = time.perf_counter()
+        oracle.fwd(*args, D=to_f64(inp["D"]), z=to_f64(inp["z"]),
+                   delta_bias=to_f64(inp["delta_bias"]), precision="f32")
+        return time.perf_counter() - t
+
+    k0 = max(cores, 8)
+    t0 = run(k0)
+    k = int(min(cfg.d_inner, max(k0, k0 * budget_s / max(t0, 1e-6))))
+    k = max(cores, (k // cores) * cores) if k >= cores else k
+    t = run(k)
+    chts_per_s = L * k / t
+    bytes_per_chts = cfg.compulsory_bytes() / cfg.ch_ts
+    return {"value": chts_per_s * bytes_per_chts / 1e9, "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "sample": f"{k} channels x {L} steps of batch entry 0 ({L * k} channel-timesteps, "
+                      f"{t:.1f} s), fp32-state oracle; effective bytes scaled per channel-timestep",
+            "ch_ts_per_s": chts_per_s}
+
+
+def run_ours(args):
+    import torch
+
+    import selective_state_space_37_b200 as ss
+    from ss_inputs import CONFIGS
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=device)
+        dist = tdist
+    ss.lib()
+    cfg = CONFIGS[args.workload]
+    hbm, peak_kind = peaks()
+    clocks = ClockSampler(local)
+    ms, inp, y, st, ws = time_fwd(ss, torch, cfg, device, args.steps, args.warmup,
+                                  seed_offset=1000 * rank, dist=dist, clocks=clocks)
+    if dist is not None:
+        t = torch.tensor([ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    step_ms = ms / args.steps
+    per_gpu_bytes = cfg.compulsory_bytes()
+    value = world * per_gpu_bytes * args.steps / (ms * 1e-3) / 1e9
+    achieved = per_gpu_bytes / (step_ms * 1e-3) / 1e9
+
+    e2e = None
+    if args.e2e_steps > 0:
+        e_ms, h2d, d2h = time_e2e(ss, torch, cfg, device, inp, args.e2e_steps)
+        if dist is not None:
+            t = torch.tensor([e_ms], device=device)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * per_gpu_bytes / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e_ms}
+    del inp, y, st, ws
+    torch.cuda.empty_cache()
+
+    extras = {}
+    if not args.no_extras and world == 1:
+        for name in ("mamba130m", "million"):
+            c = CONFIGS[name]
+            steps = 20 if name == "mamba130m" else 3
+            m, i2, y2, s2, w2 = time_fwd(ss, torch, c, device, steps, 2)
+            sms = m / steps
+            gbs = c.compulsory_bytes() / (sms * 1e-3) / 1e9
+            extras[name] = {"ms_per_step": sms, "GB_s": gbs, "frac_of_hbm": gbs / hbm,
+                            "ch_ts_per_s": c.ch_ts / (sms * 1e-3),
+                            "chunk_len": ss.fwd_chunk_len(c.batch, c.seqlen, c.d_inner)}
+            del i2, y2, s2, w2
+            torch.cuda.empty_cache()
+        dms, dbytes = time_decode(ss, torch, device)
+        extras["decode"] = {"ms_per_step": dms, "steps_per_s": 1e3 / dms,
+                            "GB_s": dbytes / (dms * 1e-3) / 1e9,
+                            "frac_of_hbm": dbytes / (dms * 1e-3) / 1e9 / hbm,
+                            "note": "1000 ss_step calls in one CUDA graph, batch 256, d_inner 5120"}
+        torch.cuda.empty_cache()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg)
+
+    if rank == 0:
+        out = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "description": cfg.description,
+                       "batch": cfg.batch, "seq_len": cfg.seqlen, "d_inner": cfg.d_inner,
+                       "d_state": cfg.d_state, "io_dtype": cfg.dtype, "state_dtype": "fp32",
+                       "gate": cfg.gate, "parallelism": f"independent replica per GPU x{world}",
+                       "chunk_len": ss.fwd_chunk_len(cfg.batch, cfg.seqlen, cfg.d_inner),
+                       "l2": "inputs (%.2f GB) larger than the 126 MB L2; no flush"
+                             % (cfg.compulsory_bytes() / 1e9),
+                       "compulsory_bytes_per_step": per_gpu_bytes},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": profiled_traffic(cfg.name),
+                         "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "ss_fwd_kernel"},
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+            "ch_ts_per_s": world * cfg.ch_ts / (step_ms * 1e-3),
+            "extras": extras or None,
+        }
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from ss_inputs import CONFIGS, fwd_inputs, to_f64
+    cfg = CONFIGS[args.workload]
+    cores = oracle.max_threads()
+    L = cfg.seqlen
+    # size one step to about one second of oracle work
+    probe_k = max(cores, 8)
+    inp = fwd_inputs(1, L, probe_k, cfg.d_state, cfg.dtype, cfg.seed, "cpu", gate=cfg.gate,
+                     D_kind=cfg.D_kind)
+    arrs = {n: to_f64(inp[n]) for n in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+
+    def step(a):
+        oracle.fwd(a["u"], a["delta"], a["A"], a["B"], a["C"], D=a["D"], z=a["z"],
+                   delta_bias=a["delta_bias"], precision="f32")
+
+    t = time.perf_counter()
+    step(arrs)
+    t_probe = time.perf_counter() - t
+    k = int(min(cfg.d_inner, max(probe_k, probe_k * 1.0 / max(t_probe, 1e-6))))
+    inp = fwd_inputs(1, L, k, cfg.d_state, cfg.dtype, cfg.seed, "cpu", gate=cfg.gate,
+                     D_kind=cfg.D_kind)
+    arrs = {n: to_f64(inp[n]) for n in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+    for _ in range(args.warmup):
+        step(arrs)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step(arrs)
+    el = time.perf_counter() - t
+    bytes_per_chts = cfg.compulsory_bytes() / cfg.ch_ts
+    value = L * k * args.steps * bytes_per_chts / el / 1e9
+    sample = (f"{k} channels x {L} steps of batch entry 0 per step ({L * k} channel-timesteps), "
+              f"fp32-state oracle; effective bytes scaled per channel-timestep")
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+           "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+           "config": {"workload": cfg.name, "description": cfg.description, "batch": cfg.batch,
+                      "seq_len": cfg.seqlen, "d_inner": cfg.d_inner, "d_state": cfg.d_state,
+                      "io_dtype": cfg.dtype, "state_dtype": "fp32", "gate": cfg.gate},
+           "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample, "value": value,
+                            "unit": "GB/s"},
+           "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0},
+           "gpu_launches": 0}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

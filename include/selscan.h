@@ -1,0 +1,165 @@
+/*
+ * selscan.h -- C ABI of libselscan, the B200 (sm_100a) selective-scan library.
+ *
+ * Two operations, both from the selective state-space model of Mamba:
+ *
+ *   ss_fwd   the forward scan over a whole sequence ("Algorithm 2" selective
+ *            SSM of the mamba README, Usage > Selective SSM; equations of
+ *            "Understanding Mamba and Selective State Space Models (SSMs)",
+ *            §2.2 first and second cut, §3.1, §4.3):
+ *              Δ_t   = softplus(Δraw_t + bias)                  (§2.2 closing tip)
+ *              h_t,n = exp(Δ_t A_n) h_{t-1},n + Δ_t B_t,n u_t   (§2.2 first cut)
+ *              y_t   = (Σ_n C_t,n h_t,n + D u_t) · z_t σ(z_t)    (§3.1, §2.1; gate optional)
+ *            with h_{-1} = 0 (§2.2 second cut), per channel, A diagonal (§4.3).
+ *   ss_step  one decode step on a carried state: the same body for a single
+ *            token, reading and overwriting the state (the streaming "step"
+ *            function of the Mamba tutorial, §"state management", and the
+ *            "constant memory per token" property of the model-architecture
+ *            page).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every tensor pointer is a DEVICE pointer (cudaMalloc / torch CUDA
+ *   memory) on the current device, contiguous row-major, 16-byte aligned.
+ *   The caller owns all buffers; the library allocates nothing.
+ * - Element type of u, delta, z, B, C and y: bf16 when SS_BF16 is set in
+ *   `flags`, else fp32.  A, D, delta_bias and the states are always fp32.
+ * - Layouts: u, delta, z, y [batch, seqlen, d_inner] (token-major, channels
+ *   contiguous); B, C [batch, seqlen, d_state] (one group shared by all
+ *   channels); A [d_inner, d_state]; D, delta_bias [d_inner];
+ *   last_state / state [batch, d_inner, d_state].
+ * - d_state must be 16 (SS_ERR_UNSUPPORTED otherwise).
+ * - Calls are asynchronous on launch->stream.  A device-side failure (a
+ *   cross-chunk wait that ran out) is recorded in the workspace and reported
+ *   by ss_check(), or by the call itself when SS_SYNC_CHECK is set.
+ * - Invalid arguments return SS_ERR_INVALID_ARG and launch nothing.
+ *   Calls never trap or abort.
+ */
+#ifndef SELSCAN_H
+#define SELSCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+/* Exported symbols keep default visibility even when the library is built
+ * with -fvisibility=hidden. */
+#if defined(__GNUC__)
+#define SS_API __attribute__((visibility("default")))
+#else
+#define SS_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Problem sizes.  seqlen is ignored by ss_step. */
+typedef struct ss_dims {
+    int64_t batch;
+    int64_t seqlen;
+    int64_t d_inner;
+    int64_t d_state;
+} ss_dims;
+
+/* Launch context.
+ *   stream          cudaStream_t to launch on (NULL: the legacy default stream).
+ *   workspace       device scratch of at least ss_fwd_workspace_bytes() bytes
+ *                   (never less than 256: it always holds the device status
+ *                   word), 16-byte aligned.  ss_fwd overwrites it on every
+ *                   call; calls that overlap in time must not share one.
+ *                   ss_step does not use it.
+ *   workspace_bytes its size.
+ *   timeout_iters   bound on the polls of one cross-chunk wait (0: library
+ *                   default, about one second).  When it runs out the call
+ *                   records SS_ERR_TIMEOUT and finishes without hanging.
+ *   chunk_len       timesteps per time chunk; 0 lets the library choose.  Any
+ *                   positive value is accepted (it is rounded up to a multiple
+ *                   of the 32-step tile); results agree up to rounding. */
+typedef struct ss_launch {
+    void*    stream;
+    void*    workspace;
+    size_t   workspace_bytes;
+    uint32_t timeout_iters;
+    int32_t  chunk_len;
+} ss_launch;
+
+/* Status codes. */
+enum {
+    SS_OK              = 0,
+    SS_ERR_INVALID_ARG = -1,   /* NULL required pointer, negative size, misalignment, overflow */
+    SS_ERR_UNSUPPORTED = -2,   /* d_state != 16 */
+    SS_ERR_CUDA        = -3,   /* a CUDA runtime call or launch failed */
+    SS_ERR_TIMEOUT     = -4,   /* a bounded cross-chunk wait ran out (results invalid) */
+    SS_ERR_WORKSPACE   = -5    /* workspace missing or smaller than required */
+};
+
+/* Flags. */
+enum {
+    SS_BF16            = 1u << 0,  /* u, delta, z, B, C, y are bf16 (else fp32) */
+    SS_DELTA_SOFTPLUS  = 1u << 1,  /* Δ = softplus(delta + delta_bias); else Δ = delta + delta_bias */
+    SS_SYNC_CHECK      = 1u << 2,  /* synchronize the stream and return the device status */
+    SS_FORCE_GENERAL_A = 1u << 3,  /* skip the A[d,n] = a_d (n+1) fast path even when A has that form */
+    SS_TEST_DROP_CARRY = 1u << 30  /* TEST ONLY: the first chunk of batch 0, channel block 0 never
+                                      publishes its carry, so its successor's bounded wait runs out
+                                      (exercises SS_ERR_TIMEOUT without a hang) */
+};
+
+/* ss_fwd -- selective-scan forward pass over [batch, seqlen] tokens.
+ *   u          [batch, seqlen, d_inner]  input sequence (x_n of §2.2)
+ *   delta      [batch, seqlen, d_inner]  Δ before bias and softplus
+ *   delta_bias [d_inner] fp32 or NULL    added to delta before softplus
+ *   A          [d_inner, d_state] fp32   diagonal state matrix (negative reals)
+ *   B, C       [batch, seqlen, d_state]  input / output projections per token
+ *   D          [d_inner] fp32 or NULL    skip weight (NULL: no skip term)
+ *   z          [batch, seqlen, d_inner] or NULL   gate input (NULL: no gate)
+ *   y          [batch, seqlen, d_inner]  output, written in the I/O type
+ *   last_state [batch, d_inner, d_state] fp32 or NULL   h after the last token
+ * seqlen == 0 writes zeros to last_state; batch == 0 or d_inner == 0 is a no-op.
+ * Returns SS_OK or an error code (see above). */
+SS_API int ss_fwd(const void* u, const void* delta, const float* delta_bias, const float* A,
+           const void* B, const void* C, const float* D, const void* z, void* y,
+           float* last_state, uint32_t flags, const ss_dims* dims, const ss_launch* launch);
+
+/* ss_step -- one decode step: for every (b, channel) the state row is
+ * advanced by one token and y is produced, as ss_fwd would do for that token.
+ *   state      [batch, d_inner, d_state] fp32, read and overwritten in place
+ *   u, delta   [batch, d_inner]          this token's input and raw Δ
+ *   A          [d_inner, d_state] fp32
+ *   B, C       [batch, d_state]
+ *   D          [d_inner] fp32 or NULL
+ *   z          [batch, d_inner] or NULL
+ *   y          [batch, d_inner]          output
+ *   delta_bias [d_inner] fp32 or NULL
+ * dims->seqlen is ignored; launch->workspace is not used.  Returns SS_OK or
+ * an error code. */
+SS_API int ss_step(float* state, const void* u, const void* delta, const float* A, const void* B,
+            const void* C, const float* D, const void* z, void* y, const float* delta_bias,
+            uint32_t flags, const ss_dims* dims, const ss_launch* launch);
+
+/* Workspace bytes ss_fwd needs for these sizes, flags and chunk length
+ * (chunk_len 0: the library's own choice, the same one ss_fwd makes):
+ * 256 bytes of header without time chunking, plus per-chunk carry records
+ * (48 floats per (batch, chunk, channel)) and status words with it.
+ * 0 for sizes ss_fwd would reject. */
+SS_API size_t ss_fwd_workspace_bytes(const ss_dims* dims, uint32_t flags, int32_t chunk_len);
+
+/* Chunk length ss_fwd uses for these sizes when launch->chunk_len is 0
+ * (0 when the scan is not split in time). */
+SS_API int32_t ss_fwd_chunk_len(const ss_dims* dims, uint32_t flags);
+
+/* Synchronize launch->stream and return the device-side status recorded in
+ * launch->workspace by the last ss_fwd on it (SS_OK when there is no
+ * workspace), or SS_ERR_CUDA if the stream reports an error. */
+SS_API int ss_check(const ss_launch* launch);
+
+/* Human-readable name of a status code (static storage). */
+SS_API const char* ss_status_string(int status);
+
+/* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
+SS_API int ss_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SELSCAN_H */

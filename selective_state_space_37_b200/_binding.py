@@ -1,0 +1,244 @@
+"""ctypes binding of libselscan (the C ABI declared in include/selscan.h).
+
+Argument marshalling only: every step of the scan runs in the library's CUDA
+kernels.  PyTorch supplies device memory (tensors, the cached workspace) and
+the current stream.  There is no CPU fallback: if the library is missing or a
+call fails, an exception is raised.
+"""
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "csrc", "libselscan.so")
+
+SS_OK = 0
+SS_ERR_INVALID_ARG = -1
+SS_ERR_UNSUPPORTED = -2
+SS_ERR_CUDA = -3
+SS_ERR_TIMEOUT = -4
+SS_ERR_WORKSPACE = -5
+
+SS_BF16 = 1 << 0
+SS_DELTA_SOFTPLUS = 1 << 1
+SS_SYNC_CHECK = 1 << 2
+SS_FORCE_GENERAL_A = 1 << 3
+SS_TEST_DROP_CARRY = 1 << 30
+
+D_STATE = 16
+
+# Every symbol include/selscan.h declares.
+EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
+            "ss_status_string", "ss_version")
+
+
+class ss_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64),
+                ("d_inner", ctypes.c_int64), ("d_state", ctypes.c_int64)]
+
+
+class ss_launch(ctypes.Structure):
+    _fields_ = [("stream", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_size_t), ("timeout_iters", ctypes.c_uint32),
+                ("chunk_len", ctypes.c_int32)]
+
+
+class SelscanError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+_lib = None
+_lock = threading.Lock()
+
+
+def lib():
+    """The loaded library with argument types set (raises if not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libselscan.so not found at {LIB_PATH}; build it with "
+                "`python -m selective_state_space_37_b200.csrc.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, f32p = ctypes.c_void_p, ctypes.c_void_p
+        L.ss_fwd.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, vp, f32p, ctypes.c_uint32,
+                             ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch)]
+        L.ss_fwd.restype = ctypes.c_int
+        L.ss_step.argtypes = [f32p, vp, vp, f32p, vp, vp, f32p, vp, vp, f32p, ctypes.c_uint32,
+                              ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch)]
+        L.ss_step.restype = ctypes.c_int
+        L.ss_fwd_workspace_bytes.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32, ctypes.c_int32]
+        L.ss_fwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ss_fwd_chunk_len.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32]
+        L.ss_fwd_chunk_len.restype = ctypes.c_int32
+        L.ss_check.argtypes = [ctypes.POINTER(ss_launch)]
+        L.ss_check.restype = ctypes.c_int
+        L.ss_status_string.argtypes = [ctypes.c_int]
+        L.ss_status_string.restype = ctypes.c_char_p
+        L.ss_version.argtypes = []
+        L.ss_version.restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().ss_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _io_flag(t):
+    if t.dtype == torch.bfloat16:
+        return SS_BF16
+    if t.dtype == torch.float32:
+        return 0
+    raise TypeError(f"u/delta/z/B/C must be bfloat16 or float32, got {t.dtype}")
+
+
+def _check(t, name, shape, dtype, device):
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+_ws_cache = {}
+
+
+def workspace_for(nbytes, device, stream_handle):
+    """A cached device workspace of at least nbytes for (device, stream)."""
+    key = (device.index, int(stream_handle))
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _stream_handle(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def fwd_workspace_bytes(batch, seqlen, d_inner, bf16=True, chunk_len=0, d_state=D_STATE):
+    dims = ss_dims(batch, seqlen, d_inner, d_state)
+    return int(lib().ss_fwd_workspace_bytes(ctypes.byref(dims), SS_BF16 if bf16 else 0, int(chunk_len)))
+
+
+def fwd_chunk_len(batch, seqlen, d_inner, bf16=True, d_state=D_STATE):
+    dims = ss_dims(batch, seqlen, d_inner, d_state)
+    return int(lib().ss_fwd_chunk_len(ctypes.byref(dims), SS_BF16 if bf16 else 0))
+
+
+def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, y=None, last_state=None,
+           return_last_state=True, softplus=True, force_general_A=False, chunk_len=0,
+           timeout_iters=0, workspace=None, stream=None, sync_check=False, extra_flags=0):
+    """Selective-scan forward pass through libselscan's ss_fwd.
+
+    u, delta, z: [batch, L, d_inner]; B, C: [batch, L, 16] (bf16 or fp32, all the
+    same); A: [d_inner, 16] fp32; D, delta_bias: [d_inner] fp32 or None.
+    Returns (y, last_state); last_state is None when return_last_state is False
+    and none was passed in.
+    """
+    if u.dim() != 3:
+        raise ValueError("u must be [batch, L, d_inner]")
+    batch, L, d = u.shape
+    dev = u.device
+    if dev.type != "cuda":
+        raise ValueError("ss_fwd runs on CUDA tensors only")
+    io = u.dtype
+    for t, nm, shp in ((u, "u", (batch, L, d)), (delta, "delta", (batch, L, d)),
+                       (z, "z", (batch, L, d)), (B, "B", (batch, L, D_STATE)),
+                       (C, "C", (batch, L, D_STATE))):
+        _check(t, nm, shp, io, dev)
+    _check(A, "A", (d, D_STATE), torch.float32, dev)
+    _check(D, "D", (d,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (d,), torch.float32, dev)
+    if y is None:
+        y = torch.empty((batch, L, d), dtype=io, device=dev)
+    _check(y, "y", (batch, L, d), io, dev)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, d, D_STATE), dtype=torch.float32, device=dev)
+    _check(last_state, "last_state", (batch, d, D_STATE), torch.float32, dev)
+    flags = _io_flag(u) | (SS_DELTA_SOFTPLUS if softplus else 0) | int(extra_flags)
+    if force_general_A:
+        flags |= SS_FORCE_GENERAL_A
+    if sync_check:
+        flags |= SS_SYNC_CHECK
+    sh = _stream_handle(stream, dev)
+    dims = ss_dims(batch, L, d, D_STATE)
+    need = int(lib().ss_fwd_workspace_bytes(ctypes.byref(dims), flags, int(chunk_len)))
+    if workspace is None:
+        workspace = workspace_for(need, dev, sh)
+    launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                       int(timeout_iters), int(chunk_len))
+    rc = lib().ss_fwd(_ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                      _ptr(z), _ptr(y), _ptr(last_state), flags, ctypes.byref(dims),
+                      ctypes.byref(launch))
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_fwd")
+    return y, last_state
+
+
+def ss_check(workspace, stream=None, device=None):
+    """Synchronize and return the device status recorded in `workspace`."""
+    dev = workspace.device if device is None else device
+    sh = _stream_handle(stream, dev)
+    launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(), 0, 0)
+    return int(lib().ss_check(ctypes.byref(launch)))
+
+
+def ss_step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, *, y=None, softplus=True,
+            stream=None, sync_check=False):
+    """One decode step through libselscan's ss_step; `state` is updated in place.
+
+    state: [batch, d_inner, 16] fp32; u, delta, z: [batch, d_inner]; B, C: [batch, 16]
+    (bf16 or fp32); A: [d_inner, 16] fp32; D, delta_bias: [d_inner] fp32 or None.
+    Returns y [batch, d_inner].
+    """
+    if state.dim() != 3:
+        raise ValueError("state must be [batch, d_inner, 16]")
+    batch, d, _ = state.shape
+    dev = state.device
+    if dev.type != "cuda":
+        raise ValueError("ss_step runs on CUDA tensors only")
+    io = u.dtype
+    _check(state, "state", (batch, d, D_STATE), torch.float32, dev)
+    for t, nm, shp in ((u, "u", (batch, d)), (delta, "delta", (batch, d)), (z, "z", (batch, d)),
+                       (B, "B", (batch, D_STATE)), (C, "C", (batch, D_STATE))):
+        _check(t, nm, shp, io, dev)
+    _check(A, "A", (d, D_STATE), torch.float32, dev)
+    _check(D, "D", (d,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (d,), torch.float32, dev)
+    if y is None:
+        y = torch.empty((batch, d), dtype=io, device=dev)
+    _check(y, "y", (batch, d), io, dev)
+    flags = _io_flag(u) | (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
+    sh = _stream_handle(stream, dev)
+    dims = ss_dims(batch, 1, d, D_STATE)
+    launch = ss_launch(sh, None, 0, 0, 0)
+    rc = lib().ss_step(_ptr(state), _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                       _ptr(z), _ptr(y), _ptr(delta_bias), flags, ctypes.byref(dims),
+                       ctypes.byref(launch))
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_step")
+    return y

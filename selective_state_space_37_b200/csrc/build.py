@@ -1,0 +1,55 @@
+"""Build libselscan.so in-tree for sm_100a with nvcc (no GPU needed).
+
+    python -m selective_state_space_37_b200.csrc.build [--force] [--verbose]
+
+The CUDA runtime is linked statically so the library loads in any process
+(with or without torch) on a machine with a CUDA 12.9-capable driver.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(os.path.dirname(HERE))
+LIB = os.path.join(HERE, "libselscan.so")
+SOURCES = ["selscan.cu"]
+HEADERS = ["common.cuh", "fwd.cuh", "step.cuh"]
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+NVCC_FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
+    "--expt-relaxed-constexpr",
+    "-cudart", "static",
+]
+
+
+def _inputs():
+    files = [os.path.join(HERE, s) for s in SOURCES + HEADERS]
+    files.append(os.path.join(ROOT, "include", "selscan.h"))
+    files.append(os.path.abspath(__file__))
+    return files
+
+
+def up_to_date() -> bool:
+    if not os.path.exists(LIB):
+        return False
+    t = os.path.getmtime(LIB)
+    return all(os.path.getmtime(f) <= t for f in _inputs())
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and up_to_date():
+        return LIB
+    cmd = [NVCC, *NVCC_FLAGS]
+    if verbose:
+        cmd += ["-Xptxas", "-v"]
+    cmd += ["-shared", "-o", LIB + ".tmp"] + [os.path.join(HERE, s) for s in SOURCES]
+    subprocess.run(cmd, check=True)
+    os.replace(LIB + ".tmp", LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))

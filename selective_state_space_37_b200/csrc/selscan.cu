@@ -1,0 +1,299 @@
+// selscan.cu -- the C ABI of libselscan (declared in include/selscan.h):
+// argument validation, work decomposition, workspace layout, TMA descriptor
+// set-up and kernel launches.  No allocation happens here: every buffer,
+// including the workspace, belongs to the caller.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/selscan.h"
+#include "fwd.cuh"
+#include "step.cuh"
+
+using namespace selscan;
+
+namespace {
+
+constexpr int kVersion = 10000;             // 1.0.0
+constexpr size_t kHeaderBytes = 256;        // error word, ticket counter
+constexpr uint32_t kDefaultPolls = 1u << 21;
+constexpr uint64_t kTmaWaitNs = 2000000000ull;
+constexpr int kMaxDevices = 64;
+constexpr uint32_t kKnownFlags = SS_BF16 | SS_DELTA_SOFTPLUS | SS_SYNC_CHECK | SS_FORCE_GENERAL_A |
+                                 SS_TEST_DROP_CARRY;
+
+int sm_count_of_current_device() {
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+    if (dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < kMaxDevices) cache[dev] = n;
+    return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Resident CTAs per SM for the bf16 / fp32 forward kernels (shared memory bound).
+int ctas_per_sm(bool bf16) { return bf16 ? 2 : 1; }
+
+// Library choice of chunk length: enough (batch, chunk, channel-block) items
+// for two waves of resident CTAs; 0 = no time chunking.
+int32_t auto_chunk_len(const ss_dims* dims, uint32_t flags) {
+    const int64_t L = dims->seqlen;
+    if (L <= kTT) return 0;
+    const int64_t nblk = ceil_div(dims->d_inner, kCB);
+    const int64_t base = dims->batch * nblk;
+    if (base <= 0) return 0;
+    const int64_t slots = static_cast<int64_t>(sm_count_of_current_device()) * ctas_per_sm(flags & SS_BF16);
+    const int64_t nchunks = ceil_div(2 * slots, base);
+    if (nchunks <= 1) return 0;
+    int64_t chunk = ceil_div(ceil_div(L, nchunks), kTT) * kTT;
+    if (chunk >= L) return 0;
+    if (chunk > (1 << 30)) chunk = 1 << 30;
+    return static_cast<int32_t>(chunk);
+}
+
+struct Plan {
+    int64_t chunk_len;   // 0: unchunked
+    int64_t nchunks;
+    int64_t nblk;
+    size_t status_off, status_bytes, rec_off, rec_bytes, total;
+};
+
+Plan make_plan(const ss_dims* dims, uint32_t flags, int32_t chunk_req) {
+    Plan pl{};
+    const int64_t L = dims->seqlen;
+    pl.nblk = ceil_div(std::max<int64_t>(dims->d_inner, 1), kCB);
+    int64_t chunk = chunk_req > 0 ? ceil_div(chunk_req, kTT) * kTT : auto_chunk_len(dims, flags);
+    if (chunk <= 0 || chunk >= L) chunk = 0;
+    pl.chunk_len = chunk;
+    pl.nchunks = chunk > 0 ? ceil_div(L, chunk) : 1;
+    pl.status_off = kHeaderBytes;
+    if (pl.nchunks > 1) {
+        pl.status_bytes = static_cast<size_t>(dims->batch * pl.nchunks * pl.nblk) * sizeof(uint32_t);
+        pl.rec_off = (pl.status_off + pl.status_bytes + 255) / 256 * 256;
+        pl.rec_bytes = static_cast<size_t>(dims->batch * pl.nchunks * dims->d_inner) * kRec * sizeof(float);
+        pl.total = pl.rec_off + pl.rec_bytes;
+    } else {
+        pl.status_bytes = 0;
+        pl.rec_off = kHeaderBytes;
+        pl.rec_bytes = 0;
+        pl.total = kHeaderBytes;
+    }
+    return pl;
+}
+
+// ------------------------------------------------------------ TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a [batch, rows, inner] row-major tensor, box [1, box_rows, box_inner].
+bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint64_t rows, uint64_t batch,
+              uint32_t box_inner, uint32_t box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const uint64_t es = bf16 ? 2 : 4;
+    cuuint64_t dims[3] = {inner, rows, batch};
+    cuuint64_t strides[2] = {inner * es, rows * inner * es};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3,
+                           const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <typename IO, bool TMA, int STAGES>
+int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
+    auto kern = ss_fwd_kernel<IO, TMA, STAGES>;
+    const size_t smem = sizeof(FwdSmem<IO, STAGES>);
+    static bool attr_set[kMaxDevices] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+            return SS_ERR_CUDA;
+        if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
+    }
+    kern<<<static_cast<unsigned>(items), kNT, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
+    return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+int validate_dims(const ss_dims* dims, bool need_seqlen) {
+    if (!dims) return SS_ERR_INVALID_ARG;
+    if (dims->batch < 0 || dims->d_inner < 0 || dims->d_state <= 0) return SS_ERR_INVALID_ARG;
+    if (need_seqlen && dims->seqlen < 0) return SS_ERR_INVALID_ARG;
+    if (dims->d_state != kN) return SS_ERR_UNSUPPORTED;
+    const int64_t lim = int64_t(1) << 31;
+    if (dims->batch >= lim || dims->d_inner >= lim) return SS_ERR_INVALID_ARG;
+    if (need_seqlen) {
+        if (dims->seqlen >= lim) return SS_ERR_INVALID_ARG;
+        // batch * seqlen * d_inner elements must stay far below 2^62
+        const double elems = double(dims->batch) * double(dims->seqlen) * double(dims->d_inner);
+        if (elems > 4.0e18) return SS_ERR_INVALID_ARG;
+    }
+    return SS_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ss_status_string(int status) {
+    switch (status) {
+        case SS_OK: return "SS_OK";
+        case SS_ERR_INVALID_ARG: return "SS_ERR_INVALID_ARG";
+        case SS_ERR_UNSUPPORTED: return "SS_ERR_UNSUPPORTED";
+        case SS_ERR_CUDA: return "SS_ERR_CUDA";
+        case SS_ERR_TIMEOUT: return "SS_ERR_TIMEOUT";
+        case SS_ERR_WORKSPACE: return "SS_ERR_WORKSPACE";
+        default: return "SS_ERR_UNKNOWN";
+    }
+}
+
+int ss_version(void) { return kVersion; }
+
+int32_t ss_fwd_chunk_len(const ss_dims* dims, uint32_t flags) {
+    if (validate_dims(dims, true) != SS_OK) return 0;
+    return static_cast<int32_t>(make_plan(dims, flags, 0).chunk_len);
+}
+
+size_t ss_fwd_workspace_bytes(const ss_dims* dims, uint32_t flags, int32_t chunk_len) {
+    if (validate_dims(dims, true) != SS_OK) return 0;
+    return make_plan(dims, flags, chunk_len).total;
+}
+
+int ss_check(const ss_launch* launch) {
+    if (!launch) return SS_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
+    if (!launch->workspace || launch->workspace_bytes < sizeof(uint32_t)) return SS_OK;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, launch->workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return SS_ERR_CUDA;
+    return static_cast<int>(word);
+}
+
+int ss_fwd(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+           const void* C, const float* D, const void* z, void* y, float* last_state, uint32_t flags,
+           const ss_dims* dims, const ss_launch* launch) {
+    int rc = validate_dims(dims, true);
+    if (rc != SS_OK) return rc;
+    if (!launch || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, d = dims->d_inner;
+    if (batch == 0 || d == 0) return SS_OK;
+    cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
+    if (L == 0) {
+        if (last_state && !aligned16(last_state)) return SS_ERR_INVALID_ARG;
+        if (last_state &&
+            cudaMemsetAsync(last_state, 0, static_cast<size_t>(batch * d * kN) * sizeof(float), stream) !=
+                cudaSuccess)
+            return SS_ERR_CUDA;
+        return SS_OK;
+    }
+    if (!u || !delta || !A || !B || !C || !y) return SS_ERR_INVALID_ARG;
+    const void* ptrs[] = {u, delta, delta_bias, A, B, C, D, z, y, last_state};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
+
+    const bool bf16 = (flags & SS_BF16) != 0;
+    const Plan pl = make_plan(dims, flags, launch->chunk_len);
+    if (!launch->workspace || launch->workspace_bytes < pl.total || !aligned16(launch->workspace))
+        return SS_ERR_WORKSPACE;
+    const int64_t items = batch * pl.nchunks * pl.nblk;
+    if (items >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+
+    unsigned char* ws = static_cast<unsigned char*>(launch->workspace);
+    if (cudaMemsetAsync(ws, 0, pl.status_off + pl.status_bytes, stream) != cudaSuccess) return SS_ERR_CUDA;
+
+    FwdParams p{};
+    p.u = u; p.delta = delta; p.bias = delta_bias; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
+    p.y = y; p.last_state = last_state;
+    p.L = L; p.batch = static_cast<int>(batch); p.d = static_cast<int>(d);
+    p.chunk_len = static_cast<int>(pl.chunk_len > 0 ? pl.chunk_len : L);
+    p.nchunks = static_cast<int>(pl.nchunks); p.nblk = static_cast<int>(pl.nblk);
+    p.pflags = ((flags & SS_DELTA_SOFTPLUS) ? kPfSoftplus : 0u) | ((flags & SS_FORCE_GENERAL_A) ? kPfForceGeneral : 0u) |
+               ((flags & SS_TEST_DROP_CARRY) ? kPfTestDrop : 0u) | (z ? kPfHasZ : 0u) |
+               (delta_bias ? kPfHasBias : 0u) | (D ? kPfHasD : 0u);
+    p.hdr = reinterpret_cast<uint32_t*>(ws);
+    p.status = reinterpret_cast<uint32_t*>(ws + pl.status_off);
+    p.rec = reinterpret_cast<float*>(ws + pl.rec_off);
+    p.wait_ns = kTmaWaitNs;
+    p.poll_limit = launch->timeout_iters ? launch->timeout_iters : kDefaultPolls;
+
+    // TMA needs 16-byte row strides: d * element size a multiple of 16.
+    const bool tma = ((d * (bf16 ? 2 : 4)) % 16) == 0;
+    CUtensorMap maps[5];
+    std::memset(maps, 0, sizeof(maps));
+    if (tma) {
+        bool ok = make_map(&maps[0], u, bf16, d, L, batch, kCB, kTT) &&
+                  make_map(&maps[1], delta, bf16, d, L, batch, kCB, kTT) &&
+                  make_map(&maps[2], z ? z : u, bf16, d, L, batch, kCB, kTT) &&
+                  make_map(&maps[3], B, bf16, kN, L, batch, kN, kTT) &&
+                  make_map(&maps[4], C, bf16, kN, L, batch, kN, kTT);
+        if (!ok) return SS_ERR_CUDA;
+    }
+    if (bf16) {
+        rc = tma ? launch_fwd<__nv_bfloat16, true, 3>(p, items, maps, stream)
+                 : launch_fwd<__nv_bfloat16, false, 1>(p, items, maps, stream);
+    } else {
+        rc = tma ? launch_fwd<float, true, 2>(p, items, maps, stream)
+                 : launch_fwd<float, false, 1>(p, items, maps, stream);
+    }
+    if (rc != SS_OK) return rc;
+    if (flags & SS_SYNC_CHECK) return ss_check(launch);
+    return SS_OK;
+}
+
+int ss_step(float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
+            const float* D, const void* z, void* y, const float* delta_bias, uint32_t flags, const ss_dims* dims,
+            const ss_launch* launch) {
+    int rc = validate_dims(dims, false);
+    if (rc != SS_OK) return rc;
+    if (!launch || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, d = dims->d_inner;
+    if (batch == 0 || d == 0) return SS_OK;
+    if (!state || !u || !delta || !A || !B || !C || !y) return SS_ERR_INVALID_ARG;
+    const void* ptrs[] = {state, u, delta, A, B, C, D, z, y, delta_bias};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
+    const bool bf16 = (flags & SS_BF16) != 0;
+    StepParams p{};
+    p.state = state; p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z; p.y = y;
+    p.bias = delta_bias; p.channels = batch * d; p.d = static_cast<int>(d);
+    p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
+    const int64_t threads = p.channels * 4;
+    const int64_t blocks = ceil_div(threads, kStepThreads);
+    if (blocks >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
+    if (bf16)
+        ss_step_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+    else
+        ss_step_kernel<float><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+    if (flags & SS_SYNC_CHECK) {
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
+    }
+    return SS_OK;
+}
+
+}  // extern "C"
