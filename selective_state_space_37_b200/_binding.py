@@ -12,7 +12,9 @@ import threading
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "csrc", "libselscan.so")
+# SELSCAN_LIB selects another build of the same library (e.g. one compiled
+# with different tuning macros); default: the in-tree build.
+LIB_PATH = os.environ.get("SELSCAN_LIB") or os.path.join(_HERE, "csrc", "libselscan.so")
 
 SS_OK = 0
 SS_ERR_INVALID_ARG = -1

@@ -39,17 +39,22 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(f) <= t for f in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    cmd = [NVCC, *NVCC_FLAGS]
+def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()) -> str:
+    """Compile the library to `out`; `defines` are extra -D tuning macros
+    (SELSCAN_CTAS_PER_SM, SELSCAN_GROUP, SELSCAN_UNROLL_TILE)."""
+    if not force and out == LIB and not defines and up_to_date():
+        return out
+    cmd = [NVCC, *NVCC_FLAGS] + [f"-D{d}" for d in defines]
     if verbose:
         cmd += ["-Xptxas", "-v"]
-    cmd += ["-shared", "-o", LIB + ".tmp"] + [os.path.join(HERE, s) for s in SOURCES]
+    cmd += ["-shared", "-o", out + ".tmp"] + [os.path.join(HERE, s) for s in SOURCES]
     subprocess.run(cmd, check=True)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(out + ".tmp", out)
+    return out
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    defs = [a[2:] for a in sys.argv[1:] if a.startswith("-D")]
+    outs = [a.split("=", 1)[1] for a in sys.argv[1:] if a.startswith("--out=")]
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv,
+                out=outs[0] if outs else LIB, defines=defs))

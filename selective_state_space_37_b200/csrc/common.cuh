@@ -43,26 +43,68 @@ __device__ __forceinline__ float rcp_approx(float x) {
     return r;
 }
 
-// Fast path (bf16 I/O): softplus(x) = log(1 + e^x), identity above 20.
-// e^x by the hardware ex2; log1p(e) by a 3-term series for small e (truncation
-// below e^4/4 relative e^3/4 <= 7e-6 for e < 0.03) and by the hardware lg2 of
-// (1 + e) otherwise.  Relative error about 1e-5, far inside the bf16 bound.
-__device__ __forceinline__ float softplus_fast(float x) {
-    const float e = ex2_approx(x * kLog2e);
-    const float series = e * fmaf(e, fmaf(e, 0.33333334f, -0.5f), 1.0f);
-    const float viaLog = lg2_approx(1.0f + e) * kLn2;
-    const float r = (e < 0.03f) ? series : viaLog;
-    return (x > 20.0f) ? x : r;
+__device__ __forceinline__ float tanh_approx(float x) {
+    float r;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
+
+// Fast path, in base-2 units: given y2 = x * log2(e), returns
+// softplus(x) / ln 2 = log2(1 + 2^y2), identity above x = 20.  Hardware ex2 and
+// lg2; for very negative x the absolute error of softplus(x) stays below
+// ~1e-7 (1 + e^x rounds to 1), far inside the bf16 parity bound.
+__device__ __forceinline__ float softplus_log2_fast(float y2) {
+    const float l = lg2_approx(1.0f + ex2_approx(y2));
+    return (y2 > 20.0f * kLog2e) ? y2 : l;
+}
+
+// z * sigmoid(z) through tanh: sigmoid(z) = (1 + tanh(z/2)) / 2, so
+// z * sigmoid(z) = h + h * tanh(h) with h = z/2 (one hardware op).
+__device__ __forceinline__ float silu_tanh(float zv) {
+    const float h = 0.5f * zv;
+    return fmaf(h, tanh_approx(h), h);
+}
+
+// Branch-free choice: a where the mask is all ones, b where it is zero (one
+// logic op; keeps runtime options out of the control flow of unrolled loops).
+__device__ __forceinline__ float blend(uint32_t mask, float a, float b) {
+    return __uint_as_float((__float_as_uint(a) & mask) | (__float_as_uint(b) & ~mask));
+}
+
+// ------------------------------------------------------------ packed fp32x2
+// Two fp32 lanes in one 64-bit register pair; the sm_100 f32x2 instructions
+// do two lane operations per issue slot.
+typedef unsigned long long f32x2;
+__device__ __forceinline__ f32x2 pk2(float lo, float hi) {
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk2(f32x2 v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
+    f32x2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
+    f32x2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
 // Accurate path (fp32 I/O): the CUDA math library.
 __device__ __forceinline__ float softplus_accurate(float x) {
     return (x > 20.0f) ? x : log1pf(expf(x));
 }
 
-// z * sigmoid(z).
-__device__ __forceinline__ float silu_fast(float zv) {
-    return zv * rcp_approx(1.0f + ex2_approx(-zv * kLog2e));
-}
+// z * sigmoid(z), accurate path.
 __device__ __forceinline__ float silu_accurate(float zv) {
     return zv / (1.0f + expf(-zv));
 }
@@ -96,6 +138,11 @@ __device__ __forceinline__ void fence_mbar_init() {
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Orders this thread's generic-proxy global writes before later async-proxy
+// (TMA) reads of the same addresses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)

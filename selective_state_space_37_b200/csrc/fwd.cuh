@@ -9,42 +9,65 @@
 // starting from h = 0 (§2.2 second cut), A diagonal (§4.3).
 //
 // Work decomposition
-//   One CTA = one work item = (batch b, time chunk c, block of kCB channels);
-//   one thread owns one channel and keeps its kN fp32 states in registers for
-//   the whole chunk.  Tiles of kTT timesteps of u / Δraw / z ([kTT x kCB]) and
-//   of B / C ([kTT x kN], shared by every channel) are brought into shared
-//   memory by TMA (cp.async.bulk.tensor, no multicast) through a ring of
-//   STAGES buffers completed on mbarriers; B and C are widened to fp32 once
-//   per tile for all channels.
+//   One CTA = one work item = (batch b, time chunk c, block of kCB channels).
+//   Two threads share a channel: lanes l and l^16 of a warp, each keeping
+//   kHalf of the kN fp32 states in registers (as packed fp32x2 pairs) for the
+//   whole chunk, so one warp serves 16 channels.  Splitting the state gives
+//   each scheduler two warps' worth of independent instructions for the same
+//   number of channels, without cutting time into more chunks.
+//   Tiles of kTT timesteps of u / Δraw / z ([kTT x kCB]) and of B / C
+//   ([kTT x kN], shared by every channel) arrive in shared memory by TMA
+//   (cp.async.bulk.tensor, no multicast) through a ring of STAGES buffers
+//   completed on mbarriers; B and C are widened to fp32 once per tile.
 //
-// Time chunking (the "hardware-aware parallel scan": the recurrence is linear,
-// so a chunk maps its entry state h0 to P ⊙ h0 + h_loc with P = Π exp(Δ A)):
+// Per thread pair, timesteps go in groups of kG: each thread computes the
+//   per-step scalars (Δ, Δu, Du, gate) of half the group's steps, the pair
+//   swaps Δ and Δu by shuffle, both threads advance their half-states through
+//   all kG steps in order, and each thread finishes the outputs of the steps
+//   it prepared after one shuffle of the partial readouts.
+//
+// Time chunking (the recurrence is linear, so a chunk maps its entry state h0
+//   to P ⊙ h0 + h_loc with P = Π exp(Δ A)):
 //   Items take tickets from a global counter in chunk-major order.  An item
 //   whose predecessor chunk has already published its inclusive end state
 //   starts from it and is exact at once.  Otherwise it scans from zero
 //   (writing provisional outputs), publishes its aggregate (P, h_loc), looks
 //   back through its predecessors' aggregates to the nearest inclusive state
 //   (decoupled look-back; every wait is bounded), publishes its own inclusive
-//   state and adds Σ_n C_t,n P_t,n h0_n · gate to each of its outputs.
-//   Tickets are taken in start order, so an item only ever waits on items
-//   that are already running, and those publish before they wait.
+//   state, then re-streams Δraw, z and its provisional y through the same TMA
+//   ring and adds (Σ_n C_t,n P_t,n h0_n) · gate_t to each output.  Tickets are
+//   taken in start order, so an item only ever waits on items that are
+//   already running, and those publish before they wait.
 //
-// A = a_d (n+1) fast path (bf16 I/O only): exp(Δ a_d (n+1)) = r^(n+1) with
-//   r = exp(Δ a_d), one hardware exp per channel-timestep plus a product
-//   ladder, instead of kN exps.  Detected per CTA with an exact test on A.
+// Units on the bf16 path: Δ is carried as λ = Δ / ln 2, so the decay is
+//   2^(λ A), Δ·B·u = λ·(ln 2·B)·u (ln 2 folded into B once per tile), and the
+//   softplus input is formed by one fused multiply-add.
+//
+// A = a_d (n+1) fast path (bf16 I/O): exp(Δ a_d (n+1)) = r^(n+1).  A thread
+//   gets its first decay r^(8p+1) and r from the hardware exp and the rest of
+//   its eight by a product ladder on pairs.  Detected per CTA with an exact
+//   test on A.
 #pragma once
 
 #include <type_traits>
 
 #include "common.cuh"
 
+#ifndef SELSCAN_GROUP
+#define SELSCAN_GROUP 8
+#endif
+
 namespace selscan {
 
 constexpr int kN = 16;      // d_state
+constexpr int kHalf = 8;    // states per thread
 constexpr int kTT = 32;     // timesteps per tile
-constexpr int kNT = 128;    // threads per CTA
-constexpr int kCB = kNT;    // channels per CTA (one per thread)
+constexpr int kG = SELSCAN_GROUP;   // timesteps per software-pipelined group
+constexpr int kNT = 256;    // threads per CTA
+constexpr int kCB = 128;    // channels per CTA (two threads per channel)
 constexpr int kRec = 48;    // floats per carry record: P[16], h_loc[16], inclusive[16]
+static_assert(kG % 2 == 0 && kTT % kG == 0, "groups hold an even number of steps and tile a tile");
+static_assert(kNT == 2 * kCB, "two threads per channel");
 
 enum : uint32_t { kStNone = 0, kStAgg = 1, kStIncl = 2, kStTimeout = 0xFFFFFFFFu };
 enum : uint32_t {
@@ -70,7 +93,8 @@ struct FwdParams {
     int64_t L;
     int batch, d, chunk_len, nchunks, nblk;
     uint32_t pflags;
-    uint32_t* hdr;       // [0]: error status (negative code as uint32), [1]: ticket counter
+    uint32_t* hdr;       // [0]: error status (negative code as uint32), [1]: ticket counter,
+                         // [2]: number of provisional items (diagnostic)
     uint32_t* status;    // [batch][nchunks][nblk] publication state of each item
     float* rec;          // [batch][nchunks][d][kRec] carry records
     uint64_t wait_ns;    // bound on one TMA completion wait
@@ -79,12 +103,12 @@ struct FwdParams {
 
 template <typename IO, int STAGES>
 struct FwdSmem {
-    IO u[STAGES][kTT][kCB];
+    IO a[STAGES][kTT][kCB];          // u (scan pass) or provisional y (fix-up pass)
     IO dt[STAGES][kTT][kCB];
     IO z[STAGES][kTT][kCB];
     IO B[STAGES][kTT][kN];
     IO C[STAGES][kTT][kN];
-    float bc[STAGES][kTT][2 * kN];   // B (ln-free, fp32) then C, per timestep
+    float bc[STAGES][kTT][2 * kN];   // per timestep: B (scaled to the λ units) then C, fp32
     uint64_t full[STAGES];
     int item;
     uint32_t st;
@@ -94,111 +118,520 @@ __device__ __forceinline__ void record_error(uint32_t* hdr, int code) {
     atomicCAS(&hdr[0], 0u, static_cast<uint32_t>(code));
 }
 
-// r^1 .. r^16 by a balanced product ladder (depth 5).
-__device__ __forceinline__ void power_ladder(float r, float (&pw)[kN]) {
-    pw[0] = r;
-    pw[1] = r * r;
-    pw[2] = pw[1] * r;
-    pw[3] = pw[1] * pw[1];
-    pw[4] = pw[3] * r;
-    pw[5] = pw[3] * pw[1];
-    pw[6] = pw[3] * pw[2];
-    pw[7] = pw[3] * pw[3];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) pw[8 + j] = pw[7] * pw[j];
-}
+// Value held by the other thread of this channel (lane ^ 16).
+__device__ __forceinline__ float partner(float v) { return __shfl_xor_sync(0xffffffffu, v, 16); }
 
+// λ for one element: Δ/ln 2 on the fast path (bias_s = bias·log2 e), Δ itself
+// on the accurate path (bias_s = bias).  sp_mask selects the softplus.
 template <bool FAST>
-__device__ __forceinline__ float delta_act(float x, bool softplus) {
-    if (!softplus) return x;
-    return FAST ? softplus_fast(x) : softplus_accurate(x);
+__device__ __forceinline__ float lam_of(float xraw, float bias_s, uint32_t sp_mask) {
+    if (FAST) {
+        const float y2 = fmaf(xraw, kLog2e, bias_s);
+        return blend(sp_mask, softplus_log2_fast(y2), y2);
+    }
+    const float x = xraw + bias_s;
+    return blend(sp_mask, softplus_accurate(x), x);
 }
 
 template <bool FAST>
 __device__ __forceinline__ float gate_of(float zv) {
-    return FAST ? silu_fast(zv) : silu_accurate(zv);
+    return FAST ? silu_tanh(zv) : silu_accurate(zv);
 }
 
-// decay exp(Δ A_n); A2 holds A·log2(e) on the fast path and A itself otherwise.
+// exp(Δ A) from λ and raw A.
 template <bool FAST>
-__device__ __forceinline__ float decay_of(float dl, float a2) {
-    return FAST ? ex2_approx(dl * a2) : expf(dl * a2);
+__device__ __forceinline__ float decay_of(float lam, float a) {
+    return FAST ? ex2_approx(lam * a) : expf(lam * a);
 }
 
-// One tile of nt timesteps for this thread's channel.
-template <typename IO, bool FAST, bool STRUCT, bool TRACK>
-__device__ __forceinline__ void scan_tile(const IO* __restrict__ us, const IO* __restrict__ dts,
-                                          const IO* __restrict__ zs, const float* __restrict__ bc,
-                                          int nt, float (&h)[kN], float (&P)[kN], float& R, float a2,
-                                          const float (&A2)[kN], float biasv, float Dv, bool softplus,
-                                          bool has_z, bool valid, IO* __restrict__ yrow, int64_t d) {
-#pragma unroll 1
-    for (int tt = 0; tt < nt; ++tt) {
-        const float uu = to_f32(us[tt * kCB]);
-        const float dl = delta_act<FAST>(to_f32(dts[tt * kCB]) + biasv, softplus);
-        const float4* bq = reinterpret_cast<const float4*>(bc + tt * 2 * kN);
-        float Bv[kN], Cv[kN];
+struct ChanParams {
+    float Av[kHalf];   // raw A of this thread's states 8p .. 8p+7
+    float a;           // A[ch, 0]; on the structured path A[ch, n] = a (n + 1)
+    float ab;          // a (8p + 1): exponent factor of this half's first decay
+    float bias_s;      // bias in the softplus input's scale
+    float Dv;
+    uint32_t sp_mask;  // all ones: Δ goes through softplus
+    uint32_t z_mask;   // all ones: the silu(z) gate is on
+    uint32_t hi_mask;  // all ones on the thread holding the upper half (p = 1)
+    int p;             // 0: states 0..7, 1: states 8..15
+    bool valid;        // channel < d_inner
+};
+
+// Decays of this thread's eight states as pairs, for the structured path:
+// (r^(8p+1), r^(8p+2)), ..., (r^(8p+7), r^(8p+8)) from base = r^(8p+1).
+__device__ __forceinline__ void half_ladder(float base, float r, f32x2 (&Q)[4]) {
+    const float r2 = r * r;
+    const f32x2 R2 = pk2(r2, r2);
+    Q[0] = pk2(base, base * r);
+    Q[1] = mul2(Q[0], R2);
+    Q[2] = mul2(Q[1], R2);
+    Q[3] = mul2(Q[2], R2);
+}
+
+// Loads this thread's four B pairs and four C pairs of one timestep row.
+__device__ __forceinline__ void load_bc(const float* __restrict__ bcrow, int p, f32x2 (&Bp)[4], f32x2 (&Cp)[4]) {
+    const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcrow + kHalf * p);
+    const ulonglong2 b0 = q[0], b1 = q[1];
+    const ulonglong2 c0 = q[4], c1 = q[5];
+    Bp[0] = b0.x; Bp[1] = b0.y; Bp[2] = b1.x; Bp[3] = b1.y;
+    Cp[0] = c0.x; Cp[1] = c0.y; Cp[2] = c1.x; Cp[3] = c1.y;
+}
+__device__ __forceinline__ void load_c(const float* __restrict__ bcrow, int p, f32x2 (&Cp)[4]) {
+    const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcrow + kN + kHalf * p);
+    const ulonglong2 c0 = q[0], c1 = q[1];
+    Cp[0] = c0.x; Cp[1] = c0.y; Cp[2] = c1.x; Cp[3] = c1.y;
+}
+
+// This thread's half of the readout Σ_n C_n h_n.
+__device__ __forceinline__ float half_dot(const f32x2 (&Cp)[4], const f32x2 (&H)[4]) {
+    f32x2 a0 = mul2(Cp[0], H[0]);
+    f32x2 a1 = mul2(Cp[1], H[1]);
+    a0 = fma2(Cp[2], H[2], a0);
+    a1 = fma2(Cp[3], H[3], a1);
+    float lo, hi;
+    upk2(add2(a0, a1), lo, hi);
+    return lo + hi;
+}
+
+// One state update of this thread's half for one timestep.
+template <bool FAST, bool STRUCT, bool TRACK>
+__device__ __forceinline__ void half_update(float lam, float du, const f32x2 (&Bp)[4], f32x2 (&H)[4],
+                                            f32x2 (&PP)[4], float& R, const ChanParams& cp) {
+    const f32x2 DU = pk2(du, du);
+    if (STRUCT) {
+        const float r = ex2_approx(lam * cp.a);
+        f32x2 Q[4];
+        half_ladder(ex2_approx(lam * cp.ab), r, Q);
 #pragma unroll
-        for (int q = 0; q < kN / 4; ++q) {
-            const float4 b4 = bq[q];
-            const float4 c4 = bq[kN / 4 + q];
-            Bv[4 * q + 0] = b4.x; Bv[4 * q + 1] = b4.y; Bv[4 * q + 2] = b4.z; Bv[4 * q + 3] = b4.w;
-            Cv[4 * q + 0] = c4.x; Cv[4 * q + 1] = c4.y; Cv[4 * q + 2] = c4.z; Cv[4 * q + 3] = c4.w;
+        for (int m = 0; m < 4; ++m) H[m] = fma2(Q[m], H[m], mul2(DU, Bp[m]));
+        if (TRACK) R *= r;
+    } else {
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const f32x2 P = pk2(decay_of<FAST>(lam, cp.Av[2 * m]), decay_of<FAST>(lam, cp.Av[2 * m + 1]));
+            H[m] = fma2(P, H[m], mul2(DU, Bp[m]));
+            if (TRACK) PP[m] = mul2(PP[m], P);
         }
-        const float du = dl * uu;
-        if (STRUCT) {
-            const float r = ex2_approx(dl * a2);
-            float pw[kN];
-            power_ladder(r, pw);
+    }
+}
+
+// A group of NSTEP (even) timesteps of the scan, rows j0 .. j0+NSTEP-1.
+// us/dts/zs point at this channel's column of the tile (row 0); yrow at this
+// channel's output for row 0 of the tile.
+template <typename IO, bool FAST, bool STRUCT, bool TRACK, int NSTEP>
+__device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* __restrict__ dts,
+                                           const IO* __restrict__ zs, const float* __restrict__ bc, int j0,
+                                           f32x2 (&H)[4], f32x2 (&PP)[4], float& R, const ChanParams& cp,
+                                           IO* __restrict__ yrow, int64_t d) {
+    constexpr int NH = NSTEP / 2;
+    // Phase A: this thread prepares steps j0 + 2i + p.
+    float lo[NH], dlo[NH], su[NH], g[NH];
 #pragma unroll
-            for (int n = 0; n < kN; ++n) h[n] = fmaf(pw[n], h[n], du * Bv[n]);
-            if (TRACK) R *= r;
+    for (int i = 0; i < NH; ++i) {
+        const int row = (j0 + 2 * i + cp.p) * kCB;
+        const float uu = to_f32(us[row]);
+        lo[i] = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
+        dlo[i] = lo[i] * uu;
+        su[i] = cp.Dv * uu;
+        g[i] = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+    }
+    float lam[NSTEP], du[NSTEP];
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+        const float lx = partner(lo[i]);
+        const float dx = partner(dlo[i]);
+        lam[2 * i] = blend(cp.hi_mask, lx, lo[i]);
+        lam[2 * i + 1] = blend(cp.hi_mask, lo[i], lx);
+        du[2 * i] = blend(cp.hi_mask, dx, dlo[i]);
+        du[2 * i + 1] = blend(cp.hi_mask, dlo[i], dx);
+    }
+    // Phase B: the state updates, in time order.
+    float part[NSTEP];
+#pragma unroll
+    for (int j = 0; j < NSTEP; ++j) {
+        f32x2 Bp[4], Cp[4];
+        load_bc(bc + (j0 + j) * 2 * kN, cp.p, Bp, Cp);
+        half_update<FAST, STRUCT, TRACK>(lam[j], du[j], Bp, H, PP, R, cp);
+        part[j] = half_dot(Cp, H);
+    }
+    // Finish the outputs of this thread's steps: y = (lower + upper + D u) gate.
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+        const float send = blend(cp.hi_mask, part[2 * i], part[2 * i + 1]);
+        const float mine = blend(cp.hi_mask, part[2 * i + 1], part[2 * i]);
+        const float yv = (mine + partner(send) + su[i]) * g[i];
+        if (cp.valid) yrow[static_cast<int64_t>(j0 + 2 * i + cp.p) * d] = from_f32<IO>(yv);
+    }
+}
+
+// One timestep of the scan (ragged tails); both threads prepare it.
+template <typename IO, bool FAST, bool STRUCT, bool TRACK>
+__device__ __forceinline__ void scan_one(const IO* __restrict__ us, const IO* __restrict__ dts,
+                                         const IO* __restrict__ zs, const float* __restrict__ bc, int j,
+                                         f32x2 (&H)[4], f32x2 (&PP)[4], float& R, const ChanParams& cp,
+                                         IO* __restrict__ yrow, int64_t d) {
+    const int row = j * kCB;
+    const float uu = to_f32(us[row]);
+    const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
+    const float g = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+    f32x2 Bp[4], Cp[4];
+    load_bc(bc + j * 2 * kN, cp.p, Bp, Cp);
+    half_update<FAST, STRUCT, TRACK>(lam, lam * uu, Bp, H, PP, R, cp);
+    const float part = half_dot(Cp, H);
+    const float yv = (part + partner(part) + cp.Dv * uu) * g;
+    if (cp.valid && cp.p == 0) yrow[static_cast<int64_t>(j) * d] = from_f32<IO>(yv);
+}
+
+// This thread's half of the entry-state correction Σ_n C_n P_t,n h0_n.
+template <bool FAST, bool STRUCT>
+__device__ __forceinline__ float half_corr(float lam, const f32x2 (&Cp)[4], const f32x2 (&H0)[4], f32x2 (&PQ)[4],
+                                           float& Rq, const ChanParams& cp) {
+    f32x2 CH[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) CH[m] = mul2(Cp[m], H0[m]);
+    if (STRUCT) {
+        Rq *= ex2_approx(lam * cp.a);
+        // Σ_m c_m Rq^(8p+1+m) = Rq^(8p+1) · Σ_k (c_2k + c_2k+1 Rq) (Rq^2)^k
+        const float R2 = Rq * Rq;
+        const float R8 = (R2 * R2) * (R2 * R2);
+        const float base = blend(cp.hi_mask, R8 * Rq, Rq);
+        float s = 0.0f;
+#pragma unroll
+        for (int m = 3; m >= 0; --m) {
+            float c0, c1;
+            upk2(CH[m], c0, c1);
+            s = fmaf(s, R2, fmaf(c1, Rq, c0));
+        }
+        return s * base;
+    } else {
+        f32x2 a0 = pk2(0.0f, 0.0f), a1 = pk2(0.0f, 0.0f);
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            PQ[m] = mul2(PQ[m], pk2(decay_of<FAST>(lam, cp.Av[2 * m]), decay_of<FAST>(lam, cp.Av[2 * m + 1])));
+            if (m & 1) a1 = fma2(CH[m], PQ[m], a1);
+            else       a0 = fma2(CH[m], PQ[m], a0);
+        }
+        float lo, hi;
+        upk2(add2(a0, a1), lo, hi);
+        return lo + hi;
+    }
+}
+
+// A group of NSTEP (even) timesteps of the fix-up pass.
+template <typename IO, bool FAST, bool STRUCT, int NSTEP>
+__device__ __forceinline__ void fix_group(const IO* __restrict__ ys, const IO* __restrict__ dts,
+                                          const IO* __restrict__ zs, const float* __restrict__ bc, int j0,
+                                          const f32x2 (&H0)[4], f32x2 (&PQ)[4], float& Rq, const ChanParams& cp,
+                                          IO* __restrict__ yrow, int64_t d) {
+    constexpr int NH = NSTEP / 2;
+    float lo[NH], g[NH], yo[NH];
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+        const int row = (j0 + 2 * i + cp.p) * kCB;
+        lo[i] = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
+        g[i] = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+        yo[i] = to_f32(ys[row]);
+    }
+    float lam[NSTEP];
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+        const float lx = partner(lo[i]);
+        lam[2 * i] = blend(cp.hi_mask, lx, lo[i]);
+        lam[2 * i + 1] = blend(cp.hi_mask, lo[i], lx);
+    }
+    float part[NSTEP];
+#pragma unroll
+    for (int j = 0; j < NSTEP; ++j) {
+        f32x2 Cp[4];
+        load_c(bc + (j0 + j) * 2 * kN, cp.p, Cp);
+        part[j] = half_corr<FAST, STRUCT>(lam[j], Cp, H0, PQ, Rq, cp);
+    }
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+        const float send = blend(cp.hi_mask, part[2 * i], part[2 * i + 1]);
+        const float mine = blend(cp.hi_mask, part[2 * i + 1], part[2 * i]);
+        const float yv = fmaf(mine + partner(send), g[i], yo[i]);
+        if (cp.valid) yrow[static_cast<int64_t>(j0 + 2 * i + cp.p) * d] = from_f32<IO>(yv);
+    }
+}
+
+template <typename IO, bool FAST, bool STRUCT>
+__device__ __forceinline__ void fix_one(const IO* __restrict__ ys, const IO* __restrict__ dts,
+                                        const IO* __restrict__ zs, const float* __restrict__ bc, int j,
+                                        const f32x2 (&H0)[4], f32x2 (&PQ)[4], float& Rq, const ChanParams& cp,
+                                        IO* __restrict__ yrow, int64_t d) {
+    const int row = j * kCB;
+    const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
+    const float g = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+    f32x2 Cp[4];
+    load_c(bc + j * 2 * kN, cp.p, Cp);
+    const float part = half_corr<FAST, STRUCT>(lam, Cp, H0, PQ, Rq, cp);
+    const float yv = fmaf(part + partner(part), g, to_f32(ys[row]));
+    if (cp.valid && cp.p == 0) yrow[static_cast<int64_t>(j) * d] = from_f32<IO>(yv);
+}
+
+// Coordinates and tile-ring plumbing of one work item.
+template <typename IO, bool USE_TMA, int STAGES>
+struct ItemCtx {
+    const FwdParams* p;
+    FwdSmem<IO, STAGES>* S;
+    const CUtensorMap *tm_u, *tm_dt, *tm_z, *tm_B, *tm_C, *tm_y;
+    int tid, b, c, g, ntiles;
+    int cc;             // this thread's channel within the block
+    int64_t t_begin, t_end, d;
+    bool has_z;
+    float bscale;
+    uint32_t bytes_scan, bytes_fix;
+
+    // pass 0: u, Δraw, z, B, C;  pass 1: provisional y, Δraw, z, C
+    __device__ __forceinline__ void issue(int k, int s, int pass) const {
+        const int t0 = static_cast<int>(t_begin + static_cast<int64_t>(k) * kTT);
+        uint64_t* bar = &S->full[s];
+        mbar_arrive_expect_tx(bar, pass == 0 ? bytes_scan : bytes_fix);
+        tma_load_3d(&S->a[s][0][0], pass == 0 ? tm_u : tm_y, g * kCB, t0, b, bar);
+        tma_load_3d(&S->dt[s][0][0], tm_dt, g * kCB, t0, b, bar);
+        if (has_z) tma_load_3d(&S->z[s][0][0], tm_z, g * kCB, t0, b, bar);
+        if (pass == 0) tma_load_3d(&S->B[s][0][0], tm_B, 0, t0, b, bar);
+        tma_load_3d(&S->C[s][0][0], tm_C, 0, t0, b, bar);
+    }
+
+    __device__ __forceinline__ void fill_plain(int k, int pass) const {
+        const int64_t t0 = t_begin + static_cast<int64_t>(k) * kTT;
+        const IO* ga = static_cast<const IO*>(pass == 0 ? p->u : p->y);
+        const IO* gd = static_cast<const IO*>(p->delta);
+        const IO* gz = static_cast<const IO*>(p->z);
+        for (int i = tid; i < kTT * kCB; i += kNT) {
+            const int r = i / kCB, col = i % kCB;
+            const int64_t t = t0 + r;
+            const int ch = g * kCB + col;
+            const bool ok = (t < p->L) && (ch < p->d);
+            const int64_t idx = (static_cast<int64_t>(b) * p->L + t) * d + ch;
+            S->a[0][r][col] = ok ? ga[idx] : from_f32<IO>(0.f);
+            S->dt[0][r][col] = ok ? gd[idx] : from_f32<IO>(0.f);
+            if (has_z) S->z[0][r][col] = ok ? gz[idx] : from_f32<IO>(0.f);
+        }
+        const IO* gB = static_cast<const IO*>(p->B);
+        const IO* gC = static_cast<const IO*>(p->C);
+        for (int i = tid; i < kTT * kN; i += kNT) {
+            const int r = i / kN, n = i % kN;
+            const int64_t t = t0 + r;
+            const bool ok = t < p->L;
+            const int64_t idx = (static_cast<int64_t>(b) * p->L + t) * kN + n;
+            if (pass == 0) S->B[0][r][n] = ok ? gB[idx] : from_f32<IO>(0.f);
+            S->C[0][r][n] = ok ? gC[idx] : from_f32<IO>(0.f);
+        }
+    }
+
+    // Waits for (or loads) tile k of this pass -- tile number kk of the CTA --
+    // widens its B/C to fp32, and refills the stage the previous tile freed.
+    __device__ __forceinline__ int acquire(int k, int kk, int pass) const {
+        const int s = USE_TMA ? (kk % STAGES) : 0;
+        if constexpr (USE_TMA) {
+            if (!mbar_wait_bounded(&S->full[s], static_cast<uint32_t>((kk / STAGES) & 1), p->wait_ns))
+                record_error(p->hdr, -4);
         } else {
-#pragma unroll
-            for (int n = 0; n < kN; ++n) {
-                const float a = decay_of<FAST>(dl, A2[n]);
-                h[n] = fmaf(a, h[n], du * Bv[n]);
-                if (TRACK) P[n] *= a;
+            __syncthreads();
+            fill_plain(k, pass);
+            __syncthreads();
+        }
+        for (int i = tid; i < kTT * kN; i += kNT) {
+            const int r = i / kN, n = i % kN;
+            if (pass == 0) S->bc[s][r][n] = to_f32(S->B[s][r][n]) * bscale;
+            S->bc[s][r][kN + n] = to_f32(S->C[s][r][n]);
+        }
+        __syncthreads();
+        if constexpr (USE_TMA) {
+            if (tid == 0 && k >= 1 && k + STAGES - 1 < ntiles) {
+                fence_proxy_async_smem();
+                issue(k + STAGES - 1, (kk - 1 + STAGES) % STAGES, pass);
             }
         }
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int n = 0; n < kN; ++n) acc[n & 3] = fmaf(Cv[n], h[n], acc[n & 3]);
-        float yv = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        yv = fmaf(Dv, uu, yv);
-        if (has_z) yv *= gate_of<FAST>(to_f32(zs[tt * kCB]));
-        if (valid) yrow[tt * d] = from_f32<IO>(yv);
+        return s;
     }
-}
+};
 
-// Loads 16 consecutive IO elements (16-byte aligned) as fp32.
-__device__ __forceinline__ void load16(const float* p, float (&v)[kN]) {
-    const float4* q = reinterpret_cast<const float4*>(p);
+// The scan (and, for a provisional chunk, look-back and fix-up) of one item,
+// specialised on the decay form and on whether the entry state is known.
+template <typename IO, bool USE_TMA, int STAGES, bool STRUCT, bool EXACT>
+__device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it, const ChanParams& cp,
+                                         f32x2 (&H)[4]) {
+    constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
+    constexpr bool TRACK = !EXACT;
+    const FwdParams& p = *it.p;
+    auto& S = *it.S;
+    const int tid = it.tid;
+    const int64_t d = it.d;
+    const int hp = kHalf * cp.p;   // first state index of this thread
+
+    f32x2 PP[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float4 f = __ldg(q + i);
-        v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+    for (int m = 0; m < 4; ++m) PP[m] = pk2(1.f, 1.f);
+    float R = 1.f;
+    int64_t t = it.t_begin;
+    IO* ybase = static_cast<IO*>(p.y) + (static_cast<int64_t>(it.b) * p.L + it.t_begin) * d + (it.g * kCB + it.cc);
+    int kk = 0;   // tiles consumed so far by this CTA (both passes)
+
+    for (int k = 0; k < it.ntiles; ++k, ++kk) {
+        const int s = it.acquire(k, kk, 0);
+        const int nt = static_cast<int>((it.t_end - t) < kTT ? (it.t_end - t) : kTT);
+        const IO* us = &S.a[s][0][it.cc];
+        const IO* dts = &S.dt[s][0][it.cc];
+        const IO* zs = &S.z[s][0][it.cc];
+        const float* bc = &S.bc[s][0][0];
+        IO* yrow = ybase + (t - it.t_begin) * d;
+        int j0 = 0;
+        for (; j0 + kG <= nt; j0 += kG) scan_group<IO, FAST, STRUCT, TRACK, kG>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+        for (; j0 < nt; ++j0)           scan_one<IO, FAST, STRUCT, TRACK>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+        t += nt;
     }
-}
-__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[kN]) {
-    const uint4* q = reinterpret_cast<const uint4*>(p);
+
+    // ------------------------------------------------------------ epilogue
+    const int b = it.b, c = it.c, g = it.g;
+    const int ch = g * kCB + it.cc;
+    const bool last = (c == p.nchunks - 1);
+    const bool drop = (p.pflags & kPfTestDrop) && b == 0 && c == 0 && g == 0;
+    uint32_t* st_me = p.status + (static_cast<int64_t>(b) * p.nchunks + c) * p.nblk + g;
+    float* rec_me = p.rec + ((static_cast<int64_t>(b) * p.nchunks + c) * d + ch) * kRec + hp;
+    float* ls = p.last_state ? p.last_state + (static_cast<int64_t>(b) * d + ch) * kN + hp : nullptr;
+
+    float h[kHalf];
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const uint4 w = __ldg(q + i);
-        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    for (int m = 0; m < 4; ++m) upk2(H[m], h[2 * m], h[2 * m + 1]);
+
+    if constexpr (EXACT) {
+        if (!last) {
+            if (cp.valid) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            v[8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
-            v[8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+                for (int n = 0; n < kHalf; ++n) __stcg(rec_me + 32 + n, h[n]);
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0 && !drop) st_release_gpu(st_me, kStIncl);
+        } else if (cp.valid && ls) {
+#pragma unroll
+            for (int n = 0; n < kHalf; ++n) ls[n] = h[n];
+        }
+        return;
+    } else {
+        // Provisional chunk: make the provisional y visible to the TMA reads
+        // of the fix-up pass, then publish the aggregate (P, h_loc).
+        fence_proxy_async_global();
+        float P[kHalf];
+        if (STRUCT) {
+            const float R2 = R * R;
+            const float R8 = (R2 * R2) * (R2 * R2);
+            f32x2 Q[4];
+            half_ladder(blend(cp.hi_mask, R8 * R, R), R, Q);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) upk2(Q[m], P[2 * m], P[2 * m + 1]);
+        } else {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) upk2(PP[m], P[2 * m], P[2 * m + 1]);
+        }
+        if (cp.valid) {
+#pragma unroll
+            for (int n = 0; n < kHalf; ++n) {
+                __stcg(rec_me + n, P[n]);
+                __stcg(rec_me + 16 + n, h[n]);
+            }
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) st_release_gpu(st_me, kStAgg);
+
+        // Start streaming the fix-up tiles while the look-back runs.
+        if constexpr (USE_TMA) {
+            if (tid == 0) {
+                tma_prefetch_desc(it.tm_y);
+                for (int s = 0; s < STAGES && s < it.ntiles; ++s) it.issue(s, (kk + s) % STAGES, 1);
+            }
+        }
+
+        // Decoupled look-back: h0 = XP ⊙ I_j + Xh, walking j = c-1, c-2, ...
+        float XP[kHalf], Xh[kHalf];
+#pragma unroll
+        for (int n = 0; n < kHalf; ++n) { XP[n] = 1.f; Xh[n] = 0.f; }
+        for (int j = c - 1; j >= 0; --j) {
+            if (tid == 0) {
+                const uint32_t* sp = p.status + (static_cast<int64_t>(b) * p.nchunks + j) * p.nblk + g;
+                uint32_t sv = ld_acquire_gpu(sp);
+                uint32_t polls = 0;
+                while (sv == kStNone) {
+                    if (++polls > p.poll_limit) {
+                        sv = kStTimeout;
+                        record_error(p.hdr, -4);
+                        break;
+                    }
+                    __nanosleep(128);
+                    sv = ld_acquire_gpu(sp);
+                }
+                S.st = sv;
+            }
+            __syncthreads();
+            const uint32_t sv = S.st;
+            __syncthreads();
+            if (sv == kStTimeout) break;
+            if (cp.valid) {
+                const float* rj = p.rec + ((static_cast<int64_t>(b) * p.nchunks + j) * d + ch) * kRec + hp;
+                if (sv == kStIncl) {
+#pragma unroll
+                    for (int n = 0; n < kHalf; ++n) Xh[n] = fmaf(XP[n], __ldcg(rj + 32 + n), Xh[n]);
+                } else {
+#pragma unroll
+                    for (int n = 0; n < kHalf; ++n) {
+                        Xh[n] = fmaf(XP[n], __ldcg(rj + 16 + n), Xh[n]);
+                        XP[n] *= __ldcg(rj + n);
+                    }
+                }
+            }
+            if (sv == kStIncl) break;
+        }
+
+        // Inclusive end state of this chunk: I = P ⊙ h0 + h_loc.
+        if (!last) {
+            if (cp.valid) {
+#pragma unroll
+                for (int n = 0; n < kHalf; ++n) __stcg(rec_me + 32 + n, fmaf(P[n], Xh[n], h[n]));
+            }
+            __threadfence();
+            __syncthreads();
+            if (tid == 0) st_release_gpu(st_me, kStIncl);
+        } else if (cp.valid && ls) {
+#pragma unroll
+            for (int n = 0; n < kHalf; ++n) ls[n] = fmaf(P[n], Xh[n], h[n]);
+        }
+
+        // Fix-up pass over this chunk's outputs.
+        f32x2 H0[4], PQ[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            H0[m] = pk2(Xh[2 * m], Xh[2 * m + 1]);
+            PQ[m] = pk2(1.f, 1.f);
+        }
+        float Rq = 1.f;
+        t = it.t_begin;
+        for (int k = 0; k < it.ntiles; ++k, ++kk) {
+            const int s = it.acquire(k, kk, 1);
+            const int nt = static_cast<int>((it.t_end - t) < kTT ? (it.t_end - t) : kTT);
+            const IO* ys = &S.a[s][0][it.cc];
+            const IO* dts = &S.dt[s][0][it.cc];
+            const IO* zs = &S.z[s][0][it.cc];
+            const float* bc = &S.bc[s][0][0];
+            IO* yrow = ybase + (t - it.t_begin) * d;
+            int j0 = 0;
+            for (; j0 + kG <= nt; j0 += kG) fix_group<IO, FAST, STRUCT, kG>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
+            for (; j0 < nt; ++j0)           fix_one<IO, FAST, STRUCT>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
+            t += nt;
         }
     }
 }
 
-template <typename IO, bool USE_TMA, int STAGES>
-__global__ void __launch_bounds__(kNT)
+template <typename IO, bool USE_TMA, int STAGES, int MINB>
+__global__ void __launch_bounds__(kNT, MINB)
 ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_u,
               const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_z,
-              const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C) {
+              const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
+              const __grid_constant__ CUtensorMap tm_y) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     auto& S = *reinterpret_cast<FwdSmem<IO, STAGES>*>(smem_raw);
@@ -208,94 +641,73 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
     if (tid == 0) S.item = (p.nchunks > 1) ? static_cast<int>(atomicAdd(&p.hdr[1], 1u))
                                            : static_cast<int>(blockIdx.x);
     __syncthreads();
-    const int item = S.item;
-    const int g = item % p.nblk;
-    const int rest = item / p.nblk;
-    const int b = rest % p.batch;
-    const int c = rest / p.batch;
-    const int ch = g * kCB + tid;
-    const bool valid = ch < p.d;
-    const int64_t t_begin = static_cast<int64_t>(c) * p.chunk_len;
-    const int64_t t_end = min(p.L, t_begin + p.chunk_len);
-    const int ntiles = static_cast<int>((t_end - t_begin + kTT - 1) / kTT);
-    const bool has_z = (p.pflags & kPfHasZ) != 0;
-    const bool softplus = (p.pflags & kPfSoftplus) != 0;
-    const int64_t d = p.d;
+    ItemCtx<IO, USE_TMA, STAGES> it;
+    it.p = &p;
+    it.S = &S;
+    it.tm_u = &tm_u; it.tm_dt = &tm_dt; it.tm_z = &tm_z; it.tm_B = &tm_B; it.tm_C = &tm_C; it.tm_y = &tm_y;
+    it.tid = tid;
+    {
+        const int item = S.item;
+        it.g = item % p.nblk;
+        const int rest = item / p.nblk;
+        it.b = rest % p.batch;
+        it.c = rest / p.batch;
+    }
+    const int lane = tid & 31;
+    it.cc = (tid >> 5) * 16 + (lane & 15);
+    it.t_begin = static_cast<int64_t>(it.c) * p.chunk_len;
+    it.t_end = min(p.L, it.t_begin + p.chunk_len);
+    it.ntiles = static_cast<int>((it.t_end - it.t_begin + kTT - 1) / kTT);
+    it.d = p.d;
+    it.has_z = (p.pflags & kPfHasZ) != 0;
+    it.bscale = FAST ? kLn2 : 1.0f;
+    const int nact = it.has_z ? 3 : 2;   // per-channel tensors streamed per pass
+    it.bytes_scan = static_cast<uint32_t>((nact * kTT * kCB + 2 * kTT * kN) * sizeof(IO));
+    it.bytes_fix = static_cast<uint32_t>((nact * kTT * kCB + kTT * kN) * sizeof(IO));
+    const int ch = it.g * kCB + it.cc;
 
     // ------------------------------------------------- per-channel parameters
-    float A2[kN];
+    ChanParams cp;
+    cp.p = lane >> 4;
+    cp.hi_mask = cp.p ? 0xffffffffu : 0u;
+    cp.valid = ch < p.d;
+    cp.z_mask = it.has_z ? 0xffffffffu : 0u;
+    cp.sp_mask = (p.pflags & kPfSoftplus) ? 0xffffffffu : 0u;
+    const int hp = kHalf * cp.p;
     bool structured = true;
     {
-        float Arow[kN];
+        const float* Arow = p.A + static_cast<int64_t>(cp.valid ? ch : 0) * kN;
+        cp.a = cp.valid ? __ldg(Arow) : -1.0f;
 #pragma unroll
-        for (int n = 0; n < kN; ++n) Arow[n] = valid ? __ldg(p.A + static_cast<int64_t>(ch) * kN + n)
-                                                     : -static_cast<float>(n + 1);
-#pragma unroll
-        for (int n = 0; n < kN; ++n) {
-            structured = structured && (Arow[n] == Arow[0] * static_cast<float>(n + 1));
-            A2[n] = FAST ? Arow[n] * kLog2e : Arow[n];
+        for (int n = 0; n < kHalf; ++n) {
+            cp.Av[n] = cp.valid ? __ldg(Arow + hp + n) : -static_cast<float>(hp + n + 1);
+            structured = structured && (cp.Av[n] == cp.a * static_cast<float>(hp + n + 1));
         }
     }
     const int all_struct = __syncthreads_and(structured ? 1 : 0);
     const bool use_struct = FAST && all_struct && !(p.pflags & kPfForceGeneral);
-    const float a2 = A2[0];
-    const float Dv = (valid && (p.pflags & kPfHasD)) ? __ldg(p.D + ch) : 0.f;
-    const float biasv = (valid && (p.pflags & kPfHasBias)) ? __ldg(p.bias + ch) : 0.f;
+    cp.ab = cp.a * static_cast<float>(hp + 1);
+    cp.Dv = (cp.valid && (p.pflags & kPfHasD)) ? __ldg(p.D + ch) : 0.f;
+    const float biasv = (cp.valid && (p.pflags & kPfHasBias)) ? __ldg(p.bias + ch) : 0.f;
+    cp.bias_s = FAST ? biasv * kLog2e : biasv;
 
     // ------------------------------------------------------- entry state
-    float h[kN];
+    f32x2 H[4];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = 0.f;
+    for (int m = 0; m < 4; ++m) H[m] = pk2(0.f, 0.f);
     bool exact = true;
-    if (c > 0) {
+    if (it.c > 0) {
         if (tid == 0)
-            S.st = ld_acquire_gpu(p.status + (static_cast<int64_t>(b) * p.nchunks + (c - 1)) * p.nblk + g);
+            S.st = ld_acquire_gpu(p.status + (static_cast<int64_t>(it.b) * p.nchunks + (it.c - 1)) * p.nblk + it.g);
         __syncthreads();
         exact = (S.st == kStIncl);
-        if (exact && valid) {
-            const float* r = p.rec + ((static_cast<int64_t>(b) * p.nchunks + (c - 1)) * d + ch) * kRec + 32;
+        if (exact && cp.valid) {
+            const float* r = p.rec + ((static_cast<int64_t>(it.b) * p.nchunks + (it.c - 1)) * it.d + ch) * kRec + 32 + hp;
 #pragma unroll
-            for (int n = 0; n < kN; ++n) h[n] = __ldcg(r + n);
+            for (int m = 0; m < 4; ++m) H[m] = pk2(__ldcg(r + 2 * m), __ldcg(r + 2 * m + 1));
         }
     }
-
-    // ------------------------------------------------------- tile pipeline
-    const uint32_t tile_bytes = static_cast<uint32_t>(((has_z ? 3 : 2) * kTT * kCB + 2 * kTT * kN) * sizeof(IO));
-    auto issue = [&](int k, int s) {
-        const int t0 = static_cast<int>(t_begin + static_cast<int64_t>(k) * kTT);
-        mbar_arrive_expect_tx(&S.full[s], tile_bytes);
-        tma_load_3d(&S.u[s][0][0], &tm_u, g * kCB, t0, b, &S.full[s]);
-        tma_load_3d(&S.dt[s][0][0], &tm_dt, g * kCB, t0, b, &S.full[s]);
-        if (has_z) tma_load_3d(&S.z[s][0][0], &tm_z, g * kCB, t0, b, &S.full[s]);
-        tma_load_3d(&S.B[s][0][0], &tm_B, 0, t0, b, &S.full[s]);
-        tma_load_3d(&S.C[s][0][0], &tm_C, 0, t0, b, &S.full[s]);
-    };
-    auto fill_plain = [&](int k) {
-        const int64_t t0 = t_begin + static_cast<int64_t>(k) * kTT;
-        const IO* gu = static_cast<const IO*>(p.u);
-        const IO* gd = static_cast<const IO*>(p.delta);
-        const IO* gz = static_cast<const IO*>(p.z);
-        for (int i = tid; i < kTT * kCB; i += kNT) {
-            const int r = i / kCB, col = i % kCB;
-            const int64_t t = t0 + r;
-            const int cc = g * kCB + col;
-            const bool ok = (t < p.L) && (cc < p.d);
-            const int64_t idx = (static_cast<int64_t>(b) * p.L + t) * d + cc;
-            S.u[0][r][col] = ok ? gu[idx] : from_f32<IO>(0.f);
-            S.dt[0][r][col] = ok ? gd[idx] : from_f32<IO>(0.f);
-            if (has_z) S.z[0][r][col] = ok ? gz[idx] : from_f32<IO>(0.f);
-        }
-        const IO* gB = static_cast<const IO*>(p.B);
-        const IO* gC = static_cast<const IO*>(p.C);
-        for (int i = tid; i < kTT * kN; i += kNT) {
-            const int r = i / kN, n = i % kN;
-            const int64_t t = t0 + r;
-            const bool ok = t < p.L;
-            const int64_t idx = (static_cast<int64_t>(b) * p.L + t) * kN + n;
-            S.B[0][r][n] = ok ? gB[idx] : from_f32<IO>(0.f);
-            S.C[0][r][n] = ok ? gC[idx] : from_f32<IO>(0.f);
-        }
-    };
+    if (!exact && tid == 0) atomicAdd(&p.hdr[2], 1u);
 
     if constexpr (USE_TMA) {
         if (tid == 0) {
@@ -304,187 +716,21 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
             fence_mbar_init();
             tma_prefetch_desc(&tm_u);
             tma_prefetch_desc(&tm_dt);
-            if (has_z) tma_prefetch_desc(&tm_z);
+            if (it.has_z) tma_prefetch_desc(&tm_z);
             tma_prefetch_desc(&tm_B);
             tma_prefetch_desc(&tm_C);
         }
         __syncthreads();
         if (tid == 0)
-            for (int s = 0; s < STAGES && s < ntiles; ++s) issue(s, s);
+            for (int s = 0; s < STAGES && s < it.ntiles; ++s) it.issue(s, s, 0);
     }
 
-    float P[kN];
-#pragma unroll
-    for (int n = 0; n < kN; ++n) P[n] = 1.f;
-    float R = 1.f;
-    int64_t t = t_begin;
-    IO* yrow = static_cast<IO*>(p.y) + (static_cast<int64_t>(b) * p.L + t_begin) * d + ch;
-
-    for (int k = 0; k < ntiles; ++k) {
-        const int s = USE_TMA ? (k % STAGES) : 0;
-        if constexpr (USE_TMA) {
-            if (!mbar_wait_bounded(&S.full[s], static_cast<uint32_t>((k / STAGES) & 1), p.wait_ns))
-                record_error(p.hdr, -4);
-        } else {
-            __syncthreads();
-            fill_plain(k);
-            __syncthreads();
-        }
-        for (int i = tid; i < kTT * kN; i += kNT) {
-            const int r = i / kN, n = i % kN;
-            S.bc[s][r][n] = to_f32(S.B[s][r][n]);
-            S.bc[s][r][kN + n] = to_f32(S.C[s][r][n]);
-        }
-        __syncthreads();
-        if constexpr (USE_TMA) {
-            if (tid == 0 && k >= 1 && k + STAGES - 1 < ntiles) {
-                fence_proxy_async_smem();
-                issue(k + STAGES - 1, (k - 1) % STAGES);
-            }
-        }
-        const int nt = static_cast<int>((t_end - t) < kTT ? (t_end - t) : kTT);
-        const IO* us = &S.u[s][0][tid];
-        const IO* dts = &S.dt[s][0][tid];
-        const IO* zs = &S.z[s][0][tid];
-        const float* bc = &S.bc[s][0][0];
-        if (use_struct) {
-            if (exact) scan_tile<IO, FAST, true, false>(us, dts, zs, bc, nt, h, P, R, a2, A2, biasv, Dv, softplus, has_z, valid, yrow, d);
-            else       scan_tile<IO, FAST, true, true >(us, dts, zs, bc, nt, h, P, R, a2, A2, biasv, Dv, softplus, has_z, valid, yrow, d);
-        } else {
-            if (exact) scan_tile<IO, FAST, false, false>(us, dts, zs, bc, nt, h, P, R, a2, A2, biasv, Dv, softplus, has_z, valid, yrow, d);
-            else       scan_tile<IO, FAST, false, true >(us, dts, zs, bc, nt, h, P, R, a2, A2, biasv, Dv, softplus, has_z, valid, yrow, d);
-        }
-        t += nt;
-        yrow += static_cast<int64_t>(nt) * d;
-    }
-
-    // ------------------------------------------------------------ epilogue
-    const bool last = (c == p.nchunks - 1);
-    const bool drop = (p.pflags & kPfTestDrop) && b == 0 && c == 0 && g == 0;
-    uint32_t* st_me = p.status + (static_cast<int64_t>(b) * p.nchunks + c) * p.nblk + g;
-    float* rec_me = p.rec + ((static_cast<int64_t>(b) * p.nchunks + c) * d + ch) * kRec;
-
-    if (exact) {
-        if (!last) {
-            if (valid) {
-#pragma unroll
-                for (int n = 0; n < kN; ++n) __stcg(rec_me + 32 + n, h[n]);
-            }
-            __threadfence();
-            __syncthreads();
-            if (tid == 0 && !drop) st_release_gpu(st_me, kStIncl);
-        } else if (valid && p.last_state) {
-            float* ls = p.last_state + (static_cast<int64_t>(b) * d + ch) * kN;
-#pragma unroll
-            for (int n = 0; n < kN; ++n) ls[n] = h[n];
-        }
-        return;
-    }
-
-    // Provisional chunk: publish the aggregate (P, h_loc) first.
-    if (use_struct) power_ladder(R, P);
-    if (valid) {
-#pragma unroll
-        for (int n = 0; n < kN; ++n) {
-            __stcg(rec_me + n, P[n]);
-            __stcg(rec_me + 16 + n, h[n]);
-        }
-    }
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) st_release_gpu(st_me, kStAgg);
-
-    // Decoupled look-back: h0 = XP ⊙ I_j + Xh, walking j = c-1, c-2, ...
-    float XP[kN], Xh[kN];
-#pragma unroll
-    for (int n = 0; n < kN; ++n) { XP[n] = 1.f; Xh[n] = 0.f; }
-    for (int j = c - 1; j >= 0; --j) {
-        if (tid == 0) {
-            const uint32_t* sp = p.status + (static_cast<int64_t>(b) * p.nchunks + j) * p.nblk + g;
-            uint32_t sv = ld_acquire_gpu(sp);
-            uint32_t it = 0;
-            while (sv == kStNone) {
-                if (++it > p.poll_limit) {
-                    sv = kStTimeout;
-                    record_error(p.hdr, -4);
-                    break;
-                }
-                __nanosleep(128);
-                sv = ld_acquire_gpu(sp);
-            }
-            S.st = sv;
-        }
-        __syncthreads();
-        const uint32_t sv = S.st;
-        __syncthreads();
-        if (sv == kStTimeout) break;
-        if (valid) {
-            const float* rj = p.rec + ((static_cast<int64_t>(b) * p.nchunks + j) * d + ch) * kRec;
-            if (sv == kStIncl) {
-#pragma unroll
-                for (int n = 0; n < kN; ++n) Xh[n] = fmaf(XP[n], __ldcg(rj + 32 + n), Xh[n]);
-            } else {
-#pragma unroll
-                for (int n = 0; n < kN; ++n) {
-                    Xh[n] = fmaf(XP[n], __ldcg(rj + 16 + n), Xh[n]);
-                    XP[n] *= __ldcg(rj + n);
-                }
-            }
-        }
-        if (sv == kStIncl) break;
-    }
-
-    // Inclusive end state of this chunk: I = P ⊙ h0 + h_loc.
-    if (!last) {
-        if (valid) {
-#pragma unroll
-            for (int n = 0; n < kN; ++n) __stcg(rec_me + 32 + n, fmaf(P[n], Xh[n], h[n]));
-        }
-        __threadfence();
-        __syncthreads();
-        if (tid == 0) st_release_gpu(st_me, kStIncl);
-    } else if (valid && p.last_state) {
-        float* ls = p.last_state + (static_cast<int64_t>(b) * d + ch) * kN;
-#pragma unroll
-        for (int n = 0; n < kN; ++n) ls[n] = fmaf(P[n], Xh[n], h[n]);
-    }
-
-    // Fix-up: y_t += (Σ_n C_t,n · P_t,n · h0_n) · gate_t, P_t the in-chunk
-    // prefix decay, recomputed exactly as during the scan.
-    if (!valid) return;
-    const IO* gd = static_cast<const IO*>(p.delta);
-    const IO* gz = static_cast<const IO*>(p.z);
-    const IO* gC = static_cast<const IO*>(p.C);
-    IO* gy = static_cast<IO*>(p.y);
-    float Rq = 1.f;
-    float Pq[kN];
-#pragma unroll
-    for (int n = 0; n < kN; ++n) Pq[n] = 1.f;
-#pragma unroll 1
-    for (int64_t tq = t_begin; tq < t_end; ++tq) {
-        const int64_t row = static_cast<int64_t>(b) * p.L + tq;
-        const int64_t idx = row * d + ch;
-        const float dl = delta_act<FAST>(to_f32(gd[idx]) + biasv, softplus);
-        float Cv[kN];
-        load16(gC + row * kN, Cv);
-        float corr;
-        if (use_struct) {
-            Rq *= ex2_approx(dl * a2);
-            float acc = Cv[kN - 1] * Xh[kN - 1];
-#pragma unroll
-            for (int n = kN - 2; n >= 0; --n) acc = fmaf(acc, Rq, Cv[n] * Xh[n]);
-            corr = acc * Rq;
-        } else {
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int n = 0; n < kN; ++n) {
-                Pq[n] *= decay_of<FAST>(dl, A2[n]);
-                acc[n & 3] = fmaf(Cv[n] * Pq[n], Xh[n], acc[n & 3]);
-            }
-            corr = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-        }
-        if (has_z) corr *= gate_of<FAST>(to_f32(gz[idx]));
-        gy[idx] = from_f32<IO>(to_f32(gy[idx]) + corr);
+    if (use_struct) {
+        if (exact) run_item<IO, USE_TMA, STAGES, true, true>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, true, false>(it, cp, H);
+    } else {
+        if (exact) run_item<IO, USE_TMA, STAGES, false, true>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, false, false>(it, cp, H);
     }
 }
 

@@ -18,7 +18,7 @@ using namespace selscan;
 namespace {
 
 constexpr int kVersion = 10000;             // 1.0.0
-constexpr size_t kHeaderBytes = 256;        // error word, ticket counter
+constexpr size_t kHeaderBytes = 256;        // error word, ticket counter, provisional-item count
 constexpr uint32_t kDefaultPolls = 1u << 21;
 constexpr uint64_t kTmaWaitNs = 2000000000ull;
 constexpr int kMaxDevices = 64;
@@ -40,21 +40,31 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Resident CTAs per SM for the bf16 / fp32 forward kernels (shared memory bound).
-int ctas_per_sm(bool bf16) { return bf16 ? 2 : 1; }
+// Resident forward CTAs per SM and depth of each CTA's tile ring (shared
+// memory: 4 stages ~ 120 KB, 3 stages ~ 92 KB of bf16 tiles).
+#ifndef SELSCAN_CTAS_PER_SM
+#define SELSCAN_CTAS_PER_SM 1
+#endif
+constexpr int kCtasPerSm = SELSCAN_CTAS_PER_SM;
+constexpr int kStagesBf16 = kCtasPerSm == 1 ? 4 : 3;
+// Items per resident CTA slot the automatic chunking aims for (load balance:
+// the last wave is at most 1/kWaves of the work), and the shortest chunk.
+constexpr int64_t kWaves = 8;
+constexpr int64_t kMinChunk = 256;
 
-// Library choice of chunk length: enough (batch, chunk, channel-block) items
-// for two waves of resident CTAs; 0 = no time chunking.
+// Library choice of chunk length; 0 = no time chunking.
 int32_t auto_chunk_len(const ss_dims* dims, uint32_t flags) {
+    (void)flags;
     const int64_t L = dims->seqlen;
-    if (L <= kTT) return 0;
+    if (L <= kMinChunk) return 0;
     const int64_t nblk = ceil_div(dims->d_inner, kCB);
     const int64_t base = dims->batch * nblk;
     if (base <= 0) return 0;
-    const int64_t slots = static_cast<int64_t>(sm_count_of_current_device()) * ctas_per_sm(flags & SS_BF16);
-    const int64_t nchunks = ceil_div(2 * slots, base);
+    const int64_t slots = static_cast<int64_t>(sm_count_of_current_device()) * kCtasPerSm;
+    const int64_t nchunks = ceil_div(kWaves * slots, base);
     if (nchunks <= 1) return 0;
     int64_t chunk = ceil_div(ceil_div(L, nchunks), kTT) * kTT;
+    if (chunk < kMinChunk) chunk = kMinChunk;
     if (chunk >= L) return 0;
     if (chunk > (1 << 30)) chunk = 1 << 30;
     return static_cast<int32_t>(chunk);
@@ -123,7 +133,7 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint6
 
 template <typename IO, bool TMA, int STAGES>
 int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
-    auto kern = ss_fwd_kernel<IO, TMA, STAGES>;
+    auto kern = ss_fwd_kernel<IO, TMA, STAGES, kCtasPerSm>;
     const size_t smem = sizeof(FwdSmem<IO, STAGES>);
     static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
@@ -134,7 +144,8 @@ int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaS
             return SS_ERR_CUDA;
         if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
     }
-    kern<<<static_cast<unsigned>(items), kNT, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4]);
+    kern<<<static_cast<unsigned>(items), kNT, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4],
+                                                              maps[5]);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
@@ -242,18 +253,19 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
 
     // TMA needs 16-byte row strides: d * element size a multiple of 16.
     const bool tma = ((d * (bf16 ? 2 : 4)) % 16) == 0;
-    CUtensorMap maps[5];
+    CUtensorMap maps[6];
     std::memset(maps, 0, sizeof(maps));
     if (tma) {
         bool ok = make_map(&maps[0], u, bf16, d, L, batch, kCB, kTT) &&
                   make_map(&maps[1], delta, bf16, d, L, batch, kCB, kTT) &&
                   make_map(&maps[2], z ? z : u, bf16, d, L, batch, kCB, kTT) &&
                   make_map(&maps[3], B, bf16, kN, L, batch, kN, kTT) &&
-                  make_map(&maps[4], C, bf16, kN, L, batch, kN, kTT);
+                  make_map(&maps[4], C, bf16, kN, L, batch, kN, kTT) &&
+                  make_map(&maps[5], y, bf16, d, L, batch, kCB, kTT);
         if (!ok) return SS_ERR_CUDA;
     }
     if (bf16) {
-        rc = tma ? launch_fwd<__nv_bfloat16, true, 3>(p, items, maps, stream)
+        rc = tma ? launch_fwd<__nv_bfloat16, true, kStagesBf16>(p, items, maps, stream)
                  : launch_fwd<__nv_bfloat16, false, 1>(p, items, maps, stream);
     } else {
         rc = tma ? launch_fwd<float, true, 2>(p, items, maps, stream)
@@ -281,8 +293,7 @@ int ss_step(float* state, const void* u, const void* delta, const float* A, cons
     p.state = state; p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z; p.y = y;
     p.bias = delta_bias; p.channels = batch * d; p.d = static_cast<int>(d);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
-    const int64_t threads = p.channels * 4;
-    const int64_t blocks = ceil_div(threads, kStepThreads);
+    const int64_t blocks = ceil_div(p.channels, kStepChanPerBlock);
     if (blocks >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
     cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
     if (bf16)

@@ -7,7 +7,9 @@
 // token.  The kernel is bound by HBM traffic on the state (read + write), so
 // the state moves in fully coalesced 16-byte accesses: four consecutive
 // threads share one channel, each owning four consecutive states, and the
-// readout Σ_n C_n h_n is finished with two butterfly shuffles.
+// readout Σ_n C_n h_n is finished with two butterfly shuffles.  Each thread
+// serves kStepCPT channels (kStepThreads/4 apart) and issues all their state
+// loads before computing, to keep more bytes in flight per thread.
 #pragma once
 
 #include <type_traits>
@@ -17,6 +19,8 @@
 namespace selscan {
 
 constexpr int kStepThreads = 256;
+constexpr int kStepCPT = 2;                                       // channels per thread
+constexpr int kStepChanPerBlock = kStepThreads / 4 * kStepCPT;    // 128
 
 struct StepParams {
     float* state;
@@ -51,51 +55,64 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
 template <typename IO>
 __global__ void __launch_bounds__(kStepThreads) ss_step_kernel(const __grid_constant__ StepParams p) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
-    const int64_t gid = static_cast<int64_t>(blockIdx.x) * kStepThreads + threadIdx.x;
-    const int64_t chan = gid >> 2;            // (b * d + ch)
-    const int q = static_cast<int>(gid & 3);  // states 4q .. 4q+3
-    const bool valid = chan < p.channels;
-    const int64_t cs = valid ? chan : 0;
-    const int64_t b = cs / p.d;
-    const int ch = static_cast<int>(cs % p.d);
+    const int q = threadIdx.x & 3;   // states 4q .. 4q+3
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * kStepChanPerBlock + (threadIdx.x >> 2);
 
-    float4* srow = reinterpret_cast<float4*>(p.state + cs * 16) + q;
-    float4 h4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Bv[4], Cv[4], Av[4];
-    float uu = 0.f, xr = 0.f, zz = 0.f, Dv = 0.f, bv = 0.f;
-    if (valid) {
-        h4 = *srow;
+    int64_t cs[kStepCPT];
+    bool valid[kStepCPT];
+    float4 h4[kStepCPT];
+    float uu[kStepCPT], xr[kStepCPT], zz[kStepCPT];
+#pragma unroll
+    for (int k = 0; k < kStepCPT; ++k) {
+        const int64_t chan = base + k * (kStepThreads / 4);
+        valid[k] = chan < p.channels;
+        cs[k] = valid[k] ? chan : 0;
+        h4[k] = valid[k] ? *(reinterpret_cast<const float4*>(p.state + cs[k] * 16) + q)
+                         : make_float4(0.f, 0.f, 0.f, 0.f);
+        uu[k] = valid[k] ? to_f32(static_cast<const IO*>(p.u)[cs[k]]) : 0.f;
+        xr[k] = valid[k] ? to_f32(static_cast<const IO*>(p.delta)[cs[k]]) : 0.f;
+        zz[k] = (valid[k] && p.z) ? to_f32(static_cast<const IO*>(p.z)[cs[k]]) : 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < kStepCPT; ++k) {
+        const int64_t b = cs[k] / p.d;
+        const int ch = static_cast<int>(cs[k] % p.d);
+        float Bv[4], Cv[4], Av[4];
         load4<IO>(static_cast<const IO*>(p.B) + b * 16 + 4 * q, Bv);
         load4<IO>(static_cast<const IO*>(p.C) + b * 16 + 4 * q, Cv);
         load4<float>(p.A + static_cast<int64_t>(ch) * 16 + 4 * q, Av);
-        uu = to_f32(static_cast<const IO*>(p.u)[cs]);
-        xr = to_f32(static_cast<const IO*>(p.delta)[cs]);
-        if (p.z) zz = to_f32(static_cast<const IO*>(p.z)[cs]);
-        if (p.D) Dv = __ldg(p.D + ch);
-        if (p.bias) bv = __ldg(p.bias + ch);
-    } else {
+        const float Dv = p.D ? __ldg(p.D + ch) : 0.f;
+        const float bv = p.bias ? __ldg(p.bias + ch) : 0.f;
+        // λ = Δ / ln 2 on the fast path (decay 2^(λ A), Δ u = λ (ln 2 u)); Δ itself otherwise.
+        float lam, dscale;
+        if (FAST) {
+            const float y2 = fmaf(xr[k], kLog2e, bv * kLog2e);
+            lam = p.softplus ? softplus_log2_fast(y2) : y2;
+            dscale = kLn2;
+        } else {
+            const float x = xr[k] + bv;
+            lam = p.softplus ? softplus_accurate(x) : x;
+            dscale = 1.0f;
+        }
+        const float du = lam * (dscale * uu[k]);
+        float hv[4] = {h4[k].x, h4[k].y, h4[k].z, h4[k].w};
+        float acc = 0.f;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) { Bv[k] = 0.f; Cv[k] = 0.f; Av[k] = -1.f; }
-    }
-    float dl = xr + bv;
-    if (p.softplus) dl = FAST ? softplus_fast(dl) : softplus_accurate(dl);
-    const float du = dl * uu;
-    float hv[4] = {h4.x, h4.y, h4.z, h4.w};
-    float acc = 0.f;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const float a = FAST ? ex2_approx(dl * (Av[k] * kLog2e)) : expf(dl * Av[k]);
-        hv[k] = fmaf(a, hv[k], du * Bv[k]);
-        acc = fmaf(Cv[k], hv[k], acc);
-    }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (!valid) return;
-    *srow = make_float4(hv[0], hv[1], hv[2], hv[3]);
-    if (q == 0) {
-        float yv = fmaf(Dv, uu, acc);
-        if (p.z) yv *= FAST ? silu_fast(zz) : silu_accurate(zz);
-        static_cast<IO*>(p.y)[cs] = from_f32<IO>(yv);
+        for (int m = 0; m < 4; ++m) {
+            const float a = FAST ? ex2_approx(lam * Av[m]) : expf(lam * Av[m]);
+            hv[m] = fmaf(a, hv[m], du * Bv[m]);
+            acc = fmaf(Cv[m], hv[m], acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (valid[k]) {
+            *(reinterpret_cast<float4*>(p.state + cs[k] * 16) + q) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+            if (q == 0) {
+                float yv = fmaf(Dv, uu[k], acc);
+                if (p.z) yv *= FAST ? silu_tanh(zz[k]) : silu_accurate(zz[k]);
+                static_cast<IO*>(p.y)[cs[k]] = from_f32<IO>(yv);
+            }
+        }
     }
 }
 
