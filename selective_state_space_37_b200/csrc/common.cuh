@@ -72,32 +72,17 @@ __device__ __forceinline__ float blend(uint32_t mask, float a, float b) {
 }
 
 // ------------------------------------------------------------ packed fp32x2
-// Two fp32 lanes in one 64-bit register pair; the sm_100 f32x2 instructions
-// do two lane operations per issue slot.
-typedef unsigned long long f32x2;
-__device__ __forceinline__ f32x2 pk2(float lo, float hi) {
-    f32x2 r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
+// Two fp32 lanes per operand; on sm_100 each packed instruction does two
+// lane operations per issue slot (the CUDA float2 arithmetic intrinsics).
+typedef float2 f32x2;
+__device__ __forceinline__ f32x2 pk2(float lo, float hi) { return make_float2(lo, hi); }
 __device__ __forceinline__ void upk2(f32x2 v, float& lo, float& hi) {
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    lo = v.x;
+    hi = v.y;
 }
-__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) {
-    f32x2 d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
-    f32x2 d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) {
-    f32x2 d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b) { return __fadd2_rn(a, b); }
 
 // Accurate path (fp32 I/O): the CUDA math library.
 __device__ __forceinline__ float softplus_accurate(float x) {

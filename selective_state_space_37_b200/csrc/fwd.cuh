@@ -56,6 +56,12 @@
 #ifndef SELSCAN_GROUP
 #define SELSCAN_GROUP 8
 #endif
+#ifndef SELSCAN_STAGED
+#define SELSCAN_STAGED 0
+#endif
+#ifndef SELSCAN_UNROLL_TILE
+#define SELSCAN_UNROLL_TILE 1
+#endif
 
 namespace selscan {
 
@@ -170,16 +176,16 @@ __device__ __forceinline__ void half_ladder(float base, float r, f32x2 (&Q)[4]) 
 
 // Loads this thread's four B pairs and four C pairs of one timestep row.
 __device__ __forceinline__ void load_bc(const float* __restrict__ bcrow, int p, f32x2 (&Bp)[4], f32x2 (&Cp)[4]) {
-    const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcrow + kHalf * p);
-    const ulonglong2 b0 = q[0], b1 = q[1];
-    const ulonglong2 c0 = q[4], c1 = q[5];
-    Bp[0] = b0.x; Bp[1] = b0.y; Bp[2] = b1.x; Bp[3] = b1.y;
-    Cp[0] = c0.x; Cp[1] = c0.y; Cp[2] = c1.x; Cp[3] = c1.y;
+    const float4* q = reinterpret_cast<const float4*>(bcrow + kHalf * p);
+    const float4 b0 = q[0], b1 = q[1];
+    const float4 c0 = q[4], c1 = q[5];
+    Bp[0] = pk2(b0.x, b0.y); Bp[1] = pk2(b0.z, b0.w); Bp[2] = pk2(b1.x, b1.y); Bp[3] = pk2(b1.z, b1.w);
+    Cp[0] = pk2(c0.x, c0.y); Cp[1] = pk2(c0.z, c0.w); Cp[2] = pk2(c1.x, c1.y); Cp[3] = pk2(c1.z, c1.w);
 }
 __device__ __forceinline__ void load_c(const float* __restrict__ bcrow, int p, f32x2 (&Cp)[4]) {
-    const ulonglong2* q = reinterpret_cast<const ulonglong2*>(bcrow + kN + kHalf * p);
-    const ulonglong2 c0 = q[0], c1 = q[1];
-    Cp[0] = c0.x; Cp[1] = c0.y; Cp[2] = c1.x; Cp[3] = c1.y;
+    const float4* q = reinterpret_cast<const float4*>(bcrow + kN + kHalf * p);
+    const float4 c0 = q[0], c1 = q[1];
+    Cp[0] = pk2(c0.x, c0.y); Cp[1] = pk2(c0.z, c0.w); Cp[2] = pk2(c1.x, c1.y); Cp[3] = pk2(c1.z, c1.w);
 }
 
 // This thread's half of the readout Σ_n C_n h_n.
@@ -247,12 +253,42 @@ __device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* 
     }
     // Phase B: the state updates, in time order.
     float part[NSTEP];
+#if SELSCAN_STAGED
+    if (STRUCT) {
+        // Decay pairs and input pairs of every step first (independent work),
+        // then the chained updates and readouts.
+        f32x2 Q[NSTEP][4], V[NSTEP][4];
 #pragma unroll
-    for (int j = 0; j < NSTEP; ++j) {
-        f32x2 Bp[4], Cp[4];
-        load_bc(bc + (j0 + j) * 2 * kN, cp.p, Bp, Cp);
-        half_update<FAST, STRUCT, TRACK>(lam[j], du[j], Bp, H, PP, R, cp);
-        part[j] = half_dot(Cp, H);
+        for (int j = 0; j < NSTEP; ++j) {
+            const float4* q = reinterpret_cast<const float4*>(bc + (j0 + j) * 2 * kN + kHalf * cp.p);
+            const float4 b0 = q[0], b1 = q[1];
+            const f32x2 DU = pk2(du[j], du[j]);
+            V[j][0] = mul2(DU, pk2(b0.x, b0.y));
+            V[j][1] = mul2(DU, pk2(b0.z, b0.w));
+            V[j][2] = mul2(DU, pk2(b1.x, b1.y));
+            V[j][3] = mul2(DU, pk2(b1.z, b1.w));
+            const float r = ex2_approx(lam[j] * cp.a);
+            half_ladder(ex2_approx(lam[j] * cp.ab), r, Q[j]);
+            if (TRACK) R *= r;
+        }
+#pragma unroll
+        for (int j = 0; j < NSTEP; ++j) {
+#pragma unroll
+            for (int m = 0; m < 4; ++m) H[m] = fma2(Q[j][m], H[m], V[j][m]);
+            f32x2 Cp[4];
+            load_c(bc + (j0 + j) * 2 * kN, cp.p, Cp);
+            part[j] = half_dot(Cp, H);
+        }
+    } else
+#endif
+    {
+#pragma unroll
+        for (int j = 0; j < NSTEP; ++j) {
+            f32x2 Bp[4], Cp[4];
+            load_bc(bc + (j0 + j) * 2 * kN, cp.p, Bp, Cp);
+            half_update<FAST, STRUCT, TRACK>(lam[j], du[j], Bp, H, PP, R, cp);
+            part[j] = half_dot(Cp, H);
+        }
     }
     // Finish the outputs of this thread's steps: y = (lower + upper + D u) gate.
 #pragma unroll
@@ -479,9 +515,15 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
         const IO* zs = &S.z[s][0][it.cc];
         const float* bc = &S.bc[s][0][0];
         IO* yrow = ybase + (t - it.t_begin) * d;
-        int j0 = 0;
-        for (; j0 + kG <= nt; j0 += kG) scan_group<IO, FAST, STRUCT, TRACK, kG>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
-        for (; j0 < nt; ++j0)           scan_one<IO, FAST, STRUCT, TRACK>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+        if (SELSCAN_UNROLL_TILE && nt == kTT) {
+#pragma unroll
+            for (int gi = 0; gi < kTT / kG; ++gi)
+                scan_group<IO, FAST, STRUCT, TRACK, kG>(us, dts, zs, bc, gi * kG, H, PP, R, cp, yrow, d);
+        } else {
+            int j0 = 0;
+            for (; j0 + kG <= nt; j0 += kG) scan_group<IO, FAST, STRUCT, TRACK, kG>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+            for (; j0 < nt; ++j0)           scan_one<IO, FAST, STRUCT, TRACK>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+        }
         t += nt;
     }
 
