@@ -158,6 +158,40 @@ SS_API const char* ss_status_string(int status);
 /* Library version, as MAJOR*10000 + MINOR*100 + PATCH. */
 SS_API int ss_version(void);
 
+/* Capacity of the scratch array behind ss_fwd_noalloc, in bytes. */
+#define SS_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* ss_fwd_noalloc -- ss_fwd for callers that cannot allocate device memory.
+ * (An engineering addition: the paper has no counterpart.)
+ *
+ * Some callers have no way to hand ss_fwd a workspace: runtimes that plan
+ * every byte of device memory ahead of time and forbid allocation while
+ * serving, plugin interfaces of host frameworks that pass an operator its
+ * inputs and outputs but no allocator or scratch buffer, and latency-bound
+ * paths that cannot afford cudaMalloc, which may synchronize the device.
+ * This entry point takes the same arguments as ss_fwd except the launch
+ * context (only a stream) and uses, as its workspace, one array of
+ * SS_NOALLOC_SCRATCH_BYTES that the library reserves in device memory when
+ * it is loaded (every GPU that loads the library holds it until the process
+ * exits).  It calls no cudaMalloc, cudaFree or allocating library routine.
+ *
+ * - The first call on each device looks up that array's device address for
+ *   the current device (once; later calls reuse it).  Make that first call
+ *   before any stream capture.
+ * - Problems whose scratch need (ss_fwd_workspace_bytes with chunk_len 0)
+ *   exceeds SS_NOALLOC_SCRATCH_BYTES are rejected with SS_ERR_WORKSPACE
+ *   before anything is launched.
+ * - Every call on a device shares the one array; each call resets the parts
+ *   that must start at zero.  Calls whose work overlaps on the GPU (other
+ *   streams, other host threads) race on it and give wrong results: order
+ *   them on one stream.
+ * - Pass SS_SYNC_CHECK in flags to synchronize and get the device status;
+ *   ss_check cannot be used (the array is not exposed).
+ * Returns the same codes as ss_fwd. */
+SS_API int ss_fwd_noalloc(const void* u, const void* delta, const float* delta_bias, const float* A,
+                          const void* B, const void* C, const float* D, const void* z, void* y,
+                          float* last_state, uint32_t flags, const ss_dims* dims, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -33,7 +33,7 @@ D_STATE = 16
 
 # Every symbol include/selscan.h declares.
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
-            "ss_status_string", "ss_version")
+            "ss_status_string", "ss_version", "ss_fwd_noalloc")
 
 
 class ss_dims(ctypes.Structure):
@@ -87,6 +87,9 @@ def lib():
         L.ss_status_string.restype = ctypes.c_char_p
         L.ss_version.argtypes = []
         L.ss_version.restype = ctypes.c_int
+        L.ss_fwd_noalloc.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, vp, f32p, ctypes.c_uint32,
+                                     ctypes.POINTER(ss_dims), vp]
+        L.ss_fwd_noalloc.restype = ctypes.c_int
         _lib = L
     return _lib
 

@@ -165,6 +165,27 @@ int validate_dims(const ss_dims* dims, bool need_seqlen) {
     return SS_OK;
 }
 
+// ------------------------------------------------ allocation-free entry point
+// Workspace of ss_fwd_noalloc: one array in device memory per device that
+// loads this library, kept until the process exits.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SS_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (the host-side name is only a stand-in for it).
+void* noalloc_scratch_address() {
+    static void* addr[kMaxDevices] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        addr[dev] = p;
+    }
+    return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -305,6 +326,24 @@ int ss_step(float* state, const void* u, const void* delta, const float* A, cons
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
     }
     return SS_OK;
+}
+
+int ss_fwd_noalloc(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+                   const void* C, const float* D, const void* z, void* y, float* last_state, uint32_t flags,
+                   const ss_dims* dims, void* stream) {
+    // The same plan ss_fwd makes for these sizes decides the scratch need.
+    const size_t need = ss_fwd_workspace_bytes(dims, flags, 0);
+    if (need > SS_NOALLOC_SCRATCH_BYTES) return SS_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (need > 0) {
+        scratch = noalloc_scratch_address();
+        if (!scratch) return SS_ERR_CUDA;
+    }
+    ss_launch launch{};
+    launch.stream = stream;
+    launch.workspace = scratch;
+    launch.workspace_bytes = scratch ? SS_NOALLOC_SCRATCH_BYTES : 0;
+    return ss_fwd(u, delta, delta_bias, A, B, C, D, z, y, last_state, flags, dims, &launch);
 }
 
 }  // extern "C"
