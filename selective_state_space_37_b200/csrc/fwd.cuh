@@ -65,12 +65,19 @@
 
 namespace selscan {
 
+#ifndef SELSCAN_CB
+#define SELSCAN_CB 128
+#endif
+#ifndef SELSCAN_TT
+#define SELSCAN_TT 32
+#endif
+
 constexpr int kN = 16;      // d_state
 constexpr int kHalf = 8;    // states per thread
-constexpr int kTT = 32;     // timesteps per tile
+constexpr int kTT = SELSCAN_TT;     // timesteps per tile
 constexpr int kG = SELSCAN_GROUP;   // timesteps per software-pipelined group
-constexpr int kNT = 256;    // threads per CTA
-constexpr int kCB = 128;    // channels per CTA (two threads per channel)
+constexpr int kCB = SELSCAN_CB;     // channels per CTA (two threads per channel)
+constexpr int kNT = 2 * kCB;        // threads per CTA
 constexpr int kRec = 48;    // floats per carry record: P[16], h_loc[16], inclusive[16]
 static_assert(kG % 2 == 0 && kTT % kG == 0, "groups hold an even number of steps and tile a tile");
 static_assert(kNT == 2 * kCB, "two threads per channel");

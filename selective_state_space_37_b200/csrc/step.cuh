@@ -19,8 +19,8 @@
 namespace selscan {
 
 constexpr int kStepThreads = 256;
-constexpr int kStepCPT = 2;                                       // channels per thread
-constexpr int kStepChanPerBlock = kStepThreads / 4 * kStepCPT;    // 128
+constexpr int kStepCPT = 1;                                       // channels per thread
+constexpr int kStepChanPerBlock = kStepThreads / 4 * kStepCPT;    // 64
 
 struct StepParams {
     float* state;
