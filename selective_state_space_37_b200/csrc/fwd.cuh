@@ -20,10 +20,10 @@
 //   (cp.async.bulk.tensor, no multicast) through a ring of STAGES buffers
 //   completed on mbarriers; B and C are widened to fp32 once per tile.
 //
-// Per thread pair, timesteps go in groups of kG: each thread computes the
+// Per thread pair, timesteps go in groups of G: each thread computes the
 //   per-step scalars (Δ, Δu, Du, gate) of half the group's steps, the pair
 //   swaps Δ and Δu by shuffle, both threads advance their half-states through
-//   all kG steps in order, and each thread finishes the outputs of the steps
+//   all G steps in order, and each thread finishes the outputs of the steps
 //   it prepared after one shuffle of the partial readouts.
 //
 // Time chunking (the recurrence is linear, so a chunk maps its entry state h0
@@ -53,33 +53,14 @@
 
 #include "common.cuh"
 
-#ifndef SELSCAN_GROUP
-#define SELSCAN_GROUP 8
-#endif
-#ifndef SELSCAN_STAGED
-#define SELSCAN_STAGED 0
-#endif
-#ifndef SELSCAN_UNROLL_TILE
-#define SELSCAN_UNROLL_TILE 1
-#endif
-
 namespace selscan {
-
-#ifndef SELSCAN_CB
-#define SELSCAN_CB 128
-#endif
-#ifndef SELSCAN_TT
-#define SELSCAN_TT 32
-#endif
 
 constexpr int kN = 16;      // d_state
 constexpr int kHalf = 8;    // states per thread
-constexpr int kTT = SELSCAN_TT;     // timesteps per tile
-constexpr int kG = SELSCAN_GROUP;   // timesteps per software-pipelined group
-constexpr int kCB = SELSCAN_CB;     // channels per CTA (two threads per channel)
+constexpr int kTT = 32;     // timesteps per tile
+constexpr int kCB = 128;    // channels per CTA (two threads per channel)
 constexpr int kNT = 2 * kCB;        // threads per CTA
 constexpr int kRec = 48;    // floats per carry record: P[16], h_loc[16], inclusive[16]
-static_assert(kG % 2 == 0 && kTT % kG == 0, "groups hold an even number of steps and tile a tile");
 static_assert(kNT == 2 * kCB, "two threads per channel");
 
 enum : uint32_t { kStNone = 0, kStAgg = 1, kStIncl = 2, kStTimeout = 0xFFFFFFFFu };
@@ -260,42 +241,12 @@ __device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* 
     }
     // Phase B: the state updates, in time order.
     float part[NSTEP];
-#if SELSCAN_STAGED
-    if (STRUCT) {
-        // Decay pairs and input pairs of every step first (independent work),
-        // then the chained updates and readouts.
-        f32x2 Q[NSTEP][4], V[NSTEP][4];
 #pragma unroll
-        for (int j = 0; j < NSTEP; ++j) {
-            const float4* q = reinterpret_cast<const float4*>(bc + (j0 + j) * 2 * kN + kHalf * cp.p);
-            const float4 b0 = q[0], b1 = q[1];
-            const f32x2 DU = pk2(du[j], du[j]);
-            V[j][0] = mul2(DU, pk2(b0.x, b0.y));
-            V[j][1] = mul2(DU, pk2(b0.z, b0.w));
-            V[j][2] = mul2(DU, pk2(b1.x, b1.y));
-            V[j][3] = mul2(DU, pk2(b1.z, b1.w));
-            const float r = ex2_approx(lam[j] * cp.a);
-            half_ladder(ex2_approx(lam[j] * cp.ab), r, Q[j]);
-            if (TRACK) R *= r;
-        }
-#pragma unroll
-        for (int j = 0; j < NSTEP; ++j) {
-#pragma unroll
-            for (int m = 0; m < 4; ++m) H[m] = fma2(Q[j][m], H[m], V[j][m]);
-            f32x2 Cp[4];
-            load_c(bc + (j0 + j) * 2 * kN, cp.p, Cp);
-            part[j] = half_dot(Cp, H);
-        }
-    } else
-#endif
-    {
-#pragma unroll
-        for (int j = 0; j < NSTEP; ++j) {
-            f32x2 Bp[4], Cp[4];
-            load_bc(bc + (j0 + j) * 2 * kN, cp.p, Bp, Cp);
-            half_update<FAST, STRUCT, TRACK>(lam[j], du[j], Bp, H, PP, R, cp);
-            part[j] = half_dot(Cp, H);
-        }
+    for (int j = 0; j < NSTEP; ++j) {
+        f32x2 Bp[4], Cp[4];
+        load_bc(bc + (j0 + j) * 2 * kN, cp.p, Bp, Cp);
+        half_update<FAST, STRUCT, TRACK>(lam[j], du[j], Bp, H, PP, R, cp);
+        part[j] = half_dot(Cp, H);
     }
     // Finish the outputs of this thread's steps: y = (lower + upper + D u) gate.
 #pragma unroll
@@ -495,7 +446,7 @@ struct ItemCtx {
 
 // The scan (and, for a provisional chunk, look-back and fix-up) of one item,
 // specialised on the decay form and on whether the entry state is known.
-template <typename IO, bool USE_TMA, int STAGES, bool STRUCT, bool EXACT>
+template <typename IO, bool USE_TMA, int STAGES, int G, bool UNROLL, bool STRUCT, bool EXACT>
 __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it, const ChanParams& cp,
                                          f32x2 (&H)[4]) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
@@ -522,13 +473,13 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
         const IO* zs = &S.z[s][0][it.cc];
         const float* bc = &S.bc[s][0][0];
         IO* yrow = ybase + (t - it.t_begin) * d;
-        if (SELSCAN_UNROLL_TILE && nt == kTT) {
+        if (UNROLL && nt == kTT) {
 #pragma unroll
-            for (int gi = 0; gi < kTT / kG; ++gi)
-                scan_group<IO, FAST, STRUCT, TRACK, kG>(us, dts, zs, bc, gi * kG, H, PP, R, cp, yrow, d);
+            for (int gi = 0; gi < kTT / G; ++gi)
+                scan_group<IO, FAST, STRUCT, TRACK, G>(us, dts, zs, bc, gi * G, H, PP, R, cp, yrow, d);
         } else {
             int j0 = 0;
-            for (; j0 + kG <= nt; j0 += kG) scan_group<IO, FAST, STRUCT, TRACK, kG>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+            for (; j0 + G <= nt; j0 += G) scan_group<IO, FAST, STRUCT, TRACK, G>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
             for (; j0 < nt; ++j0)           scan_one<IO, FAST, STRUCT, TRACK>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
         }
         t += nt;
@@ -668,14 +619,15 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
             const float* bc = &S.bc[s][0][0];
             IO* yrow = ybase + (t - it.t_begin) * d;
             int j0 = 0;
-            for (; j0 + kG <= nt; j0 += kG) fix_group<IO, FAST, STRUCT, kG>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
+            for (; j0 + G <= nt; j0 += G) fix_group<IO, FAST, STRUCT, G>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
             for (; j0 < nt; ++j0)           fix_one<IO, FAST, STRUCT>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
             t += nt;
         }
     }
 }
 
-template <typename IO, bool USE_TMA, int STAGES, int MINB>
+// MINB resident CTAs per SM, groups of G steps, whole tiles unrolled or not.
+template <typename IO, bool USE_TMA, int STAGES, int MINB, int G, bool UNROLL>
 __global__ void __launch_bounds__(kNT, MINB)
 ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_u,
               const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_z,
@@ -774,12 +726,13 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
             for (int s = 0; s < STAGES && s < it.ntiles; ++s) it.issue(s, s, 0);
     }
 
+    static_assert(G % 2 == 0 && kTT % G == 0, "groups hold an even number of steps and tile a tile");
     if (use_struct) {
-        if (exact) run_item<IO, USE_TMA, STAGES, true, true>(it, cp, H);
-        else       run_item<IO, USE_TMA, STAGES, true, false>(it, cp, H);
+        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, true, true>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, true, false>(it, cp, H);
     } else {
-        if (exact) run_item<IO, USE_TMA, STAGES, false, true>(it, cp, H);
-        else       run_item<IO, USE_TMA, STAGES, false, false>(it, cp, H);
+        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, false, true>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, false, false>(it, cp, H);
     }
 }
 

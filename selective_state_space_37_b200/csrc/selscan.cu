@@ -40,31 +40,53 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
-// Resident forward CTAs per SM and depth of each CTA's tile ring (shared
-// memory: 4 stages ~ 120 KB, 3 stages ~ 92 KB of bf16 tiles).
-#ifndef SELSCAN_CTAS_PER_SM
-#define SELSCAN_CTAS_PER_SM 1
-#endif
-constexpr int kCtasPerSm = SELSCAN_CTAS_PER_SM;
-constexpr int kStagesBf16 = kCtasPerSm == 1 ? 4 : 3;
+// Forward-kernel variants.  Wide: one resident CTA per SM (two warps per
+// scheduler), a 4-stage tile ring, groups of 8 steps with whole tiles
+// unrolled -- fastest when every SM can work on channels whose entry state is
+// known.  Narrow: two resident CTAs per SM (four warps per scheduler, <= 128
+// registers), a 3-stage ring, groups of 4 -- better latency hiding when a
+// problem has few channel blocks, so that almost every time chunk is
+// provisional anyway.
+enum Variant { kWide = 0, kNarrow = 1 };
+constexpr int kCtasPerSm[2] = {1, 2};
 // Items per resident CTA slot the automatic chunking aims for (load balance:
 // the last wave is at most 1/kWaves of the work), and the shortest chunk.
 constexpr int64_t kWaves = 8;
 constexpr int64_t kMinChunk = 256;
 
+// Variant and automatic number of time chunks for these sizes.
+struct Choice {
+    Variant v;
+    int64_t nchunks;   // 1: no time chunking
+};
+
+Choice choose(const ss_dims* dims, uint32_t flags) {
+    const int64_t L = dims->seqlen;
+    const int64_t nblk = ceil_div(std::max<int64_t>(dims->d_inner, 1), kCB);
+    const int64_t base = std::max<int64_t>(dims->batch * nblk, 1);
+    const int64_t sms = sm_count_of_current_device();
+    const bool bf16 = (flags & SS_BF16) != 0;
+    Choice ch{kWide, 1};
+    if (base >= sms || !bf16) {
+        ch.nchunks = ceil_div(kWaves * sms * kCtasPerSm[kWide], base);
+    } else if (2 * base >= sms) {
+        ch.nchunks = 2;   // two waves of half-length chunks; most second halves start exact
+    } else {
+        ch.v = kNarrow;
+        ch.nchunks = ceil_div(kWaves * sms * kCtasPerSm[kNarrow], base);
+    }
+    const int64_t max_chunks = std::max<int64_t>(L / kMinChunk, 1);
+    ch.nchunks = std::min(ch.nchunks, max_chunks);
+    return ch;
+}
+
 // Library choice of chunk length; 0 = no time chunking.
 int32_t auto_chunk_len(const ss_dims* dims, uint32_t flags) {
-    (void)flags;
     const int64_t L = dims->seqlen;
     if (L <= kMinChunk) return 0;
-    const int64_t nblk = ceil_div(dims->d_inner, kCB);
-    const int64_t base = dims->batch * nblk;
-    if (base <= 0) return 0;
-    const int64_t slots = static_cast<int64_t>(sm_count_of_current_device()) * kCtasPerSm;
-    const int64_t nchunks = ceil_div(kWaves * slots, base);
-    if (nchunks <= 1) return 0;
-    int64_t chunk = ceil_div(ceil_div(L, nchunks), kTT) * kTT;
-    if (chunk < kMinChunk) chunk = kMinChunk;
+    const Choice ch = choose(dims, flags);
+    if (ch.nchunks <= 1) return 0;
+    int64_t chunk = ceil_div(ceil_div(L, ch.nchunks), kTT) * kTT;
     if (chunk >= L) return 0;
     if (chunk > (1 << 30)) chunk = 1 << 30;
     return static_cast<int32_t>(chunk);
@@ -131,9 +153,9 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint6
     return r == CUDA_SUCCESS;
 }
 
-template <typename IO, bool TMA, int STAGES>
+template <typename IO, bool TMA, int STAGES, int MINB, int G, bool UNROLL>
 int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
-    auto kern = ss_fwd_kernel<IO, TMA, STAGES, kCtasPerSm>;
+    auto kern = ss_fwd_kernel<IO, TMA, STAGES, MINB, G, UNROLL>;
     const size_t smem = sizeof(FwdSmem<IO, STAGES>);
     static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
@@ -286,11 +308,15 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
         if (!ok) return SS_ERR_CUDA;
     }
     if (bf16) {
-        rc = tma ? launch_fwd<__nv_bfloat16, true, kStagesBf16>(p, items, maps, stream)
-                 : launch_fwd<__nv_bfloat16, false, 1>(p, items, maps, stream);
+        if (choose(dims, flags).v == kNarrow)
+            rc = tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 4, false>(p, items, maps, stream)
+                     : launch_fwd<__nv_bfloat16, false, 1, 2, 4, false>(p, items, maps, stream);
+        else
+            rc = tma ? launch_fwd<__nv_bfloat16, true, 4, 1, 8, true>(p, items, maps, stream)
+                     : launch_fwd<__nv_bfloat16, false, 1, 1, 8, true>(p, items, maps, stream);
     } else {
-        rc = tma ? launch_fwd<float, true, 2>(p, items, maps, stream)
-                 : launch_fwd<float, false, 1>(p, items, maps, stream);
+        rc = tma ? launch_fwd<float, true, 2, 1, 8, false>(p, items, maps, stream)
+                 : launch_fwd<float, false, 1, 1, 8, false>(p, items, maps, stream);
     }
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) return ss_check(launch);

@@ -66,6 +66,18 @@ def test_small_bf16(shape, A_kind, chunk):
     check_full(inp, y, st, precisions=("f32",))
 
 
+@pytest.mark.parametrize("shape", [(38, 100, 512), (20, 600, 512), (19, 333, 1000)],
+                         ids=["wide_many_blocks", "wide_two_chunks", "wide_ragged"])
+def test_wide_variant_shapes(shape):
+    """Problems with at least half an SM's worth of channel blocks per SM run
+    the one-CTA-per-SM variant (the small tests above run the two-CTA one)."""
+    b, L, d = shape
+    inp = fwd_inputs(b, L, d, 16, "bf16", 40 + b + L + d, DEV, gate=True, D_kind="normal")
+    for chunk in (0, 96):
+        y, st = run(inp, chunk_len=chunk, sync_check=True)
+        check_full(inp, y, st, precisions=("f32",))
+
+
 @pytest.mark.parametrize("shape", [(2, 130, 64), (1, 70, 96), (2, 200, 30)])
 @pytest.mark.parametrize("chunk", [0, 64])
 def test_small_fp32(shape, chunk):
