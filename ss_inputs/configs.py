@@ -64,6 +64,9 @@ CONFIGS = {
                            "Mamba-2.8B-shaped layer: batch 4, L 8192, d_inner 5120, N 16"),
     "million": FwdConfig("million", 1, 1 << 20, 1536, 16, "bf16", "ones", True, 3,
                          "million-token scan: batch 1, L 1048576, d_inner 1536, N 16"),
+    "million_profile": FwdConfig("million_profile", 1, 1 << 17, 1536, 16, "bf16", "ones", True, 3,
+                                 "reduced million-token scan for profiling: batch 1, L 131072, "
+                                 "d_inner 1536, N 16"),
     "decode": StepConfig("decode", 256, 5120, 16, 1000, "bf16", True, 4,
                          "decode step: batch 256, d_inner 5120, N 16, 1000 steps"),
 }
