@@ -338,15 +338,15 @@ int ss_step(float* state, const void* u, const void* delta, const float* A, cons
     const bool bf16 = (flags & SS_BF16) != 0;
     StepParams p{};
     p.state = state; p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z; p.y = y;
-    p.bias = delta_bias; p.channels = batch * d; p.d = static_cast<int>(d);
+    p.bias = delta_bias; p.batch = batch; p.d = static_cast<int>(d);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
-    const int64_t blocks = ceil_div(p.channels, kStepChanPerBlock);
-    if (blocks >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    const dim3 grid(static_cast<unsigned>(ceil_div(d, kStepChanPerBlock)),
+                    static_cast<unsigned>(std::min<int64_t>(ceil_div(batch, 2), 65535)));
     cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
     if (bf16)
-        ss_step_kernel<__nv_bfloat16><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+        ss_step_kernel<__nv_bfloat16><<<grid, kStepThreads, 0, stream>>>(p);
     else
-        ss_step_kernel<float><<<static_cast<unsigned>(blocks), kStepThreads, 0, stream>>>(p);
+        ss_step_kernel<float><<<grid, kStepThreads, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;

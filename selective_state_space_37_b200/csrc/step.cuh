@@ -7,9 +7,9 @@
 // token.  The kernel is bound by HBM traffic on the state (read + write), so
 // the state moves in fully coalesced 16-byte accesses: four consecutive
 // threads share one channel, each owning four consecutive states, and the
-// readout Σ_n C_n h_n is finished with two butterfly shuffles.  Each thread
-// serves kStepCPT channels (kStepThreads/4 apart) and issues all their state
-// loads before computing, to keep more bytes in flight per thread.
+// readout Σ_n C_n h_n is finished with two butterfly shuffles.  A block
+// covers kStepChanPerBlock channels of one batch row, so a thread finds its
+// (batch, channel) without integer division.
 #pragma once
 
 #include <type_traits>
@@ -19,8 +19,7 @@
 namespace selscan {
 
 constexpr int kStepThreads = 256;
-constexpr int kStepCPT = 1;                                       // channels per thread
-constexpr int kStepChanPerBlock = kStepThreads / 4 * kStepCPT;    // 64
+constexpr int kStepChanPerBlock = kStepThreads / 4;   // 64 channels, four threads each
 
 struct StepParams {
     float* state;
@@ -33,7 +32,7 @@ struct StepParams {
     const void* z;
     void* y;
     const float* bias;
-    int64_t channels;   // batch * d
+    int64_t batch;
     int d;
     int softplus;
 };
@@ -52,65 +51,71 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
     v[2] = __uint_as_float(w.y << 16); v[3] = __uint_as_float(w.y & 0xffff0000u);
 }
 
+// Grid: x over blocks of kStepChanPerBlock channels of one batch row,
+// y over batch rows (strided when batch exceeds the grid's y extent).
 template <typename IO>
 __global__ void __launch_bounds__(kStepThreads) ss_step_kernel(const __grid_constant__ StepParams p) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
     const int q = threadIdx.x & 3;   // states 4q .. 4q+3
-    const int64_t base = static_cast<int64_t>(blockIdx.x) * kStepChanPerBlock + (threadIdx.x >> 2);
-
-    int64_t cs[kStepCPT];
-    bool valid[kStepCPT];
-    float4 h4[kStepCPT];
-    float uu[kStepCPT], xr[kStepCPT], zz[kStepCPT];
+    const int ch = blockIdx.x * kStepChanPerBlock + (threadIdx.x >> 2);
+    const bool valid = ch < p.d;
+    const int chs = valid ? ch : 0;
+    float Av[4];
+    load4<float>(p.A + static_cast<int64_t>(chs) * 16 + 4 * q, Av);
+    const float Dv = (valid && p.D) ? __ldg(p.D + chs) : 0.f;
+    const float bv = (valid && p.bias) ? __ldg(p.bias + chs) : 0.f;
+    // Two batch rows per iteration, all their loads issued before the math.
+    constexpr int R = 2;
+    for (int64_t b0 = blockIdx.y; b0 < p.batch; b0 += static_cast<int64_t>(R) * gridDim.y) {
+        int64_t cs[R];
+        bool ok[R];
+        float4 h4[R];
+        float uu[R], xr[R], zz[R], Bv[R][4], Cv[R][4];
 #pragma unroll
-    for (int k = 0; k < kStepCPT; ++k) {
-        const int64_t chan = base + k * (kStepThreads / 4);
-        valid[k] = chan < p.channels;
-        cs[k] = valid[k] ? chan : 0;
-        h4[k] = valid[k] ? *(reinterpret_cast<const float4*>(p.state + cs[k] * 16) + q)
-                         : make_float4(0.f, 0.f, 0.f, 0.f);
-        uu[k] = valid[k] ? to_f32(static_cast<const IO*>(p.u)[cs[k]]) : 0.f;
-        xr[k] = valid[k] ? to_f32(static_cast<const IO*>(p.delta)[cs[k]]) : 0.f;
-        zz[k] = (valid[k] && p.z) ? to_f32(static_cast<const IO*>(p.z)[cs[k]]) : 0.f;
-    }
-#pragma unroll
-    for (int k = 0; k < kStepCPT; ++k) {
-        const int64_t b = cs[k] / p.d;
-        const int ch = static_cast<int>(cs[k] % p.d);
-        float Bv[4], Cv[4], Av[4];
-        load4<IO>(static_cast<const IO*>(p.B) + b * 16 + 4 * q, Bv);
-        load4<IO>(static_cast<const IO*>(p.C) + b * 16 + 4 * q, Cv);
-        load4<float>(p.A + static_cast<int64_t>(ch) * 16 + 4 * q, Av);
-        const float Dv = p.D ? __ldg(p.D + ch) : 0.f;
-        const float bv = p.bias ? __ldg(p.bias + ch) : 0.f;
-        // λ = Δ / ln 2 on the fast path (decay 2^(λ A), Δ u = λ (ln 2 u)); Δ itself otherwise.
-        float lam, dscale;
-        if (FAST) {
-            const float y2 = fmaf(xr[k], kLog2e, bv * kLog2e);
-            lam = p.softplus ? softplus_log2_fast(y2) : y2;
-            dscale = kLn2;
-        } else {
-            const float x = xr[k] + bv;
-            lam = p.softplus ? softplus_accurate(x) : x;
-            dscale = 1.0f;
+        for (int r = 0; r < R; ++r) {
+            const int64_t b = b0 + static_cast<int64_t>(r) * gridDim.y;
+            ok[r] = valid && b < p.batch;
+            const int64_t bs = b < p.batch ? b : 0;
+            cs[r] = bs * p.d + chs;
+            h4[r] = ok[r] ? *(reinterpret_cast<const float4*>(p.state + cs[r] * 16) + q)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            uu[r] = ok[r] ? to_f32(static_cast<const IO*>(p.u)[cs[r]]) : 0.f;
+            xr[r] = ok[r] ? to_f32(static_cast<const IO*>(p.delta)[cs[r]]) : 0.f;
+            zz[r] = (ok[r] && p.z) ? to_f32(static_cast<const IO*>(p.z)[cs[r]]) : 0.f;
+            load4<IO>(static_cast<const IO*>(p.B) + bs * 16 + 4 * q, Bv[r]);
+            load4<IO>(static_cast<const IO*>(p.C) + bs * 16 + 4 * q, Cv[r]);
         }
-        const float du = lam * (dscale * uu[k]);
-        float hv[4] = {h4[k].x, h4[k].y, h4[k].z, h4[k].w};
-        float acc = 0.f;
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            const float a = FAST ? ex2_approx(lam * Av[m]) : expf(lam * Av[m]);
-            hv[m] = fmaf(a, hv[m], du * Bv[m]);
-            acc = fmaf(Cv[m], hv[m], acc);
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (valid[k]) {
-            *(reinterpret_cast<float4*>(p.state + cs[k] * 16) + q) = make_float4(hv[0], hv[1], hv[2], hv[3]);
-            if (q == 0) {
-                float yv = fmaf(Dv, uu[k], acc);
-                if (p.z) yv *= FAST ? silu_tanh(zz[k]) : silu_accurate(zz[k]);
-                static_cast<IO*>(p.y)[cs[k]] = from_f32<IO>(yv);
+        for (int r = 0; r < R; ++r) {
+            // λ = Δ / ln 2 on the fast path (decay 2^(λ A), Δ u = λ (ln 2 u)); Δ itself otherwise.
+            float lam, dscale;
+            if (FAST) {
+                const float y2 = fmaf(xr[r], kLog2e, bv * kLog2e);
+                lam = p.softplus ? softplus_log2_fast(y2) : y2;
+                dscale = kLn2;
+            } else {
+                const float x = xr[r] + bv;
+                lam = p.softplus ? softplus_accurate(x) : x;
+                dscale = 1.0f;
+            }
+            const float du = lam * (dscale * uu[r]);
+            float hv[4] = {h4[r].x, h4[r].y, h4[r].z, h4[r].w};
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float a = FAST ? ex2_approx(lam * Av[m]) : expf(lam * Av[m]);
+                hv[m] = fmaf(a, hv[m], du * Bv[r][m]);
+                acc = fmaf(Cv[r][m], hv[m], acc);
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            if (ok[r]) {
+                *(reinterpret_cast<float4*>(p.state + cs[r] * 16) + q) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+                if (q == 0) {
+                    float yv = fmaf(Dv, uu[r], acc);
+                    if (p.z) yv *= FAST ? silu_tanh(zz[r]) : silu_accurate(zz[r]);
+                    static_cast<IO*>(p.y)[cs[r]] = from_f32<IO>(yv);
+                }
             }
         }
     }
