@@ -114,6 +114,28 @@ def aggregate_value(world, per_rank_bytes, steps, ms_max):
     return world * per_rank_bytes * steps / (ms_max * 1e-3) / 1e9
 
 
+# FP32 lane operations the forward kernel issues per channel-timestep on the
+# structured-A path, counted from its source (both threads of a channel pair):
+# 4 decay exponents (λa, λa·b in each thread), 16 ladder products for the 16
+# decays, 16 Δu·B products, 16 state FMAs, 16 readout products, 6 pair-sum
+# reductions, and 9 scalar operations of the step's own (softplus argument,
+# 1 + 2^y, Δu, D u, two for the gate, three for the output).  ncu's FMA-pipe
+# activity on the 2.8B-shaped layer (47 %) agrees with this count.
+FP32_OPS_PER_CH_TS = 83
+
+
+def alu_roofline(torch, device, ch_ts_per_s, clock_summary):
+    """The forward kernel against the FP32 pipe: 128 lanes per SM (sm_100)
+    x SMs x the SM clock seen during the timed region (max clock if unsampled)."""
+    props = torch.cuda.get_device_properties(device)
+    mhz = (clock_summary or {}).get("sm_mhz") or (clock_summary or {}).get("sm_max_mhz") or 1965.0
+    peak = 128 * props.multi_processor_count * mhz * 1e6 / 1e12
+    achieved = ch_ts_per_s * FP32_OPS_PER_CH_TS / 1e12
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "T FP32 lane-ops/s",
+            "frac": achieved / peak, "ops_per_ch_ts": FP32_OPS_PER_CH_TS,
+            "peak_kind": f"128 FP32 lanes/SM x {props.multi_processor_count} SMs x {mhz:.0f} MHz"}
+
+
 class ClockSampler:
     """Samples SM clock and throttle reasons via NVML in a background thread."""
     REASONS = {
@@ -438,6 +460,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": profiled_traffic(cfg.name),
                          "peak_kind": f"{peak_kind} copy bandwidth", "kernel": "ss_fwd_kernel"},
+            "roofline_alu": alu_roofline(torch, device, cfg.ch_ts / (step_ms * 1e-3), clocks.summary()),
             "e2e": e2e,
             "gpu_launches": args.steps,
             "clocks": clocks.summary(),
