@@ -46,6 +46,8 @@ def _lib():
             fn = getattr(lib, name)
             fn.argtypes = step_args
             fn.restype = ctypes.c_int
+        lib.ss_oracle_bwd_f64.argtypes = [_DP] * 18 + [_I64, _I64, _I64, _I64, ctypes.c_int]
+        lib.ss_oracle_bwd_f64.restype = ctypes.c_int
         lib.ss_oracle_set_mutation.argtypes = [ctypes.c_int]
         lib.ss_oracle_get_mutation.restype = ctypes.c_int
         lib.ss_oracle_max_threads.restype = ctypes.c_int
@@ -142,6 +144,35 @@ def step(state, u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus=Tru
     return st, y
 
 
+def bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, dlast=None, softplus=True):
+    """Backward of fwd() in float64: gradients of J = Σ dy·y + Σ dlast·last_state.
+
+    Returns a dict with du, ddelta, dz [b,L,d] (dz only with z), dB, dC [b,L,N],
+    dA [d,N], dD [d] (only with D) and dbias [d] (only with delta_bias)."""
+    (batch, L, d, N), keep, p = _prep_fwd(u, delta, A, B, C, D, z, delta_bias)
+    dya, dyp = _arr(dy, (batch, L, d))
+    dla, dlp = _arr(dlast, (batch, d, N))
+    out = {"du": np.empty((batch, L, d)), "ddelta": np.empty((batch, L, d)),
+           "dA": np.empty((d, N)), "dB": np.empty((batch, L, N)), "dC": np.empty((batch, L, N))}
+    if D is not None:
+        out["dD"] = np.empty((d,))
+    if z is not None:
+        out["dz"] = np.empty((batch, L, d))
+    if delta_bias is not None:
+        out["dbias"] = np.empty((d,))
+
+    def op(k):
+        return out[k].ctypes.data_as(_DP) if k in out else _null()
+
+    rc = _lib().ss_oracle_bwd_f64(p[0], p[1], p[2], p[3], p[4], p[5], p[6], p[7], dyp, _ptr(dlp),
+                                  op("du"), op("ddelta"), op("dA"), op("dB"), op("dC"), op("dD"),
+                                  op("dz"), op("dbias"), batch, L, d, N, int(bool(softplus)))
+    if rc != 0:
+        raise ValueError(f"oracle bwd rejected sizes (rc={rc})")
+    del keep, dya, dla
+    return out
+
+
 def set_mutation(m: int) -> None:
     """Test-only: plant deliberate mistake number m (0 restores the oracle)."""
     _lib().ss_oracle_set_mutation(int(m))
@@ -163,7 +194,7 @@ def library_path() -> str:
     return _build.LIB
 
 
-__all__ = ["fwd", "fwd_chunked", "step", "set_mutation", "get_mutation",
+__all__ = ["fwd", "fwd_chunked", "step", "bwd", "set_mutation", "get_mutation",
            "max_threads", "set_threads", "library_path"]
 
 if os.environ.get("SS_ORACLE_THREADS"):

@@ -49,11 +49,14 @@
  * Parity pins (tests/test_oracle_pins.py): closed form at L = 1, LTI
  * reduction to a direct convolution, linearity in u, chunked = sequential,
  * causality, channel independence, limiting cases, a hand-derived worked
- * example, and step-by-step decode equivalence.
+ * example, and step-by-step decode equivalence.  The backward (adjoint) at
+ * the end of this file is pinned by central finite differences of the
+ * forward (tests/test_oracle_bwd_pins.py).
  */
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 #ifdef _OPENMP
 #include <omp.h>
 #endif
@@ -365,4 +368,129 @@ int ss_oracle_fwd_chunked_f64(const double* u, const double* delta, const double
         }
     }
     return 0;
+}
+
+/* ---------------------------------------------------------------------------
+ * Backward of the forward scan, double precision (reverse mode by hand).
+ *
+ * Given the gradient dy = ∂J/∂y [batch, L, d] of a scalar J, and optionally
+ * dlast = ∂J/∂last_state [batch, d, N], returns ∂J/∂ of every input:
+ *   du, ddelta, dz : [batch, L, d]     (ddelta is with respect to Δ_raw)
+ *   dB, dC         : [batch, L, N]     (summed over channels)
+ *   dA             : [d, N]            (summed over batch and time)
+ *   dD, dbias      : [d]               (summed over batch and time)
+ * Outputs for absent optional inputs (D, z, bias) are left untouched and
+ * may be NULL.
+ *
+ * For each (b, ch) the forward recurrence is run once, keeping x_t (the
+ * softplus input), Δ_t, the states h_t and the pre-gate output s_t.  Then
+ * time runs backwards with g_n = ∂J/∂h_t,n, starting from dlast:
+ *   ds   = dy_t · gate(z_t)                         (y = s · gate)
+ *   dz_t = dy_t · s_t · gate'(z_t),  gate'(z) = σ(z) (1 + z (1 - σ(z)))
+ *   g_n += ds · C_t,n,      dC_t,n += ds · h_t,n    (s = Σ_n C h + D u)
+ *   dD  += ds · u_t,        du_t    = ds · D
+ *   with a_n = exp(Δ A_n) and the previous state h_{t-1}:
+ *   dB_t,n += g_n Δ u_t,    du_t   += Σ_n g_n Δ B_t,n
+ *   dΔ      = Σ_n g_n (a_n A_n h_{t-1},n + B_t,n u_t)
+ *   dA_n   += g_n a_n Δ h_{t-1},n
+ *   g_n     = a_n g_n                                (h_t = a h_{t-1} + ...)
+ *   ddelta_t = dΔ · softplus'(x_t) (σ(x); 1 on the identity branch),
+ *   dbias   += ddelta_t.
+ * Channels run in parallel; the sums over channels (dB, dC) use atomic adds.
+ * Test-only mutations 10..12 plant mistakes in this adjoint:
+ *   10: softplus derivative dropped;  11: dA uses h_t instead of h_{t-1};
+ *   12: the adjoint state is not decayed between steps.
+ * Returns 0, or -1 for unsupported sizes / allocation failure.
+ * ------------------------------------------------------------------------- */
+int ss_oracle_bwd_f64(const double* u, const double* delta, const double* delta_bias,
+                      const double* A, const double* B, const double* C,
+                      const double* D, const double* z, const double* dy, const double* dlast,
+                      double* du, double* ddelta, double* dA, double* dB, double* dC,
+                      double* dD, double* dz, double* dbias,
+                      int64_t batch, int64_t L, int64_t d, int64_t N, int softplus)
+{
+    if (N < 1 || N > 256 || batch < 0 || L < 0 || d < 0) return -1;
+    for (int64_t i = 0; i < d * N; ++i) dA[i] = 0.0;
+    for (int64_t i = 0; i < batch * L * N; ++i) { dB[i] = 0.0; dC[i] = 0.0; }
+    if (D && dD) for (int64_t i = 0; i < d; ++i) dD[i] = 0.0;
+    if (delta_bias && dbias) for (int64_t i = 0; i < d; ++i) dbias[i] = 0.0;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t ch = 0; ch < d; ++ch) {
+        double* hs = (double*)malloc((size_t)(L + 1) * (size_t)N * sizeof(double));
+        double* xs = (double*)malloc((size_t)(L + 1) * 3 * sizeof(double));
+        if (!hs || !xs) {
+            free(hs);
+            free(xs);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        for (int64_t b = 0; b < batch; ++b) {
+            /* forward, keeping h_t at hs[(t + 1) N .. ], h_{-1} = 0 at hs[0 .. N) */
+            for (int64_t n = 0; n < N; ++n) hs[n] = 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const int64_t i = (b * L + t) * d + ch;
+                const int64_t bc = (b * L + t) * N;
+                const double x = delta[i] + (delta_bias ? delta_bias[ch] : 0.0);
+                const double dt = softplus ? softplus_d(x) : x;
+                const double* hp = hs + t * N;
+                double* hn = hs + (t + 1) * N;
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    hn[n] = exp(dt * A[ch * N + n]) * hp[n] + dt * B[bc + n] * u[i];
+                    acc += C[bc + n] * hn[n];
+                }
+                xs[3 * t] = x;
+                xs[3 * t + 1] = dt;
+                xs[3 * t + 2] = acc + (D ? D[ch] * u[i] : 0.0);   /* s_t */
+            }
+            /* backward */
+            double g[256];
+            for (int64_t n = 0; n < N; ++n) g[n] = dlast ? dlast[(b * d + ch) * N + n] : 0.0;
+            double dD_acc = 0.0, db_acc = 0.0;
+            for (int64_t t = L - 1; t >= 0; --t) {
+                const int64_t i = (b * L + t) * d + ch;
+                const int64_t bc = (b * L + t) * N;
+                const double x = xs[3 * t], dt = xs[3 * t + 1], s = xs[3 * t + 2];
+                const double* hp = hs + t * N;         /* h_{t-1} */
+                const double* hc = hs + (t + 1) * N;   /* h_t */
+                double ds = dy[i];
+                if (z) {
+                    const double sig = 1.0 / (1.0 + exp(-z[i]));
+                    ds = dy[i] * z[i] * sig;
+                    dz[i] = dy[i] * s * sig * (1.0 + z[i] * (1.0 - sig));
+                }
+                double du_v = 0.0;
+                if (D) {
+                    dD_acc += ds * u[i];
+                    du_v = ds * D[ch];
+                }
+                double dDelta = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double an = A[ch * N + n];
+                    const double a = exp(dt * an);
+                    g[n] += ds * C[bc + n];
+#pragma omp atomic
+                    dC[bc + n] += ds * hc[n];
+#pragma omp atomic
+                    dB[bc + n] += g[n] * dt * u[i];
+                    du_v += g[n] * dt * B[bc + n];
+                    dDelta += g[n] * (a * an * hp[n] + B[bc + n] * u[i]);
+                    dA[ch * N + n] += g[n] * a * dt * (g_mutation == 11 ? hc[n] : hp[n]);
+                    if (g_mutation != 12) g[n] *= a;
+                }
+                du[i] = du_v;
+                double dx = dDelta;
+                if (softplus && g_mutation != 10) dx = x > 20.0 ? dDelta : dDelta / (1.0 + exp(-x));
+                ddelta[i] = dx;
+                db_acc += dx;
+            }
+            if (D && dD) dD[ch] += dD_acc;
+            if (delta_bias && dbias) dbias[ch] += db_acc;
+        }
+        free(hs);
+        free(xs);
+    }
+    return failed ? -1 : 0;
 }
