@@ -1,7 +1,7 @@
 /*
  * selscan.h -- C ABI of libselscan, the B200 (sm_100a) selective-scan library.
  *
- * Two operations, both from the selective state-space model of Mamba:
+ * Three operations, all from the selective state-space model of Mamba:
  *
  *   ss_fwd   the forward scan over a whole sequence ("Algorithm 2" selective
  *            SSM of the mamba README, Usage > Selective SSM; equations of
@@ -16,6 +16,11 @@
  *            function of the Mamba tutorial, §"state management", and the
  *            "constant memory per token" property of the model-architecture
  *            page).
+ *   ss_bwd   the gradients of ss_fwd's inputs from the gradient of its outputs
+ *            (the models are trained and fine-tuned with gradient
+ *            checkpointing: "Mamba 7.9.1" article §5.3-5.4; model-architecture
+ *            page, "Common issues"); reverse-mode differentiation of the same
+ *            recurrence, recomputing the forward states from checkpoints.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -135,6 +140,43 @@ SS_API int ss_fwd(const void* u, const void* delta, const float* delta_bias, con
 SS_API int ss_step(float* state, const void* u, const void* delta, const float* A, const void* B,
             const void* C, const float* D, const void* z, void* y, const float* delta_bias,
             uint32_t flags, const ss_dims* dims, const ss_launch* launch);
+
+/* ss_bwd -- backward of ss_fwd: given dy = dJ/dy and optionally
+ * dlast_state = dJ/dlast_state for a scalar J, writes dJ/d(input) for every
+ * input of ss_fwd with the same u, delta, delta_bias, A, B, C, D, z and flags
+ * (SS_BF16, SS_DELTA_SOFTPLUS, SS_SYNC_CHECK).  With g_n = dJ/dh_t,n run
+ * backwards in time from dlast_state:
+ *   ds = dy gate(z),  dz = dy s gate'(z)  (s = Σ_n C h + D u, gate = z σ(z)),
+ *   g += ds C,  dC += ds h_t,  dB += g Δ u,  du = ds D + Σ_n g Δ B,
+ *   dΔ = Σ_n g (exp(Δ A) A h_{t-1} + B u),  dA += g exp(Δ A) Δ h_{t-1},
+ *   g <- exp(Δ A) g,  ddelta = dΔ softplus'(Δraw + bias),  ddelta_bias += ddelta.
+ * Inputs: as ss_fwd, plus
+ *   dy           [batch, seqlen, d_inner], the element type of u
+ *   dlast_state  [batch, d_inner, d_state] fp32, or NULL (zero)
+ * Outputs (all written; the accumulated ones are zeroed by the call first):
+ *   du, ddelta, dz  [batch, seqlen, d_inner], the element type of u
+ *                   (ddelta is the gradient with respect to the raw Δ;
+ *                   dz must be non-NULL exactly when z is)
+ *   dA              [d_inner, d_state] fp32 (summed over batch and time)
+ *   dB, dC          [batch, seqlen, d_state] fp32 (summed over channels)
+ *   dD, ddelta_bias [d_inner] fp32 (summed over batch and time), or NULL to
+ *                   skip; non-NULL dD needs D, non-NULL ddelta_bias needs
+ *                   delta_bias
+ * Workspace: launch->workspace of at least ss_bwd_workspace_bytes(dims)
+ * bytes (forward-state checkpoints every 64 steps), 16-byte aligned, else
+ * SS_ERR_WORKSPACE.  The sums over channels, batch and time use float
+ * atomic adds, so the last bits of dA, dB, dC, dD and ddelta_bias depend on
+ * the order the hardware applies them in.  One CTA scans a (batch, 64
+ * channel) block over the whole sequence; there is no time chunking.
+ * Errors: as ss_fwd (SS_ERR_INVALID_ARG for a NULL required pointer, a
+ * misaligned pointer or dz/z mismatch). */
+SS_API int ss_bwd(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+                  const void* C, const float* D, const void* z, const void* dy, const float* dlast_state,
+                  void* du, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+                  float* ddelta_bias, uint32_t flags, const ss_dims* dims, const ss_launch* launch);
+
+/* Workspace bytes ss_bwd needs for these sizes (0 for invalid dims). */
+SS_API size_t ss_bwd_workspace_bytes(const ss_dims* dims, uint32_t flags);
 
 /* Workspace bytes ss_fwd needs for these sizes, flags and chunk length
  * (chunk_len 0: the library's own choice, the same one ss_fwd makes):

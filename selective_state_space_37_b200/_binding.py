@@ -33,7 +33,7 @@ D_STATE = 16
 
 # Every symbol include/selscan.h declares.
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
-            "ss_status_string", "ss_version", "ss_fwd_noalloc")
+            "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes")
 
 
 class ss_dims(ctypes.Structure):
@@ -90,6 +90,12 @@ def lib():
         L.ss_fwd_noalloc.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, vp, f32p, ctypes.c_uint32,
                                      ctypes.POINTER(ss_dims), vp]
         L.ss_fwd_noalloc.restype = ctypes.c_int
+        L.ss_bwd.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, vp, f32p, vp, vp, f32p, f32p, f32p,
+                             f32p, vp, f32p, ctypes.c_uint32, ctypes.POINTER(ss_dims),
+                             ctypes.POINTER(ss_launch)]
+        L.ss_bwd.restype = ctypes.c_int
+        L.ss_bwd_workspace_bytes.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32]
+        L.ss_bwd_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -202,6 +208,65 @@ def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, y=None, last_s
     if rc != SS_OK:
         raise SelscanError(rc, "ss_fwd")
     return y, last_state
+
+
+def bwd_workspace_bytes(batch, seqlen, d_inner, bf16=True, d_state=D_STATE):
+    dims = ss_dims(batch, seqlen, d_inner, d_state)
+    return int(lib().ss_bwd_workspace_bytes(ctypes.byref(dims), SS_BF16 if bf16 else 0))
+
+
+def ss_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, dlast_state=None, *,
+           softplus=True, grads=None, workspace=None, stream=None, sync_check=False):
+    """Backward of ss_fwd through libselscan's ss_bwd.
+
+    Same inputs as ss_fwd plus dy [batch, L, d_inner] (the element type of u)
+    and dlast_state [batch, d_inner, 16] fp32 or None.  Returns a dict with
+    du, ddelta, dz (element type of u; dz only with z), dA [d_inner, 16],
+    dB, dC [batch, L, 16], dD and ddelta_bias [d_inner] (fp32; only with D /
+    delta_bias).  `grads` may supply preallocated output tensors by name.
+    """
+    if u.dim() != 3:
+        raise ValueError("u must be [batch, L, d_inner]")
+    batch, L, d = u.shape
+    dev = u.device
+    if dev.type != "cuda":
+        raise ValueError("ss_bwd runs on CUDA tensors only")
+    io = u.dtype
+    for t, nm, shp in ((u, "u", (batch, L, d)), (delta, "delta", (batch, L, d)),
+                       (z, "z", (batch, L, d)), (dy, "dy", (batch, L, d)),
+                       (B, "B", (batch, L, D_STATE)), (C, "C", (batch, L, D_STATE))):
+        _check(t, nm, shp, io, dev)
+    _check(A, "A", (d, D_STATE), torch.float32, dev)
+    _check(D, "D", (d,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (d,), torch.float32, dev)
+    _check(dlast_state, "dlast_state", (batch, d, D_STATE), torch.float32, dev)
+    g = dict(grads or {})
+    shapes = {"du": ((batch, L, d), io), "ddelta": ((batch, L, d), io), "dA": ((d, D_STATE), torch.float32),
+              "dB": ((batch, L, D_STATE), torch.float32), "dC": ((batch, L, D_STATE), torch.float32)}
+    if z is not None:
+        shapes["dz"] = ((batch, L, d), io)
+    if D is not None:
+        shapes["dD"] = ((d,), torch.float32)
+    if delta_bias is not None:
+        shapes["ddelta_bias"] = ((d,), torch.float32)
+    for k, (shp, dt) in shapes.items():
+        if k not in g:
+            g[k] = torch.empty(shp, dtype=dt, device=dev)
+        _check(g[k], k, shp, dt, dev)
+    flags = _io_flag(u) | (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
+    sh = _stream_handle(stream, dev)
+    dims = ss_dims(batch, L, d, D_STATE)
+    need = int(lib().ss_bwd_workspace_bytes(ctypes.byref(dims), flags))
+    if workspace is None:
+        workspace = workspace_for(need, dev, sh)
+    launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(), 0, 0)
+    rc = lib().ss_bwd(_ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                      _ptr(dy), _ptr(dlast_state), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]),
+                      _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g.get("dD")), _ptr(g.get("dz")),
+                      _ptr(g.get("ddelta_bias")), flags, ctypes.byref(dims), ctypes.byref(launch))
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_bwd")
+    return {k: g[k] for k in shapes}
 
 
 def ss_check(workspace, stream=None, device=None):

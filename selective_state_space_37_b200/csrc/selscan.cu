@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "../../include/selscan.h"
+#include "bwd.cuh"
 #include "fwd.cuh"
 #include "step.cuh"
 
@@ -187,6 +188,29 @@ int validate_dims(const ss_dims* dims, bool need_seqlen) {
     return SS_OK;
 }
 
+// Backward: forward-state checkpoints, [batch][ceil(L / kSeg)][d][kN] fp32.
+size_t bwd_workspace(const ss_dims* dims) {
+    const int64_t nseg = ceil_div(std::max<int64_t>(dims->seqlen, 1), kSeg);
+    return static_cast<size_t>(dims->batch * nseg * dims->d_inner) * kN * sizeof(float);
+}
+
+template <typename IO>
+int launch_bwd(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
+    auto kern = ss_bwd_kernel<IO>;
+    const size_t smem = sizeof(BwdSmem);
+    static bool attr_set[kMaxDevices] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+            return SS_ERR_CUDA;
+        if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
+    }
+    kern<<<static_cast<unsigned>(ctas), kBwdCh, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
 // ------------------------------------------------ allocation-free entry point
 // Workspace of ss_fwd_noalloc: one array in device memory per device that
 // loads this library, kept until the process exits.
@@ -348,6 +372,65 @@ int ss_step(float* state, const void* u, const void* delta, const float* A, cons
     else
         ss_step_kernel<float><<<grid, kStepThreads, 0, stream>>>(p);
     if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+    if (flags & SS_SYNC_CHECK) {
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
+    }
+    return SS_OK;
+}
+
+size_t ss_bwd_workspace_bytes(const ss_dims* dims, uint32_t flags) {
+    (void)flags;
+    if (validate_dims(dims, true) != SS_OK) return 0;
+    return bwd_workspace(dims);
+}
+
+int ss_bwd(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+           const void* C, const float* D, const void* z, const void* dy, const float* dlast_state,
+           void* du, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
+           float* ddelta_bias, uint32_t flags, const ss_dims* dims, const ss_launch* launch) {
+    int rc = validate_dims(dims, true);
+    if (rc != SS_OK) return rc;
+    if (!launch || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
+    if ((z == nullptr) != (dz == nullptr)) return SS_ERR_INVALID_ARG;
+    if ((dD && !D) || (ddelta_bias && !delta_bias)) return SS_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, d = dims->d_inner;
+    if (batch == 0 || d == 0) return SS_OK;
+    // Pointers to per-token tensors are not needed (and may be NULL) when L = 0.
+    if (!A || !dA || (L > 0 && (!u || !delta || !B || !C || !dy || !du || !ddelta || !dB || !dC)))
+        return SS_ERR_INVALID_ARG;
+    const void* ptrs[] = {u, delta, delta_bias, A, B, C, D, z, dy, dlast_state,
+                          du, ddelta, dA, dB, dC, dD, dz, ddelta_bias};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
+    // The summed gradients are accumulated: start them from zero.
+    const size_t bytes_bc = static_cast<size_t>(batch * L) * kN * sizeof(float);
+    if (cudaMemsetAsync(dA, 0, static_cast<size_t>(d) * kN * sizeof(float), stream) != cudaSuccess ||
+        (bytes_bc && cudaMemsetAsync(dB, 0, bytes_bc, stream) != cudaSuccess) ||
+        (bytes_bc && cudaMemsetAsync(dC, 0, bytes_bc, stream) != cudaSuccess) ||
+        (dD && cudaMemsetAsync(dD, 0, static_cast<size_t>(d) * sizeof(float), stream) != cudaSuccess) ||
+        (ddelta_bias && cudaMemsetAsync(ddelta_bias, 0, static_cast<size_t>(d) * sizeof(float), stream) != cudaSuccess))
+        return SS_ERR_CUDA;
+    // With no tokens, last_state = h_{-1} = 0 depends on nothing: every gradient is zero.
+    if (L == 0) return (flags & SS_SYNC_CHECK) ? (cudaStreamSynchronize(stream) == cudaSuccess ? SS_OK : SS_ERR_CUDA)
+                                              : SS_OK;
+    const size_t need = bwd_workspace(dims);
+    if (!launch->workspace || launch->workspace_bytes < need || !aligned16(launch->workspace))
+        return SS_ERR_WORKSPACE;
+    const int64_t nblk = ceil_div(d, kBwdCh);
+    const int64_t ctas = batch * nblk;
+    if (ctas >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+
+    BwdParams p{};
+    p.u = u; p.delta = delta; p.bias = delta_bias; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
+    p.dy = dy; p.dlast = dlast_state;
+    p.du = du; p.ddelta = ddelta; p.dz = dz; p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dbias = ddelta_bias;
+    p.ckpt = static_cast<float*>(launch->workspace);
+    p.L = L; p.batch = static_cast<int>(batch); p.d = static_cast<int>(d);
+    p.nseg = static_cast<int>(ceil_div(L, kSeg)); p.nblk = static_cast<int>(nblk);
+    p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
+    rc = (flags & SS_BF16) ? launch_bwd<__nv_bfloat16>(p, ctas, stream) : launch_bwd<float>(p, ctas, stream);
+    if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
     }

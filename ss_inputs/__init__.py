@@ -18,11 +18,13 @@ table, d_state = 16 as in the README usage example and the deep-dive article
   D             = 1, or N(0, 1) for the 2.8B-shaped layer
   B, C          : [batch, L, N], one group shared by all channels
   I/O dtype     : fp32 for the tiny case, bf16 otherwise; A, D, bias fp32.
+  Backward upstream gradients: dy ~ N(0, 1) in the I/O dtype and
+  dlast_state ~ N(0, 1) fp32.
 """
 from .configs import CONFIGS, FwdConfig, StepConfig, get_config
-from .gen import (fwd_inputs, step_inputs, step_sequence_inputs, general_A,
+from .gen import (bwd_upstream, fwd_inputs, step_inputs, step_sequence_inputs, general_A,
                   to_f64, sample_channels)
 
-__all__ = ["CONFIGS", "FwdConfig", "StepConfig", "get_config", "fwd_inputs",
+__all__ = ["CONFIGS", "FwdConfig", "StepConfig", "get_config", "fwd_inputs", "bwd_upstream",
            "step_inputs", "step_sequence_inputs", "general_A", "to_f64",
            "sample_channels"]

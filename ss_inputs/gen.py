@@ -10,7 +10,8 @@ import math
 import numpy as np
 import torch
 
-_TAGS = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "bias": 6, "D": 7, "A": 8, "state": 9}
+_TAGS = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "bias": 6, "D": 7, "A": 8, "state": 9,
+         "dy": 10, "dlast": 11}
 _SLICE = 1 << 26  # elements drawn per slice when filling a large tensor
 
 
@@ -87,6 +88,15 @@ def fwd_inputs(batch, seqlen, d_inner, d_state=16, dtype="bf16", seed=0, device=
         out["D"] = None
     out["delta_bias"] = delta_bias_init(d_inner, seed, "cpu").to(device) if bias else None
     return out
+
+
+def bwd_upstream(batch, seqlen, d_inner, d_state=16, dtype="bf16", seed=0, device="cpu",
+                 dlast=True):
+    """Upstream gradients of one backward call: dy [batch, seqlen, d_inner] in
+    `dtype` and dlast_state [batch, d_inner, d_state] fp32 (or None), N(0, 1)."""
+    dy = _normal((batch, seqlen, d_inner), 1.0, _torch_dtype(dtype), device, seed, "dy")
+    dl = _normal((batch, d_inner, d_state), 1.0, torch.float32, device, seed, "dlast") if dlast else None
+    return dy, dl
 
 
 def step_inputs(batch, d_inner, d_state=16, dtype="bf16", seed=0, device="cpu", gate=True,
