@@ -163,7 +163,7 @@ SS_API int ss_step(float* state, const void* u, const void* delta, const float* 
  *                   skip; non-NULL dD needs D, non-NULL ddelta_bias needs
  *                   delta_bias
  * Workspace: launch->workspace of at least ss_bwd_workspace_bytes(dims)
- * bytes (forward-state checkpoints every 64 steps), 16-byte aligned, else
+ * bytes (forward-state checkpoints every 32 steps), 16-byte aligned, else
  * SS_ERR_WORKSPACE.  The sums over channels, batch and time use float
  * atomic adds, so the last bits of dA, dB, dC, dD and ddelta_bias depend on
  * the order the hardware applies them in.  One CTA scans a (batch, 64

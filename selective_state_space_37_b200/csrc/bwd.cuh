@@ -39,7 +39,7 @@
 namespace selscan {
 
 constexpr int kBwdCh = 64;          // channels (threads) per CTA
-constexpr int kSeg = 64;            // steps per global checkpoint segment
+constexpr int kSeg = 32;            // steps per global checkpoint segment
 constexpr int kSub = 8;             // steps per shared-memory sub-segment
 constexpr int kNSub = kSeg / kSub;
 constexpr int kNP4 = kN / 4;        // float4 groups of a channel's 16 states
@@ -69,10 +69,15 @@ struct BwdParams {
     int softplus;
 };
 
+template <typename IO>
 struct BwdSmem {
     float4 hsub[kNSub][kNP4][kBwdCh];    // state entering each sub-segment
     float4 hstep[kSub][kNP4][kBwdCh];    // h_t of the current sub-segment
     float bc[kSeg][2 * kN];              // B then C of the segment, fp32
+    IO tu[kSeg][kBwdCh];                 // the segment's u, Δraw, z, dy
+    IO tdt[kSeg][kBwdCh];
+    IO tz[kSeg][kBwdCh];
+    IO tdy[kSeg][kBwdCh];
 };
 
 // Per-channel constants of the backward.
@@ -128,32 +133,44 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
     return v[0];
 }
 
+// Loads the segment's tiles: B and C (fp32) of steps t0 .. t0+nt-1 and, for
+// the block's channels, u and Δraw (and z, dy when `adjoint`).  Every load is
+// independent, so their latencies overlap; rows >= nt are left unset.
 template <typename IO>
-__device__ __forceinline__ float ld_el(const void* base, int64_t i, bool ok) {
-    return ok ? to_f32(static_cast<const IO*>(base)[i]) : 0.0f;
-}
-
-// Loads B and C of steps t0 .. t0+nt-1 into the shared tile (fp32).
-template <typename IO>
-__device__ __forceinline__ void load_bc_tile(BwdSmem& S, const BwdParams& p, int b, int64_t t0, int nt) {
-    for (int i = threadIdx.x; i < kSeg * kN; i += kBwdCh) {
+__device__ __forceinline__ void load_seg(BwdSmem<IO>& S, const BwdParams& p, int b, int blk, int64_t t0, int nt,
+                                         bool adjoint) {
+    for (int i = threadIdx.x; i < nt * kN; i += kBwdCh) {
         const int r = i / kN, n = i % kN;
-        const bool ok = r < nt;
         const int64_t idx = (static_cast<int64_t>(b) * p.L + t0 + r) * kN + n;
-        S.bc[r][n] = ld_el<IO>(p.B, idx, ok);
-        S.bc[r][kN + n] = ld_el<IO>(p.C, idx, ok);
+        S.bc[r][n] = to_f32(static_cast<const IO*>(p.B)[idx]);
+        S.bc[r][kN + n] = to_f32(static_cast<const IO*>(p.C)[idx]);
+    }
+    const int c = threadIdx.x;
+    const int64_t ch = static_cast<int64_t>(blk) * kBwdCh + c;
+    const bool ok = ch < p.d;
+    const IO zero = from_f32<IO>(0.0f);
+    for (int r = 0; r < nt; ++r) {
+        const int64_t i = (static_cast<int64_t>(b) * p.L + t0 + r) * p.d + ch;
+        S.tu[r][c] = ok ? static_cast<const IO*>(p.u)[i] : zero;
+        S.tdt[r][c] = ok ? static_cast<const IO*>(p.delta)[i] : zero;
+        if (adjoint) {
+            S.tz[r][c] = (ok && p.z) ? static_cast<const IO*>(p.z)[i] : zero;
+            S.tdy[r][c] = ok ? static_cast<const IO*>(p.dy)[i] : zero;
+        }
     }
 }
 
-// One forward step of this thread's channel: h ← a h + Δ B u.
+// One forward step (row r of the segment) of this thread's channel:
+// h ← a h + Δ B u.
 template <typename IO, bool FAST, bool STRUCT>
-__device__ __forceinline__ void fwd_step(const BwdSmem& S, const BwdParams& p, const BwdChan& cp, int64_t i,
-                                         int r, float (&h)[kN]) {
-    const float x = ld_el<IO>(p.delta, i, cp.valid) + cp.bias;
+__device__ __forceinline__ void fwd_step(const BwdSmem<IO>& S, const BwdParams& p, const BwdChan& cp, int r,
+                                         float (&h)[kN]) {
+    const int c = threadIdx.x;
+    const float x = to_f32(S.tdt[r][c]) + cp.bias;
     float dt, sig;
     if (p.softplus) softplus_and_sigmoid<FAST>(x, dt, sig);
     else dt = x;
-    const float du = dt * ld_el<IO>(p.u, i, cp.valid);
+    const float du = dt * to_f32(S.tu[r][c]);
     float a[kN];
     decays<FAST, STRUCT>(dt, cp, a);
 #pragma unroll
@@ -178,7 +195,8 @@ __device__ __forceinline__ void load_state(const float4 (&src)[kNP4][kBwdCh], in
 }
 
 template <typename IO, bool STRUCT>
-__device__ __forceinline__ void bwd_item(BwdSmem& S, const BwdParams& p, const BwdChan& cp, int b, int ch) {
+__device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, const BwdChan& cp, int b, int blk,
+                                         int ch) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
     const int tid = threadIdx.x, lane = tid & 31;
     const int64_t d = p.d;
@@ -197,9 +215,9 @@ __device__ __forceinline__ void bwd_item(BwdSmem& S, const BwdParams& p, const B
             for (int q = 0; q < kNP4; ++q) ck[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
         }
         __syncthreads();
-        load_bc_tile<IO>(S, p, b, t0, nt);
+        load_seg<IO>(S, p, b, blk, t0, nt, false);
         __syncthreads();
-        for (int r = 0; r < nt; ++r) fwd_step<IO, FAST, STRUCT>(S, p, cp, (row0 + t0 + r) * d + ch, r, h);
+        for (int r = 0; r < nt; ++r) fwd_step<IO, FAST, STRUCT>(S, p, cp, r, h);
     }
 
     // ---------------------------------------------------------------- pass 1
@@ -215,7 +233,7 @@ __device__ __forceinline__ void bwd_item(BwdSmem& S, const BwdParams& p, const B
         const int nt = static_cast<int>(min(static_cast<int64_t>(kSeg), p.L - t0));
         const int nsub = (nt + kSub - 1) / kSub;
         __syncthreads();
-        load_bc_tile<IO>(S, p, b, t0, nt);
+        load_seg<IO>(S, p, b, blk, t0, nt, true);
         __syncthreads();
         if (cp.valid) {
             const float4* ck =
@@ -234,16 +252,14 @@ __device__ __forceinline__ void bwd_item(BwdSmem& S, const BwdParams& p, const B
             store_state(S.hsub[s], tid, h);
             const int ns = min(kSub, nt - s * kSub);
             for (int j = 0; j < ns; ++j) {
-                const int r = s * kSub + j;
-                fwd_step<IO, FAST, STRUCT>(S, p, cp, (row0 + t0 + r) * d + ch, r, h);
+                fwd_step<IO, FAST, STRUCT>(S, p, cp, s * kSub + j, h);
             }
         }
         for (int s = nsub - 1; s >= 0; --s) {
             const int ns = min(kSub, nt - s * kSub);
             load_state(S.hsub[s], tid, h);
             for (int j = 0; j < ns; ++j) {
-                const int r = s * kSub + j;
-                fwd_step<IO, FAST, STRUCT>(S, p, cp, (row0 + t0 + r) * d + ch, r, h);
+                fwd_step<IO, FAST, STRUCT>(S, p, cp, s * kSub + j, h);
                 store_state(S.hstep[j], tid, h);
             }
             for (int j = ns - 1; j >= 0; --j) {
@@ -254,12 +270,12 @@ __device__ __forceinline__ void bwd_item(BwdSmem& S, const BwdParams& p, const B
                 load_state(S.hstep[j], tid, hc);
                 if (j > 0) load_state(S.hstep[j - 1], tid, hp);
                 else load_state(S.hsub[s], tid, hp);
-                const float x = ld_el<IO>(p.delta, i, cp.valid) + cp.bias;
+                const float x = to_f32(S.tdt[r][tid]) + cp.bias;
                 float dt, sig = 1.0f;
                 if (p.softplus) softplus_and_sigmoid<FAST>(x, dt, sig);
                 else dt = x;
-                const float uv = ld_el<IO>(p.u, i, cp.valid);
-                const float dyv = ld_el<IO>(p.dy, i, cp.valid);
+                const float uv = to_f32(S.tu[r][tid]);
+                const float dyv = to_f32(S.tdy[r][tid]);
                 float a[kN];
                 decays<FAST, STRUCT>(dt, cp, a);
                 // s_t = Σ_n C h_t + D u, then the gate
@@ -270,7 +286,7 @@ __device__ __forceinline__ void bwd_item(BwdSmem& S, const BwdParams& p, const B
                 const float sv = acc.x + acc.y + cp.Dv * uv;
                 float ds = dyv;
                 if (p.z) {
-                    const float zv = ld_el<IO>(p.z, i, cp.valid);
+                    const float zv = to_f32(S.tz[r][tid]);
                     const float sz = FAST ? rcp_approx(1.0f + ex2_approx(-zv * kLog2e)) : 1.0f / (1.0f + expf(-zv));
                     ds = dyv * zv * sz;
                     if (cp.valid)
@@ -315,7 +331,7 @@ __device__ __forceinline__ void bwd_item(BwdSmem& S, const BwdParams& p, const B
 template <typename IO>
 __global__ void __launch_bounds__(kBwdCh) ss_bwd_kernel(const __grid_constant__ BwdParams p) {
     extern __shared__ __align__(16) unsigned char bwd_smem_raw[];
-    auto& S = *reinterpret_cast<BwdSmem*>(bwd_smem_raw);
+    auto& S = *reinterpret_cast<BwdSmem<IO>*>(bwd_smem_raw);
     const int g = blockIdx.x % p.nblk;
     const int b = blockIdx.x / p.nblk;
     const int ch = g * kBwdCh + threadIdx.x;
@@ -335,9 +351,9 @@ __global__ void __launch_bounds__(kBwdCh) ss_bwd_kernel(const __grid_constant__ 
     cp.Dv = (cp.valid && p.D) ? p.D[ch] : 0.0f;
     const int all_struct = __syncthreads_and(structured ? 1 : 0);
     if (std::is_same<IO, __nv_bfloat16>::value && all_struct)
-        bwd_item<IO, true>(S, p, cp, b, ch);
+        bwd_item<IO, true>(S, p, cp, b, g, ch);
     else
-        bwd_item<IO, false>(S, p, cp, b, ch);
+        bwd_item<IO, false>(S, p, cp, b, g, ch);
 }
 
 }  // namespace selscan

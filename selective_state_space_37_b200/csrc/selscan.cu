@@ -197,7 +197,7 @@ size_t bwd_workspace(const ss_dims* dims) {
 template <typename IO>
 int launch_bwd(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
     auto kern = ss_bwd_kernel<IO>;
-    const size_t smem = sizeof(BwdSmem);
+    const size_t smem = sizeof(BwdSmem<IO>);
     static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
     cudaGetDevice(&dev);
