@@ -13,9 +13,11 @@
 //   dB += g Δ u,  du = ds D + Σ g Δ B,  dΔ = Σ g (a A h_{t-1} + B u),
 //   dA += g a Δ h_{t-1},  g ← a g,  dΔraw = dΔ · softplus'(x),  dbias += dΔraw.
 //
-// Work decomposition: one CTA = (batch b, block of kBwdCh channels), one
-// thread per channel holding its 16 states (8 fp32x2 pairs), the whole
-// sequence in one CTA (no time chunking).  The forward states the adjoint
+// Work decomposition: one CTA = (batch b, block of kBwdCh channels), the
+// whole sequence in one CTA (no time chunking).  Two threads share a channel
+// -- lanes l and l^16 of a warp, each with 8 of its 16 states -- so a warp
+// serves 16 channels; the per-channel sums over states (readout, du, dΔ)
+// take one shuffle each.  The forward states the adjoint
 // needs are recomputed (gradient checkpointing, two levels):
 //   pass 0   -- forward over the whole sequence, writing the state entering
 //               every kSeg-step segment to a global checkpoint buffer;
@@ -24,9 +26,10 @@
 //               sub-segment in shared memory; sub-segments last to first: a
 //               forward pass stores h_t of its kSub steps in shared memory,
 //               then the adjoint runs back over them.
-// dB and dC (sums over channels) are reduced across each warp by a
-// transposing butterfly (31 shuffles leave lane l with value l summed over
-// the warp) and added to global memory with one atomic per lane per step;
+// dB and dC (sums over channels) are reduced across each half-warp by a
+// transposing butterfly (15 shuffles leave lane j of the half with value j
+// summed over its 16 channels) and added to global memory with one atomic
+// per lane per step;
 // dA, dD, dbias accumulate per thread over time and are added at the end.
 // The library zeroes the accumulated outputs before the launch.
 #pragma once
@@ -38,7 +41,9 @@
 
 namespace selscan {
 
-constexpr int kBwdCh = 64;          // channels (threads) per CTA
+constexpr int kBwdCh = 64;          // channels per CTA
+constexpr int kBwdThreads = 2 * kBwdCh;   // two threads per channel
+constexpr int kBH = kN / 2;         // states per thread
 constexpr int kSeg = 32;            // steps per global checkpoint segment
 constexpr int kSub = 8;             // steps per shared-memory sub-segment
 constexpr int kNSub = kSeg / kSub;
@@ -80,12 +85,15 @@ struct BwdSmem {
     IO tdy[kSeg][kBwdCh];
 };
 
-// Per-channel constants of the backward.
+// Per-thread constants of the backward: this thread's channel and half.
 struct BwdChan {
-    float Al[kN];      // A[ch, n] · log2 e (exp(Δ A) = 2^(Δ Al))
-    float A[kN];
-    float al;          // structured path: A[ch, n] = a (n + 1); al = a · log2 e
+    float A[kBH];      // A[ch, 8p + m]
+    float Al[kBH];     // A[ch, 8p + m] · log2 e (exp(Δ A) = 2^(Δ Al))
+    float al;          // structured path (A[ch, n] = a (n + 1)): a · log2 e
+    float alb;         // a (8p + 1) · log2 e: exponent factor of the half's first decay
     float bias, Dv;
+    int c;             // channel within the block
+    int p;             // 0: states 0..7, 1: states 8..15
     bool valid;
 };
 
@@ -102,35 +110,18 @@ __device__ __forceinline__ void softplus_and_sigmoid(float x, float& sp, float& 
     }
 }
 
-// exp(Δ A_n) for the 16 states.
+// exp(Δ A_n) for this thread's 8 states.
 template <bool FAST, bool STRUCT>
-__device__ __forceinline__ void decays(float dt, const BwdChan& cp, float (&a)[kN]) {
+__device__ __forceinline__ void decays(float dt, const BwdChan& cp, float (&a)[kBH]) {
     if (STRUCT) {
         const float r = ex2_approx(dt * cp.al);
-        a[0] = r;
+        a[0] = ex2_approx(dt * cp.alb);   // r^(8p+1)
 #pragma unroll
-        for (int n = 1; n < kN; ++n) a[n] = a[n - 1] * r;
+        for (int m = 1; m < kBH; ++m) a[m] = a[m - 1] * r;
     } else {
 #pragma unroll
-        for (int n = 0; n < kN; ++n) a[n] = FAST ? ex2_approx(dt * cp.Al[n]) : expf(dt * cp.A[n]);
+        for (int m = 0; m < kBH; ++m) a[m] = FAST ? ex2_approx(dt * cp.Al[m]) : expf(dt * cp.A[m]);
     }
-}
-
-// Sum over the warp of v[0..31] (each lane's own 32 values): on return lane
-// l holds the warp's sum of v[l].  Each halving step keeps one half of the
-// values, sends the other to the partner lane, and adds what comes back.
-__device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) {
-        const bool up = (lane & m) != 0;
-#pragma unroll
-        for (int i = 0; i < m; ++i) {
-            const float send = up ? v[i] : v[i + m];
-            const float keep = up ? v[i + m] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, m);
-        }
-    }
-    return v[0];
 }
 
 // Loads the segment's tiles: B and C (fp32) of steps t0 .. t0+nt-1 and, for
@@ -139,17 +130,17 @@ __device__ __forceinline__ float warp_transpose_sum(float (&v)[32], int lane) {
 template <typename IO>
 __device__ __forceinline__ void load_seg(BwdSmem<IO>& S, const BwdParams& p, int b, int blk, int64_t t0, int nt,
                                          bool adjoint) {
-    for (int i = threadIdx.x; i < nt * kN; i += kBwdCh) {
+    for (int i = threadIdx.x; i < nt * kN; i += kBwdThreads) {
         const int r = i / kN, n = i % kN;
         const int64_t idx = (static_cast<int64_t>(b) * p.L + t0 + r) * kN + n;
         S.bc[r][n] = to_f32(static_cast<const IO*>(p.B)[idx]);
         S.bc[r][kN + n] = to_f32(static_cast<const IO*>(p.C)[idx]);
     }
-    const int c = threadIdx.x;
+    const int c = threadIdx.x % kBwdCh;
     const int64_t ch = static_cast<int64_t>(blk) * kBwdCh + c;
     const bool ok = ch < p.d;
     const IO zero = from_f32<IO>(0.0f);
-    for (int r = 0; r < nt; ++r) {
+    for (int r = threadIdx.x / kBwdCh; r < nt; r += kBwdThreads / kBwdCh) {
         const int64_t i = (static_cast<int64_t>(b) * p.L + t0 + r) * p.d + ch;
         S.tu[r][c] = ok ? static_cast<const IO*>(p.u)[i] : zero;
         S.tdt[r][c] = ok ? static_cast<const IO*>(p.delta)[i] : zero;
@@ -160,59 +151,59 @@ __device__ __forceinline__ void load_seg(BwdSmem<IO>& S, const BwdParams& p, int
     }
 }
 
-// One forward step (row r of the segment) of this thread's channel:
+// One forward step (row r of the segment) of this thread's half-channel:
 // h ← a h + Δ B u.
 template <typename IO, bool FAST, bool STRUCT>
 __device__ __forceinline__ void fwd_step(const BwdSmem<IO>& S, const BwdParams& p, const BwdChan& cp, int r,
-                                         float (&h)[kN]) {
-    const int c = threadIdx.x;
-    const float x = to_f32(S.tdt[r][c]) + cp.bias;
+                                         float (&h)[kBH]) {
+    const float x = to_f32(S.tdt[r][cp.c]) + cp.bias;
     float dt, sig;
     if (p.softplus) softplus_and_sigmoid<FAST>(x, dt, sig);
     else dt = x;
-    const float du = dt * to_f32(S.tu[r][c]);
-    float a[kN];
+    const float du = dt * to_f32(S.tu[r][cp.c]);
+    float a[kBH];
     decays<FAST, STRUCT>(dt, cp, a);
+    const float* Bh = &S.bc[r][kBH * cp.p];
 #pragma unroll
-    for (int n = 0; n < kN; n += 2) {
-        const f32x2 hn = fma2(pk2(a[n], a[n + 1]), pk2(h[n], h[n + 1]),
-                              mul2(pk2(du, du), pk2(S.bc[r][n], S.bc[r][n + 1])));
-        h[n] = hn.x;
-        h[n + 1] = hn.y;
+    for (int m = 0; m < kBH; m += 2) {
+        const f32x2 hn = fma2(pk2(a[m], a[m + 1]), pk2(h[m], h[m + 1]), mul2(pk2(du, du), pk2(Bh[m], Bh[m + 1])));
+        h[m] = hn.x;
+        h[m + 1] = hn.y;
     }
 }
 
-__device__ __forceinline__ void store_state(float4 (&dst)[kNP4][kBwdCh], int tid, const float (&h)[kN]) {
-#pragma unroll
-    for (int q = 0; q < kNP4; ++q) dst[q][tid] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+__device__ __forceinline__ void store_state(float4 (&dst)[kNP4][kBwdCh], const BwdChan& cp, const float (&h)[kBH]) {
+    dst[2 * cp.p][cp.c] = make_float4(h[0], h[1], h[2], h[3]);
+    dst[2 * cp.p + 1][cp.c] = make_float4(h[4], h[5], h[6], h[7]);
 }
-__device__ __forceinline__ void load_state(const float4 (&src)[kNP4][kBwdCh], int tid, float (&h)[kN]) {
-#pragma unroll
-    for (int q = 0; q < kNP4; ++q) {
-        const float4 v = src[q][tid];
-        h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
-    }
+__device__ __forceinline__ void load_state(const float4 (&src)[kNP4][kBwdCh], const BwdChan& cp, float (&h)[kBH]) {
+    const float4 v0 = src[2 * cp.p][cp.c], v1 = src[2 * cp.p + 1][cp.c];
+    h[0] = v0.x; h[1] = v0.y; h[2] = v0.z; h[3] = v0.w;
+    h[4] = v1.x; h[5] = v1.y; h[6] = v1.z; h[7] = v1.w;
 }
 
 template <typename IO, bool STRUCT>
 __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, const BwdChan& cp, int b, int blk,
                                          int ch) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
-    const int tid = threadIdx.x, lane = tid & 31;
+    const int j16 = threadIdx.x & 15;                     // lane within the half-warp
     const int64_t d = p.d;
     const int64_t row0 = static_cast<int64_t>(b) * p.L;   // (b, t) row index base
+    const int hp = kBH * cp.p;
+    const bool writer = cp.valid && cp.p == 0;            // stores the per-channel outputs
 
     // ---------------------------------------------------------------- pass 0
-    float h[kN];
+    float h[kBH];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) h[n] = 0.0f;
+    for (int m = 0; m < kBH; ++m) h[m] = 0.0f;
     for (int seg = 0; seg < p.nseg; ++seg) {
         const int64_t t0 = static_cast<int64_t>(seg) * kSeg;
         const int nt = static_cast<int>(min(static_cast<int64_t>(kSeg), p.L - t0));
         if (cp.valid) {
-            float4* ck = reinterpret_cast<float4*>(p.ckpt + ((static_cast<int64_t>(b) * p.nseg + seg) * d + ch) * kN);
-#pragma unroll
-            for (int q = 0; q < kNP4; ++q) ck[q] = make_float4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+            float4* ck =
+                reinterpret_cast<float4*>(p.ckpt + ((static_cast<int64_t>(b) * p.nseg + seg) * d + ch) * kN + hp);
+            ck[0] = make_float4(h[0], h[1], h[2], h[3]);
+            ck[1] = make_float4(h[4], h[5], h[6], h[7]);
         }
         __syncthreads();
         load_seg<IO>(S, p, b, blk, t0, nt, false);
@@ -221,11 +212,11 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
     }
 
     // ---------------------------------------------------------------- pass 1
-    float g[kN], dA_acc[kN];
+    float g[kBH], dA_acc[kBH];
 #pragma unroll
-    for (int n = 0; n < kN; ++n) {
-        g[n] = (p.dlast && cp.valid) ? p.dlast[(static_cast<int64_t>(b) * d + ch) * kN + n] : 0.0f;
-        dA_acc[n] = 0.0f;
+    for (int m = 0; m < kBH; ++m) {
+        g[m] = (p.dlast && cp.valid) ? p.dlast[(static_cast<int64_t>(b) * d + ch) * kN + hp + m] : 0.0f;
+        dA_acc[m] = 0.0f;
     }
     float dD_acc = 0.0f, dbias_acc = 0.0f;
     for (int seg = p.nseg - 1; seg >= 0; --seg) {
@@ -236,124 +227,140 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
         load_seg<IO>(S, p, b, blk, t0, nt, true);
         __syncthreads();
         if (cp.valid) {
-            const float4* ck =
-                reinterpret_cast<const float4*>(p.ckpt + ((static_cast<int64_t>(b) * p.nseg + seg) * d + ch) * kN);
-#pragma unroll
-            for (int q = 0; q < kNP4; ++q) {
-                const float4 v = ck[q];
-                h[4 * q] = v.x; h[4 * q + 1] = v.y; h[4 * q + 2] = v.z; h[4 * q + 3] = v.w;
-            }
+            const float4* ck = reinterpret_cast<const float4*>(
+                p.ckpt + ((static_cast<int64_t>(b) * p.nseg + seg) * d + ch) * kN + hp);
+            const float4 v0 = ck[0], v1 = ck[1];
+            h[0] = v0.x; h[1] = v0.y; h[2] = v0.z; h[3] = v0.w;
+            h[4] = v1.x; h[5] = v1.y; h[6] = v1.z; h[7] = v1.w;
         } else {
 #pragma unroll
-            for (int n = 0; n < kN; ++n) h[n] = 0.0f;
+            for (int m = 0; m < kBH; ++m) h[m] = 0.0f;
         }
-        // sub-checkpoints (each thread touches only its own column)
+        // sub-checkpoints (each thread touches only its own half-column)
         for (int s = 0; s < nsub; ++s) {
-            store_state(S.hsub[s], tid, h);
+            store_state(S.hsub[s], cp, h);
             const int ns = min(kSub, nt - s * kSub);
-            for (int j = 0; j < ns; ++j) {
-                fwd_step<IO, FAST, STRUCT>(S, p, cp, s * kSub + j, h);
-            }
+            for (int j = 0; j < ns; ++j) fwd_step<IO, FAST, STRUCT>(S, p, cp, s * kSub + j, h);
         }
         for (int s = nsub - 1; s >= 0; --s) {
             const int ns = min(kSub, nt - s * kSub);
-            load_state(S.hsub[s], tid, h);
+            load_state(S.hsub[s], cp, h);
             for (int j = 0; j < ns; ++j) {
                 fwd_step<IO, FAST, STRUCT>(S, p, cp, s * kSub + j, h);
-                store_state(S.hstep[j], tid, h);
+                store_state(S.hstep[j], cp, h);
             }
             for (int j = ns - 1; j >= 0; --j) {
                 const int r = s * kSub + j;
                 const int64_t t = t0 + r;
                 const int64_t i = (row0 + t) * d + ch;
-                float hp[kN], hc[kN];
-                load_state(S.hstep[j], tid, hc);
-                if (j > 0) load_state(S.hstep[j - 1], tid, hp);
-                else load_state(S.hsub[s], tid, hp);
-                const float x = to_f32(S.tdt[r][tid]) + cp.bias;
+                float hprev[kBH], hc[kBH];
+                load_state(S.hstep[j], cp, hc);
+                if (j > 0) load_state(S.hstep[j - 1], cp, hprev);
+                else load_state(S.hsub[s], cp, hprev);
+                const float x = to_f32(S.tdt[r][cp.c]) + cp.bias;
                 float dt, sig = 1.0f;
                 if (p.softplus) softplus_and_sigmoid<FAST>(x, dt, sig);
                 else dt = x;
-                const float uv = to_f32(S.tu[r][tid]);
-                const float dyv = to_f32(S.tdy[r][tid]);
-                float a[kN];
+                const float uv = to_f32(S.tu[r][cp.c]);
+                const float dyv = to_f32(S.tdy[r][cp.c]);
+                float a[kBH];
                 decays<FAST, STRUCT>(dt, cp, a);
-                // s_t = Σ_n C h_t + D u, then the gate
-                f32x2 acc = pk2(0.f, 0.f);
+                const float* Bh = &S.bc[r][hp];
+                const float* Ch = &S.bc[r][kN + hp];
+                // s_t = Σ_n C h_t + D u (both halves), then the gate
+                f32x2 acc = mul2(pk2(Ch[0], Ch[1]), pk2(hc[0], hc[1]));
 #pragma unroll
-                for (int n = 0; n < kN; n += 2)
-                    acc = fma2(pk2(S.bc[r][kN + n], S.bc[r][kN + n + 1]), pk2(hc[n], hc[n + 1]), acc);
-                const float sv = acc.x + acc.y + cp.Dv * uv;
+                for (int m = 2; m < kBH; m += 2) acc = fma2(pk2(Ch[m], Ch[m + 1]), pk2(hc[m], hc[m + 1]), acc);
+                const float sh = acc.x + acc.y;
+                const float sv = sh + partner(sh) + cp.Dv * uv;
                 float ds = dyv;
                 if (p.z) {
-                    const float zv = to_f32(S.tz[r][tid]);
+                    const float zv = to_f32(S.tz[r][cp.c]);
                     const float sz = FAST ? rcp_approx(1.0f + ex2_approx(-zv * kLog2e)) : 1.0f / (1.0f + expf(-zv));
                     ds = dyv * zv * sz;
-                    if (cp.valid)
-                        static_cast<IO*>(p.dz)[i] = from_f32<IO>(dyv * sv * sz * (1.0f + zv * (1.0f - sz)));
+                    if (writer) static_cast<IO*>(p.dz)[i] = from_f32<IO>(dyv * sv * sz * (1.0f + zv * (1.0f - sz)));
                 }
                 dD_acc += ds * uv;
-                float duv = ds * cp.Dv, dDelta = 0.0f;
+                float du_h = 0.0f, dD_h = 0.0f;
                 const float dtu = dt * uv;
-                float red[32];
+                float red[2 * kBH];
 #pragma unroll
-                for (int n = 0; n < kN; ++n) {
-                    const float Bn = S.bc[r][n], Cn = S.bc[r][kN + n];
-                    g[n] = fmaf(ds, Cn, g[n]);
-                    red[kN + n] = ds * hc[n];                 // dC contribution
-                    red[n] = g[n] * dtu;                      // dB contribution
-                    duv = fmaf(g[n] * dt, Bn, duv);
-                    const float ah = a[n] * hp[n];
-                    dDelta = fmaf(g[n], fmaf(ah, cp.A[n], Bn * uv), dDelta);
-                    dA_acc[n] = fmaf(g[n] * dt, ah, dA_acc[n]);
-                    g[n] *= a[n];
+                for (int m = 0; m < kBH; ++m) {
+                    g[m] = fmaf(ds, Ch[m], g[m]);
+                    red[kBH + m] = ds * hc[m];                // dC contribution
+                    red[m] = g[m] * dtu;                      // dB contribution
+                    du_h = fmaf(g[m] * dt, Bh[m], du_h);
+                    const float ah = a[m] * hprev[m];
+                    dD_h = fmaf(g[m], fmaf(ah, cp.A[m], Bh[m] * uv), dD_h);
+                    dA_acc[m] = fmaf(g[m] * dt, ah, dA_acc[m]);
+                    g[m] *= a[m];
                 }
-                const float dx = dDelta * sig;
+                const float duv = fmaf(ds, cp.Dv, du_h + partner(du_h));
+                const float dx = (dD_h + partner(dD_h)) * sig;
                 dbias_acc += dx;
-                if (cp.valid) {
+                if (writer) {
                     static_cast<IO*>(p.du)[i] = from_f32<IO>(duv);
                     static_cast<IO*>(p.ddelta)[i] = from_f32<IO>(dx);
                 }
-                const float tot = warp_transpose_sum(red, lane);
-                float* dst = (lane < kN ? p.dB : p.dC) + (row0 + t) * kN + (lane & (kN - 1));
-                atomicAdd(dst, tot);
+                // dB / dC summed over the half-warp's 16 channels: each halving
+                // step keeps one half of the values, sends the other to the
+                // partner lane and adds what comes back; lane j ends with value j.
+#pragma unroll
+                for (int mm = kBH; mm >= 1; mm >>= 1) {
+                    const bool up = (j16 & mm) != 0;
+#pragma unroll
+                    for (int q = 0; q < mm; ++q) {
+                        const float send = up ? red[q] : red[q + mm];
+                        const float keep = up ? red[q + mm] : red[q];
+                        red[q] = keep + __shfl_xor_sync(0xffffffffu, send, mm);
+                    }
+                }
+                float* dst = (j16 < kBH ? p.dB : p.dC) + (row0 + t) * kN + hp + (j16 & (kBH - 1));
+                atomicAdd(dst, red[0]);
             }
         }
     }
     if (cp.valid) {
 #pragma unroll
-        for (int n = 0; n < kN; ++n) atomicAdd(p.dA + static_cast<int64_t>(ch) * kN + n, dA_acc[n]);
-        if (p.dD) atomicAdd(p.dD + ch, dD_acc);
-        if (p.dbias) atomicAdd(p.dbias + ch, dbias_acc);
+        for (int m = 0; m < kBH; ++m) atomicAdd(p.dA + static_cast<int64_t>(ch) * kN + hp + m, dA_acc[m]);
+        if (cp.p == 0) {
+            if (p.dD) atomicAdd(p.dD + ch, dD_acc);
+            if (p.dbias) atomicAdd(p.dbias + ch, dbias_acc);
+        }
     }
 }
 
 template <typename IO>
-__global__ void __launch_bounds__(kBwdCh) ss_bwd_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(kBwdThreads) ss_bwd_kernel(const __grid_constant__ BwdParams p) {
     extern __shared__ __align__(16) unsigned char bwd_smem_raw[];
     auto& S = *reinterpret_cast<BwdSmem<IO>*>(bwd_smem_raw);
-    const int g = blockIdx.x % p.nblk;
+    const int blk = blockIdx.x % p.nblk;
     const int b = blockIdx.x / p.nblk;
-    const int ch = g * kBwdCh + threadIdx.x;
+    const int lane = threadIdx.x & 31;
     BwdChan cp;
+    cp.c = (threadIdx.x >> 5) * 16 + (lane & 15);
+    cp.p = lane >> 4;
+    const int ch = blk * kBwdCh + cp.c;
+    const int hp = kBH * cp.p;
     cp.valid = ch < p.d;
     bool structured = true;
     const float* Arow = p.A + static_cast<int64_t>(cp.valid ? ch : 0) * kN;
     const float a0 = cp.valid ? Arow[0] : -1.0f;
 #pragma unroll
-    for (int n = 0; n < kN; ++n) {
-        cp.A[n] = cp.valid ? Arow[n] : -static_cast<float>(n + 1);
-        cp.Al[n] = cp.A[n] * kLog2e;
-        structured = structured && (cp.A[n] == a0 * static_cast<float>(n + 1));
+    for (int m = 0; m < kBH; ++m) {
+        cp.A[m] = cp.valid ? Arow[hp + m] : -static_cast<float>(hp + m + 1);
+        cp.Al[m] = cp.A[m] * kLog2e;
+        structured = structured && (cp.A[m] == a0 * static_cast<float>(hp + m + 1));
     }
     cp.al = a0 * kLog2e;
+    cp.alb = cp.al * static_cast<float>(hp + 1);
     cp.bias = (cp.valid && p.bias) ? p.bias[ch] : 0.0f;
     cp.Dv = (cp.valid && p.D) ? p.D[ch] : 0.0f;
     const int all_struct = __syncthreads_and(structured ? 1 : 0);
     if (std::is_same<IO, __nv_bfloat16>::value && all_struct)
-        bwd_item<IO, true>(S, p, cp, b, g, ch);
+        bwd_item<IO, true>(S, p, cp, b, blk, ch);
     else
-        bwd_item<IO, false>(S, p, cp, b, g, ch);
+        bwd_item<IO, false>(S, p, cp, b, blk, ch);
 }
 
 }  // namespace selscan

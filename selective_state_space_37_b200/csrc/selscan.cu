@@ -207,7 +207,7 @@ int launch_bwd(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
             return SS_ERR_CUDA;
         if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
     }
-    kern<<<static_cast<unsigned>(ctas), kBwdCh, smem, stream>>>(p);
+    kern<<<static_cast<unsigned>(ctas), kBwdThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
