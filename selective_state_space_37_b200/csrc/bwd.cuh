@@ -153,13 +153,11 @@ __device__ __forceinline__ void load_seg(BwdSmem<IO>& S, const BwdParams& p, int
 
 // One forward step (row r of the segment) of this thread's half-channel:
 // h ← a h + Δ B u.
-template <typename IO, bool FAST, bool STRUCT>
-__device__ __forceinline__ void fwd_step(const BwdSmem<IO>& S, const BwdParams& p, const BwdChan& cp, int r,
-                                         float (&h)[kBH]) {
+template <typename IO, bool FAST, bool STRUCT, bool SP>
+__device__ __forceinline__ void fwd_step(const BwdSmem<IO>& S, const BwdChan& cp, int r, float (&h)[kBH]) {
     const float x = to_f32(S.tdt[r][cp.c]) + cp.bias;
-    float dt, sig;
-    if (p.softplus) softplus_and_sigmoid<FAST>(x, dt, sig);
-    else dt = x;
+    float dt = x, sig;
+    if (SP) softplus_and_sigmoid<FAST>(x, dt, sig);
     const float du = dt * to_f32(S.tu[r][cp.c]);
     float a[kBH];
     decays<FAST, STRUCT>(dt, cp, a);
@@ -182,7 +180,7 @@ __device__ __forceinline__ void load_state(const float4 (&src)[kNP4][kBwdCh], co
     h[4] = v1.x; h[5] = v1.y; h[6] = v1.z; h[7] = v1.w;
 }
 
-template <typename IO, bool STRUCT>
+template <typename IO, bool STRUCT, bool SP, bool HZ>
 __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, const BwdChan& cp, int b, int blk,
                                          int ch) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
@@ -208,7 +206,12 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
         __syncthreads();
         load_seg<IO>(S, p, b, blk, t0, nt, false);
         __syncthreads();
-        for (int r = 0; r < nt; ++r) fwd_step<IO, FAST, STRUCT>(S, p, cp, r, h);
+        if (nt == kSeg) {
+#pragma unroll 8
+            for (int r = 0; r < kSeg; ++r) fwd_step<IO, FAST, STRUCT, SP>(S, cp, r, h);
+        } else {
+            for (int r = 0; r < nt; ++r) fwd_step<IO, FAST, STRUCT, SP>(S, cp, r, h);
+        }
     }
 
     // ---------------------------------------------------------------- pass 1
@@ -236,18 +239,28 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
 #pragma unroll
             for (int m = 0; m < kBH; ++m) h[m] = 0.0f;
         }
-        // sub-checkpoints (each thread touches only its own half-column)
+        // sub-checkpoints (each thread touches only its own half-column); the
+        // last sub-segment's steps are not needed for them
         for (int s = 0; s < nsub; ++s) {
             store_state(S.hsub[s], cp, h);
-            const int ns = min(kSub, nt - s * kSub);
-            for (int j = 0; j < ns; ++j) fwd_step<IO, FAST, STRUCT>(S, p, cp, s * kSub + j, h);
+            if (s + 1 == nsub) break;
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) fwd_step<IO, FAST, STRUCT, SP>(S, cp, s * kSub + j, h);
         }
         for (int s = nsub - 1; s >= 0; --s) {
             const int ns = min(kSub, nt - s * kSub);
             load_state(S.hsub[s], cp, h);
-            for (int j = 0; j < ns; ++j) {
-                fwd_step<IO, FAST, STRUCT>(S, p, cp, s * kSub + j, h);
-                store_state(S.hstep[j], cp, h);
+            if (ns == kSub) {
+#pragma unroll
+                for (int j = 0; j < kSub; ++j) {
+                    fwd_step<IO, FAST, STRUCT, SP>(S, cp, s * kSub + j, h);
+                    store_state(S.hstep[j], cp, h);
+                }
+            } else {
+                for (int j = 0; j < ns; ++j) {
+                    fwd_step<IO, FAST, STRUCT, SP>(S, cp, s * kSub + j, h);
+                    store_state(S.hstep[j], cp, h);
+                }
             }
             for (int j = ns - 1; j >= 0; --j) {
                 const int r = s * kSub + j;
@@ -258,9 +271,8 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
                 if (j > 0) load_state(S.hstep[j - 1], cp, hprev);
                 else load_state(S.hsub[s], cp, hprev);
                 const float x = to_f32(S.tdt[r][cp.c]) + cp.bias;
-                float dt, sig = 1.0f;
-                if (p.softplus) softplus_and_sigmoid<FAST>(x, dt, sig);
-                else dt = x;
+                float dt = x, sig = 1.0f;
+                if (SP) softplus_and_sigmoid<FAST>(x, dt, sig);
                 const float uv = to_f32(S.tu[r][cp.c]);
                 const float dyv = to_f32(S.tdy[r][cp.c]);
                 float a[kBH];
@@ -274,7 +286,7 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
                 const float sh = acc.x + acc.y;
                 const float sv = sh + partner(sh) + cp.Dv * uv;
                 float ds = dyv;
-                if (p.z) {
+                if (HZ) {
                     const float zv = to_f32(S.tz[r][cp.c]);
                     const float sz = FAST ? rcp_approx(1.0f + ex2_approx(-zv * kLog2e)) : 1.0f / (1.0f + expf(-zv));
                     ds = dyv * zv * sz;
@@ -330,7 +342,8 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
     }
 }
 
-template <typename IO>
+// SP: Δ goes through softplus; HZ: the silu(z) gate is on.
+template <typename IO, bool SP, bool HZ>
 __global__ void __launch_bounds__(kBwdThreads) ss_bwd_kernel(const __grid_constant__ BwdParams p) {
     extern __shared__ __align__(16) unsigned char bwd_smem_raw[];
     auto& S = *reinterpret_cast<BwdSmem<IO>*>(bwd_smem_raw);
@@ -358,9 +371,9 @@ __global__ void __launch_bounds__(kBwdThreads) ss_bwd_kernel(const __grid_consta
     cp.Dv = (cp.valid && p.D) ? p.D[ch] : 0.0f;
     const int all_struct = __syncthreads_and(structured ? 1 : 0);
     if (std::is_same<IO, __nv_bfloat16>::value && all_struct)
-        bwd_item<IO, true>(S, p, cp, b, blk, ch);
+        bwd_item<IO, true, SP, HZ>(S, p, cp, b, blk, ch);
     else
-        bwd_item<IO, false>(S, p, cp, b, blk, ch);
+        bwd_item<IO, false, SP, HZ>(S, p, cp, b, blk, ch);
 }
 
 }  // namespace selscan

@@ -194,9 +194,9 @@ size_t bwd_workspace(const ss_dims* dims) {
     return static_cast<size_t>(dims->batch * nseg * dims->d_inner) * kN * sizeof(float);
 }
 
-template <typename IO>
+template <typename IO, bool SP, bool HZ>
 int launch_bwd(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
-    auto kern = ss_bwd_kernel<IO>;
+    auto kern = ss_bwd_kernel<IO, SP, HZ>;
     const size_t smem = sizeof(BwdSmem<IO>);
     static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
@@ -209,6 +209,13 @@ int launch_bwd(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
     }
     kern<<<static_cast<unsigned>(ctas), kBwdThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+template <typename IO>
+int launch_bwd_flags(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
+    const bool hz = p.z != nullptr;
+    if (p.softplus) return hz ? launch_bwd<IO, true, true>(p, ctas, stream) : launch_bwd<IO, true, false>(p, ctas, stream);
+    return hz ? launch_bwd<IO, false, true>(p, ctas, stream) : launch_bwd<IO, false, false>(p, ctas, stream);
 }
 
 // ------------------------------------------------ allocation-free entry point
@@ -429,7 +436,7 @@ int ss_bwd(const void* u, const void* delta, const float* delta_bias, const floa
     p.L = L; p.batch = static_cast<int>(batch); p.d = static_cast<int>(d);
     p.nseg = static_cast<int>(ceil_div(L, kSeg)); p.nblk = static_cast<int>(nblk);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
-    rc = (flags & SS_BF16) ? launch_bwd<__nv_bfloat16>(p, ctas, stream) : launch_bwd<float>(p, ctas, stream);
+    rc = (flags & SS_BF16) ? launch_bwd_flags<__nv_bfloat16>(p, ctas, stream) : launch_bwd_flags<float>(p, ctas, stream);
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
