@@ -50,8 +50,9 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--mode", choices=["fwd", "decode"], default="fwd",
-                    help="decode: time only the decode workload, --steps single-token steps")
+    ap.add_argument("--mode", choices=["fwd", "decode", "bwd"], default="fwd",
+                    help="decode: time only the decode workload, --steps single-token steps; "
+                         "bwd: time only ss_bwd on --workload")
     return ap.parse_args()
 
 
@@ -276,6 +277,40 @@ def time_e2e(ss, torch, cfg, device, inp, steps):
     return ms, h2d, d2h
 
 
+def time_bwd(ss, torch, cfg, device, steps, warmup):
+    """The backward (ss_bwd) of a forward workload: `steps` calls timed
+    back to back with CUDA events, inputs and upstream gradients resident."""
+    from ss_inputs import bwd_upstream, fwd_inputs
+    inp = fwd_inputs(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.d_state, cfg.dtype, cfg.seed, device,
+                     gate=cfg.gate, D_kind=cfg.D_kind)
+    dy, dl = bwd_upstream(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.d_state, cfg.dtype, cfg.seed, device)
+    stream = torch.cuda.current_stream(device)
+    ws = torch.empty(ss.bwd_workspace_bytes(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.dtype == "bf16"),
+                     dtype=torch.uint8, device=device)
+    grads = None
+
+    def one():
+        return ss.ss_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"], z=inp["z"],
+                         delta_bias=inp["delta_bias"], dlast_state=dl, grads=grads, workspace=ws,
+                         stream=stream)
+
+    grads = one()
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    del inp, dy, dl, grads, ws
+    torch.cuda.empty_cache()
+    return ms
+
+
 def time_decode(ss, torch, device, steps_total=1000, reps=3):
     """The decode workload: 1000 successive ss_step calls (batch 256, d_inner
     5120, fresh bf16 inputs per step).  The 84 MB state fits in L2, so each
@@ -438,6 +473,16 @@ def run_ours(args):
                             "graph_back_to_back_ms_per_step": dms_warm,
                             "graph_back_to_back_steps_per_s": 1e3 / dms_warm}
         torch.cuda.empty_cache()
+        for name in ("mamba2p8b", "mamba130m"):
+            c = CONFIGS[name]
+            bms = time_bwd(ss, torch, c, device, 5, 2)
+            fwd_ms = step_ms if name == cfg.name else extras.get(name, {}).get("ms_per_step")
+            gbs = c.bwd_compulsory_bytes() / (bms * 1e-3) / 1e9
+            extras["bwd_" + name] = {"ms_per_step": bms, "GB_s": gbs, "frac_of_hbm": gbs / hbm,
+                                     "ch_ts_per_s": c.ch_ts / (bms * 1e-3),
+                                     "ratio_to_fwd": (bms / fwd_ms) if fwd_ms else None,
+                                     "note": "ss_bwd (all input gradients), upstream dy and dlast_state "
+                                             "resident; one kernel launch plus the zeroing memsets"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -543,12 +588,35 @@ def run_decode_only(args):
                       "peak_kind": peak_kind, "graph_back_to_back_ms_per_step": ms_warm}), flush=True)
 
 
+def run_bwd_only(args):
+    """Backward workload alone (for profiling and quick checks): --steps ss_bwd
+    calls on --workload."""
+    import torch
+
+    import selective_state_space_37_b200 as ss
+    from ss_inputs import CONFIGS
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    ss.lib()
+    hbm, peak_kind = peaks()
+    c = CONFIGS[args.workload]
+    ms = time_bwd(ss, torch, c, device, max(args.steps, 1), args.warmup)
+    gbs = c.bwd_compulsory_bytes() / (ms * 1e-3) / 1e9
+    print(json.dumps({"metric": "selective-scan bwd effective HBM GB/s", "value": gbs, "unit": "GB/s",
+                      "n_gpus": 1, "steps": args.steps, "ms_per_step": ms, "workload": c.name,
+                      "frac_of_hbm": gbs / hbm, "peak_kind": peak_kind,
+                      "bwd_compulsory_bytes": c.bwd_compulsory_bytes(),
+                      "ch_ts_per_s": c.ch_ts / (ms * 1e-3)}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
     elif args.mode == "decode":
         run_decode_only(args)
+    elif args.mode == "bwd":
+        run_bwd_only(args)
     else:
         run_ours(args)
 

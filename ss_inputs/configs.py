@@ -31,6 +31,18 @@ class FwdConfig:
         state = self.batch * self.d_inner * self.d_state * 4
         return self.ch_ts * per_chts + bc + params + state
 
+    def bwd_compulsory_bytes(self) -> int:
+        """Bytes every backward pass must move at least once: u, delta_raw, z and
+        dy read, du, ddelta and dz written (one element each per
+        channel-timestep); B and C read and dB, dC written in fp32; A/D/bias
+        read, dA/dD/dbias written; dlast_state read."""
+        e = 4 if self.dtype == "fp32" else 2
+        per_chts = (7 if self.gate else 5) * e
+        bc = self.batch * self.seqlen * self.d_state * (2 * e + 2 * 4)
+        params = 2 * self.d_inner * (self.d_state * 4 + 8)
+        state = self.batch * self.d_inner * self.d_state * 4
+        return self.ch_ts * per_chts + bc + params + state
+
 
 @dataclass(frozen=True)
 class StepConfig:
