@@ -48,6 +48,8 @@ def _lib():
             fn.restype = ctypes.c_int
         lib.ss_oracle_bwd_f64.argtypes = [_DP] * 18 + [_I64, _I64, _I64, _I64, ctypes.c_int]
         lib.ss_oracle_bwd_f64.restype = ctypes.c_int
+        lib.ss_oracle_conv_silu_f64.argtypes = [_DP, _DP, _DP, _DP, _I64, _I64, _I64, _I64]
+        lib.ss_oracle_conv_silu_f64.restype = ctypes.c_int
         lib.ss_oracle_set_mutation.argtypes = [ctypes.c_int]
         lib.ss_oracle_get_mutation.restype = ctypes.c_int
         lib.ss_oracle_max_threads.restype = ctypes.c_int
@@ -173,6 +175,26 @@ def bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, dlast=None, soft
     return out
 
 
+def conv_silu(x, w, bias=None):
+    """Causal depthwise conv1d (width w.shape[1]) then SiLU, float64.
+    x [batch, L, d]; w [d, W]; bias [d] or None.  Returns u [batch, L, d]."""
+    xa = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    if xa.ndim != 3:
+        raise ValueError("oracle: x must be [batch, L, d]")
+    batch, L, d = xa.shape
+    wa, wp = _arr(w)
+    if wa.ndim != 2 or wa.shape[0] != d:
+        raise ValueError("oracle: w must be [d, W]")
+    ba, bp = _arr(bias, (d,))
+    u = np.empty_like(xa)
+    rc = _lib().ss_oracle_conv_silu_f64(xa.ctypes.data_as(_DP), wp, _ptr(bp), u.ctypes.data_as(_DP),
+                                        batch, L, d, wa.shape[1])
+    if rc != 0:
+        raise ValueError(f"oracle conv_silu rejected sizes (rc={rc})")
+    del ba
+    return u
+
+
 def set_mutation(m: int) -> None:
     """Test-only: plant deliberate mistake number m (0 restores the oracle)."""
     _lib().ss_oracle_set_mutation(int(m))
@@ -194,7 +216,7 @@ def library_path() -> str:
     return _build.LIB
 
 
-__all__ = ["fwd", "fwd_chunked", "step", "bwd", "set_mutation", "get_mutation",
+__all__ = ["fwd", "fwd_chunked", "step", "bwd", "conv_silu", "set_mutation", "get_mutation",
            "max_threads", "set_threads", "library_path"]
 
 if os.environ.get("SS_ORACLE_THREADS"):

@@ -494,3 +494,32 @@ int ss_oracle_bwd_f64(const double* u, const double* delta, const double* delta_
     }
     return failed ? -1 : 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Causal depthwise conv1d of width W followed by SiLU, double precision: the
+ * Conv1D embedding in front of the SSM ("Understanding Mamba and Selective
+ * State Space Models (SSMs)" §3.3: d_conv = 4, each position sees itself
+ * and the previous 3 tokens, causal), producing the scan's input u:
+ *   c_t = bias[ch] + Σ_{k=0}^{W-1} w[ch, k] · x_{t-(W-1)+k}    (x_{<0} = 0)
+ *   u_t = c_t σ(c_t)
+ * x, u : [batch, L, d];  w : [d, W];  bias : [d] or NULL.
+ * ------------------------------------------------------------------------- */
+int ss_oracle_conv_silu_f64(const double* x, const double* w, const double* bias, double* u,
+                            int64_t batch, int64_t L, int64_t d, int64_t W)
+{
+    if (W < 1 || batch < 0 || L < 0 || d < 0) return -1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t ch = 0; ch < d; ++ch) {
+            for (int64_t t = 0; t < L; ++t) {
+                double c = bias ? bias[ch] : 0.0;
+                for (int64_t k = 0; k < W; ++k) {
+                    const int64_t s = t - (W - 1) + k;
+                    if (s >= 0) c += w[ch * W + k] * x[(b * L + s) * d + ch];
+                }
+                u[(b * L + t) * d + ch] = c / (1.0 + exp(-c));
+            }
+        }
+    }
+    return 0;
+}
