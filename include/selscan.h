@@ -1,7 +1,7 @@
 /*
  * selscan.h -- C ABI of libselscan, the B200 (sm_100a) selective-scan library.
  *
- * Three operations, all from the selective state-space model of Mamba:
+ * The operations, all from the selective state-space model of Mamba:
  *
  *   ss_fwd   the forward scan over a whole sequence ("Algorithm 2" selective
  *            SSM of the mamba README, Usage > Selective SSM; equations of
@@ -16,6 +16,9 @@
  *            function of the Mamba tutorial, §"state management", and the
  *            "constant memory per token" property of the model-architecture
  *            page).
+ *   ss_fwd_conv / ss_step_conv  the same with the causal conv1d + SiLU
+ *            prologue of the Mamba block fused in ("Understanding Mamba and
+ *            Selective State Space Models (SSMs)" §3.3).
  *   ss_bwd   the gradients of ss_fwd's inputs from the gradient of its outputs
  *            (the models are trained and fine-tuned with gradient
  *            checkpointing: "Mamba 7.9.1" article §5.3-5.4; model-architecture
@@ -140,6 +143,38 @@ SS_API int ss_fwd(const void* u, const void* delta, const float* delta_bias, con
 SS_API int ss_step(float* state, const void* u, const void* delta, const float* A, const void* B,
             const void* C, const float* D, const void* z, void* y, const float* delta_bias,
             uint32_t flags, const ss_dims* dims, const ss_launch* launch);
+
+/* ss_fwd_conv -- ss_fwd with the causal conv1d + SiLU prologue fused into the
+ * scan: the input of the recurrence is
+ *   u_t = silu(conv_b + Σ_{k=0}^{3} conv_w[ch, k] · x_{t-3+k}),  x_{<0} = 0,
+ * the Conv1D layer of width d_conv = 4 in front of the SSM ("Understanding
+ * Mamba and Selective State Space Models (SSMs)" §3.3: causal, each token
+ * sees itself and the previous three; the SiLU after it is not on the
+ * pages and is the Mamba block's reading).  u never touches memory.
+ *   x          [batch, seqlen, d_inner] in the element type (takes u's place)
+ *   conv_w     [d_inner, 4] fp32; tap 3 multiplies the current token
+ *   conv_b     [d_inner] fp32, or NULL
+ *   conv_state [batch, d_inner, 3] fp32, or NULL: receives x_{L-3} .. x_{L-1}
+ *              (zero before the sequence), the state ss_step_conv continues from
+ * Everything else, including y = (Σ_n C h + D u) · gate with this u, is as in
+ * ss_fwd; errors as ss_fwd, and SS_ERR_INVALID_ARG for a NULL conv_w. */
+SS_API int ss_fwd_conv(const void* x, const float* conv_w, const float* conv_b, const void* delta,
+                       const float* delta_bias, const float* A, const void* B, const void* C, const float* D,
+                       const void* z, void* y, float* last_state, float* conv_state, uint32_t flags,
+                       const ss_dims* dims, const ss_launch* launch);
+
+/* ss_step_conv -- ss_step with the same prologue for one token:
+ *   conv_state [batch, d_inner, 3] fp32, read and overwritten: the previous
+ *              three x of each channel, oldest first
+ *   x          [batch, d_inner], this token's input (takes u's place)
+ * u = silu(conv_b + w0 s0 + w1 s1 + w2 s2 + w3 x), then the SSM step of
+ * ss_step on u, and the conv state becomes (s1, s2, x).  ss_fwd_conv over L
+ * tokens equals L calls of ss_step_conv from zero states.  Errors as ss_step,
+ * and SS_ERR_INVALID_ARG for a NULL conv_w or conv_state. */
+SS_API int ss_step_conv(float* state, float* conv_state, const void* x, const float* conv_w, const float* conv_b,
+                        const void* delta, const float* A, const void* B, const void* C, const float* D,
+                        const void* z, void* y, const float* delta_bias, uint32_t flags, const ss_dims* dims,
+                        const ss_launch* launch);
 
 /* ss_bwd -- backward of ss_fwd: given dy = dJ/dy and optionally
  * dlast_state = dJ/dlast_state for a scalar J, writes dJ/d(input) for every

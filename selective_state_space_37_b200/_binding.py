@@ -33,7 +33,8 @@ D_STATE = 16
 
 # Every symbol include/selscan.h declares.
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
-            "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes")
+            "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
+            "ss_fwd_conv", "ss_step_conv")
 
 
 class ss_dims(ctypes.Structure):
@@ -96,6 +97,12 @@ def lib():
         L.ss_bwd.restype = ctypes.c_int
         L.ss_bwd_workspace_bytes.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32]
         L.ss_bwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ss_fwd_conv.argtypes = [vp, f32p, f32p, vp, f32p, f32p, vp, vp, f32p, vp, vp, f32p, f32p,
+                                  ctypes.c_uint32, ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch)]
+        L.ss_fwd_conv.restype = ctypes.c_int
+        L.ss_step_conv.argtypes = [f32p, f32p, vp, f32p, f32p, vp, f32p, vp, vp, f32p, vp, vp, f32p,
+                                   ctypes.c_uint32, ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch)]
+        L.ss_step_conv.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -267,6 +274,81 @@ def ss_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, dlast_state=N
     if rc != SS_OK:
         raise SelscanError(rc, "ss_bwd")
     return {k: g[k] for k in shapes}
+
+
+def ss_fwd_conv(x, conv_w, delta, A, B, C, D=None, z=None, delta_bias=None, conv_b=None, *, y=None,
+                last_state=None, return_last_state=True, conv_state=None, softplus=True, chunk_len=0,
+                timeout_iters=0, workspace=None, stream=None, sync_check=False):
+    """ss_fwd with the causal conv1d (width 4) + SiLU prologue: x takes u's
+    place, conv_w [d_inner, 4] fp32, conv_b [d_inner] fp32 or None.  Returns
+    (y, last_state); pass conv_state [batch, d_inner, 3] fp32 to receive the
+    last three x of each channel (for ss_step_conv)."""
+    if x.dim() != 3:
+        raise ValueError("x must be [batch, L, d_inner]")
+    batch, L, d = x.shape
+    dev = x.device
+    io = x.dtype
+    for t, nm, shp in ((x, "x", (batch, L, d)), (delta, "delta", (batch, L, d)),
+                       (z, "z", (batch, L, d)), (B, "B", (batch, L, D_STATE)),
+                       (C, "C", (batch, L, D_STATE))):
+        _check(t, nm, shp, io, dev)
+    _check(conv_w, "conv_w", (d, 4), torch.float32, dev)
+    _check(conv_b, "conv_b", (d,), torch.float32, dev)
+    _check(A, "A", (d, D_STATE), torch.float32, dev)
+    _check(D, "D", (d,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (d,), torch.float32, dev)
+    _check(conv_state, "conv_state", (batch, d, 3), torch.float32, dev)
+    if y is None:
+        y = torch.empty((batch, L, d), dtype=io, device=dev)
+    _check(y, "y", (batch, L, d), io, dev)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, d, D_STATE), dtype=torch.float32, device=dev)
+    _check(last_state, "last_state", (batch, d, D_STATE), torch.float32, dev)
+    flags = _io_flag(x) | (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
+    sh = _stream_handle(stream, dev)
+    dims = ss_dims(batch, L, d, D_STATE)
+    need = int(lib().ss_fwd_workspace_bytes(ctypes.byref(dims), flags, int(chunk_len)))
+    if workspace is None:
+        workspace = workspace_for(need, dev, sh)
+    launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                       int(timeout_iters), int(chunk_len))
+    rc = lib().ss_fwd_conv(_ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(delta), _ptr(delta_bias), _ptr(A),
+                           _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y), _ptr(last_state), _ptr(conv_state),
+                           flags, ctypes.byref(dims), ctypes.byref(launch))
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_fwd_conv")
+    return y, last_state
+
+
+def ss_step_conv(state, conv_state, x, conv_w, delta, A, B, C, D=None, z=None, delta_bias=None, conv_b=None,
+                 *, y=None, softplus=True, stream=None, sync_check=False):
+    """One decode step with the conv prologue; state [batch, d_inner, 16] and
+    conv_state [batch, d_inner, 3] (fp32) are updated in place.  Returns y."""
+    batch, d = x.shape
+    dev = x.device
+    io = x.dtype
+    _check(state, "state", (batch, d, D_STATE), torch.float32, dev)
+    _check(conv_state, "conv_state", (batch, d, 3), torch.float32, dev)
+    for t, nm, shp in ((x, "x", (batch, d)), (delta, "delta", (batch, d)), (z, "z", (batch, d)),
+                       (B, "B", (batch, D_STATE)), (C, "C", (batch, D_STATE))):
+        _check(t, nm, shp, io, dev)
+    _check(conv_w, "conv_w", (d, 4), torch.float32, dev)
+    _check(conv_b, "conv_b", (d,), torch.float32, dev)
+    _check(A, "A", (d, D_STATE), torch.float32, dev)
+    _check(D, "D", (d,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (d,), torch.float32, dev)
+    if y is None:
+        y = torch.empty((batch, d), dtype=io, device=dev)
+    flags = _io_flag(x) | (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
+    sh = _stream_handle(stream, dev)
+    dims = ss_dims(batch, 1, d, D_STATE)
+    launch = ss_launch(sh, None, 0, 0, 0)
+    rc = lib().ss_step_conv(_ptr(state), _ptr(conv_state), _ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(delta),
+                            _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(y), _ptr(delta_bias), flags,
+                            ctypes.byref(dims), ctypes.byref(launch))
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_step_conv")
+    return y
 
 
 def ss_check(workspace, stream=None, device=None):

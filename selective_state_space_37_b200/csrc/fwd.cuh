@@ -61,6 +61,8 @@ constexpr int kTT = 32;     // timesteps per tile
 constexpr int kCB = 128;    // channels per CTA (two threads per channel)
 constexpr int kNT = 2 * kCB;        // threads per CTA
 constexpr int kRec = 48;    // floats per carry record: P[16], h_loc[16], inclusive[16]
+constexpr int kConvW = 4;   // width of the causal conv1d prologue (d_conv)
+constexpr int kHalo = kConvW - 1;   // rows of x the conv needs before a tile
 static_assert(kNT == 2 * kCB, "two threads per channel");
 
 enum : uint32_t { kStNone = 0, kStAgg = 1, kStIncl = 2, kStTimeout = 0xFFFFFFFFu };
@@ -70,7 +72,8 @@ enum : uint32_t {
     kPfTestDrop = 4u,
     kPfHasZ = 8u,
     kPfHasBias = 16u,
-    kPfHasD = 32u
+    kPfHasD = 32u,
+    kPfConv = 64u
 };
 
 struct FwdParams {
@@ -84,6 +87,8 @@ struct FwdParams {
     const void* z;
     void* y;
     float* last_state;
+    const float* conv_w;   // [d, kConvW] (conv prologue only)
+    const float* conv_b;   // [d] or null
     int64_t L;
     int batch, d, chunk_len, nchunks, nblk;
     uint32_t pflags;
@@ -97,7 +102,9 @@ struct FwdParams {
 
 template <typename IO, int STAGES>
 struct FwdSmem {
-    IO a[STAGES][kTT][kCB];          // u (scan pass) or provisional y (fix-up pass)
+    // Rows kHalo.. hold u (scan pass) or the provisional y (fix-up pass); with
+    // the conv prologue the scan pass fills rows 0.. with x from t0 - kHalo.
+    IO a[STAGES][kHalo + kTT][kCB];
     IO dt[STAGES][kTT][kCB];
     IO z[STAGES][kTT][kCB];
     IO B[STAGES][kTT][kN];
@@ -149,7 +156,23 @@ struct ChanParams {
     uint32_t hi_mask;  // all ones on the thread holding the upper half (p = 1)
     int p;             // 0: states 0..7, 1: states 8..15
     bool valid;        // channel < d_inner
+    float cw[kConvW];  // conv prologue weights (oldest tap first) and bias
+    float cb;
 };
+
+// The scan's input u at tile row j.  xs points at row 0 of this channel's
+// column of the tile.  Without the prologue u sits at row kHalo + j; with it,
+// u = silu(cb + Σ_k cw[k] x_{t-3+k}) ("Understanding Mamba and Selective
+// State Space Models (SSMs)" §3.3: causal conv of width 4 before the SSM)
+// from rows j .. j+3, which hold x from t0 - 3 (zeros before the sequence).
+template <typename IO, bool FAST, bool CONV>
+__device__ __forceinline__ float u_at(const IO* __restrict__ xs, int j, const ChanParams& cp) {
+    if (!CONV) return to_f32(xs[(j + kHalo) * kCB]);
+    float c = cp.cb;
+#pragma unroll
+    for (int k = 0; k < kConvW; ++k) c = fmaf(cp.cw[k], to_f32(xs[(j + k) * kCB]), c);
+    return FAST ? silu_tanh(c) : silu_accurate(c);
+}
 
 // Decays of this thread's eight states as pairs, for the structured path:
 // (r^(8p+1), r^(8p+2)), ..., (r^(8p+7), r^(8p+8)) from base = r^(8p+1).
@@ -212,7 +235,7 @@ __device__ __forceinline__ void half_update(float lam, float du, const f32x2 (&B
 // A group of NSTEP (even) timesteps of the scan, rows j0 .. j0+NSTEP-1.
 // us/dts/zs point at this channel's column of the tile (row 0); yrow at this
 // channel's output for row 0 of the tile.
-template <typename IO, bool FAST, bool STRUCT, bool TRACK, int NSTEP>
+template <typename IO, bool FAST, bool STRUCT, bool TRACK, int NSTEP, bool CONV>
 __device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* __restrict__ dts,
                                            const IO* __restrict__ zs, const float* __restrict__ bc, int j0,
                                            f32x2 (&H)[4], f32x2 (&PP)[4], float& R, const ChanParams& cp,
@@ -223,7 +246,7 @@ __device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* 
 #pragma unroll
     for (int i = 0; i < NH; ++i) {
         const int row = (j0 + 2 * i + cp.p) * kCB;
-        const float uu = to_f32(us[row]);
+        const float uu = u_at<IO, FAST, CONV>(us, j0 + 2 * i + cp.p, cp);
         lo[i] = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
         dlo[i] = lo[i] * uu;
         su[i] = cp.Dv * uu;
@@ -259,13 +282,13 @@ __device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* 
 }
 
 // One timestep of the scan (ragged tails); both threads prepare it.
-template <typename IO, bool FAST, bool STRUCT, bool TRACK>
+template <typename IO, bool FAST, bool STRUCT, bool TRACK, bool CONV>
 __device__ __forceinline__ void scan_one(const IO* __restrict__ us, const IO* __restrict__ dts,
                                          const IO* __restrict__ zs, const float* __restrict__ bc, int j,
                                          f32x2 (&H)[4], f32x2 (&PP)[4], float& R, const ChanParams& cp,
                                          IO* __restrict__ yrow, int64_t d) {
     const int row = j * kCB;
-    const float uu = to_f32(us[row]);
+    const float uu = u_at<IO, FAST, CONV>(us, j, cp);
     const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
     const float g = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
     f32x2 Bp[4], Cp[4];
@@ -374,6 +397,7 @@ struct ItemCtx {
     int cc;             // this thread's channel within the block
     int64_t t_begin, t_end, d;
     bool has_z;
+    bool conv;          // the scan pass streams x (with kHalo rows before the tile) for the conv prologue
     float bscale;
     uint32_t bytes_scan, bytes_fix;
 
@@ -382,7 +406,8 @@ struct ItemCtx {
         const int t0 = static_cast<int>(t_begin + static_cast<int64_t>(k) * kTT);
         uint64_t* bar = &S->full[s];
         mbar_arrive_expect_tx(bar, pass == 0 ? bytes_scan : bytes_fix);
-        tma_load_3d(&S->a[s][0][0], pass == 0 ? tm_u : tm_y, g * kCB, t0, b, bar);
+        if (pass == 0 && conv) tma_load_3d(&S->a[s][0][0], tm_u, g * kCB, t0 - kHalo, b, bar);
+        else tma_load_3d(&S->a[s][kHalo][0], pass == 0 ? tm_u : tm_y, g * kCB, t0, b, bar);
         tma_load_3d(&S->dt[s][0][0], tm_dt, g * kCB, t0, b, bar);
         if (has_z) tma_load_3d(&S->z[s][0][0], tm_z, g * kCB, t0, b, bar);
         if (pass == 0) tma_load_3d(&S->B[s][0][0], tm_B, 0, t0, b, bar);
@@ -400,9 +425,18 @@ struct ItemCtx {
             const int ch = g * kCB + col;
             const bool ok = (t < p->L) && (ch < p->d);
             const int64_t idx = (static_cast<int64_t>(b) * p->L + t) * d + ch;
-            S->a[0][r][col] = ok ? ga[idx] : from_f32<IO>(0.f);
+            S->a[0][kHalo + r][col] = ok ? ga[idx] : from_f32<IO>(0.f);
             S->dt[0][r][col] = ok ? gd[idx] : from_f32<IO>(0.f);
             if (has_z) S->z[0][r][col] = ok ? gz[idx] : from_f32<IO>(0.f);
+        }
+        if (pass == 0 && conv) {   // x rows t0 - kHalo .. t0 - 1 (zero before the sequence)
+            for (int i = tid; i < kHalo * kCB; i += kNT) {
+                const int r = i / kCB, col = i % kCB;
+                const int64_t t = t0 - kHalo + r;
+                const int ch = g * kCB + col;
+                const bool ok = (t >= 0) && (t < p->L) && (ch < p->d);
+                S->a[0][r][col] = ok ? ga[(static_cast<int64_t>(b) * p->L + t) * d + ch] : from_f32<IO>(0.f);
+            }
         }
         const IO* gB = static_cast<const IO*>(p->B);
         const IO* gC = static_cast<const IO*>(p->C);
@@ -446,7 +480,7 @@ struct ItemCtx {
 
 // The scan (and, for a provisional chunk, look-back and fix-up) of one item,
 // specialised on the decay form and on whether the entry state is known.
-template <typename IO, bool USE_TMA, int STAGES, int G, bool UNROLL, bool STRUCT, bool EXACT>
+template <typename IO, bool USE_TMA, int STAGES, int G, bool UNROLL, bool STRUCT, bool EXACT, bool CONV>
 __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it, const ChanParams& cp,
                                          f32x2 (&H)[4]) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
@@ -476,11 +510,12 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
         if (UNROLL && nt == kTT) {
 #pragma unroll
             for (int gi = 0; gi < kTT / G; ++gi)
-                scan_group<IO, FAST, STRUCT, TRACK, G>(us, dts, zs, bc, gi * G, H, PP, R, cp, yrow, d);
+                scan_group<IO, FAST, STRUCT, TRACK, G, CONV>(us, dts, zs, bc, gi * G, H, PP, R, cp, yrow, d);
         } else {
             int j0 = 0;
-            for (; j0 + G <= nt; j0 += G) scan_group<IO, FAST, STRUCT, TRACK, G>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
-            for (; j0 < nt; ++j0)           scan_one<IO, FAST, STRUCT, TRACK>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+            for (; j0 + G <= nt; j0 += G)
+                scan_group<IO, FAST, STRUCT, TRACK, G, CONV>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+            for (; j0 < nt; ++j0) scan_one<IO, FAST, STRUCT, TRACK, CONV>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
         }
         t += nt;
     }
@@ -613,7 +648,7 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
         for (int k = 0; k < it.ntiles; ++k, ++kk) {
             const int s = it.acquire(k, kk, 1);
             const int nt = static_cast<int>((it.t_end - t) < kTT ? (it.t_end - t) : kTT);
-            const IO* ys = &S.a[s][0][it.cc];
+            const IO* ys = &S.a[s][kHalo][it.cc];
             const IO* dts = &S.dt[s][0][it.cc];
             const IO* zs = &S.z[s][0][it.cc];
             const float* bc = &S.bc[s][0][0];
@@ -626,8 +661,9 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
     }
 }
 
-// MINB resident CTAs per SM, groups of G steps, whole tiles unrolled or not.
-template <typename IO, bool USE_TMA, int STAGES, int MINB, int G, bool UNROLL>
+// MINB resident CTAs per SM, groups of G steps, whole tiles unrolled or not;
+// CONV: u comes from the causal conv1d + SiLU prologue over x.
+template <typename IO, bool USE_TMA, int STAGES, int MINB, int G, bool UNROLL, bool CONV>
 __global__ void __launch_bounds__(kNT, MINB)
 ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_u,
               const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_z,
@@ -661,9 +697,10 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
     it.ntiles = static_cast<int>((it.t_end - it.t_begin + kTT - 1) / kTT);
     it.d = p.d;
     it.has_z = (p.pflags & kPfHasZ) != 0;
+    it.conv = CONV;
     it.bscale = FAST ? kLn2 : 1.0f;
     const int nact = it.has_z ? 3 : 2;   // per-channel tensors streamed per pass
-    it.bytes_scan = static_cast<uint32_t>((nact * kTT * kCB + 2 * kTT * kN) * sizeof(IO));
+    it.bytes_scan = static_cast<uint32_t>(((nact * kTT + (CONV ? kHalo : 0)) * kCB + 2 * kTT * kN) * sizeof(IO));
     it.bytes_fix = static_cast<uint32_t>((nact * kTT * kCB + kTT * kN) * sizeof(IO));
     const int ch = it.g * kCB + it.cc;
 
@@ -691,6 +728,9 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
     cp.Dv = (cp.valid && (p.pflags & kPfHasD)) ? __ldg(p.D + ch) : 0.f;
     const float biasv = (cp.valid && (p.pflags & kPfHasBias)) ? __ldg(p.bias + ch) : 0.f;
     cp.bias_s = FAST ? biasv * kLog2e : biasv;
+#pragma unroll
+    for (int k = 0; k < kConvW; ++k) cp.cw[k] = (CONV && cp.valid) ? __ldg(p.conv_w + static_cast<int64_t>(ch) * kConvW + k) : 0.f;
+    cp.cb = (CONV && cp.valid && p.conv_b) ? __ldg(p.conv_b + ch) : 0.f;
 
     // ------------------------------------------------------- entry state
     f32x2 H[4];
@@ -728,11 +768,11 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
 
     static_assert(G % 2 == 0 && kTT % G == 0, "groups hold an even number of steps and tile a tile");
     if (use_struct) {
-        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, true, true>(it, cp, H);
-        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, true, false>(it, cp, H);
+        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, true, true, CONV>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, true, false, CONV>(it, cp, H);
     } else {
-        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, false, true>(it, cp, H);
-        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, false, false>(it, cp, H);
+        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, false, true, CONV>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, false, false, CONV>(it, cp, H);
     }
 }
 

@@ -154,9 +154,9 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint6
     return r == CUDA_SUCCESS;
 }
 
-template <typename IO, bool TMA, int STAGES, int MINB, int G, bool UNROLL>
+template <typename IO, bool TMA, int STAGES, int MINB, int G, bool UNROLL, bool CONV>
 int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
-    auto kern = ss_fwd_kernel<IO, TMA, STAGES, MINB, G, UNROLL>;
+    auto kern = ss_fwd_kernel<IO, TMA, STAGES, MINB, G, UNROLL, CONV>;
     const size_t smem = sizeof(FwdSmem<IO, STAGES>);
     static bool attr_set[kMaxDevices] = {false};
     int dev = 0;
@@ -170,6 +170,22 @@ int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaS
     kern<<<static_cast<unsigned>(items), kNT, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4],
                                                               maps[5]);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
+// Forward-kernel instantiation for the variant, element type, TMA use and
+// the conv prologue.
+template <bool CONV>
+int launch_variant(bool bf16, bool tma, Variant v, const FwdParams& p, int64_t items, const CUtensorMap* maps,
+                   cudaStream_t stream) {
+    if (bf16) {
+        if (v == kNarrow)
+            return tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 4, false, CONV>(p, items, maps, stream)
+                       : launch_fwd<__nv_bfloat16, false, 1, 2, 4, false, CONV>(p, items, maps, stream);
+        return tma ? launch_fwd<__nv_bfloat16, true, 4, 1, 8, true, CONV>(p, items, maps, stream)
+                   : launch_fwd<__nv_bfloat16, false, 1, 1, 8, true, CONV>(p, items, maps, stream);
+    }
+    return tma ? launch_fwd<float, true, 2, 1, 8, false, CONV>(p, items, maps, stream)
+               : launch_fwd<float, false, 1, 1, 8, false, CONV>(p, items, maps, stream);
 }
 
 int validate_dims(const ss_dims* dims, bool need_seqlen) {
@@ -278,9 +294,12 @@ int ss_check(const ss_launch* launch) {
     return static_cast<int>(word);
 }
 
-int ss_fwd(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
-           const void* C, const float* D, const void* z, void* y, float* last_state, uint32_t flags,
-           const ss_dims* dims, const ss_launch* launch) {
+// ss_fwd and ss_fwd_conv (conv_w non-null: u is computed from x = `u` by the
+// causal conv1d + SiLU prologue).
+static int fwd_impl(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+                    const void* C, const float* D, const void* z, void* y, float* last_state, const float* conv_w,
+                    const float* conv_b, uint32_t flags, const ss_dims* dims, const ss_launch* launch) {
+    const bool conv = conv_w != nullptr;
     int rc = validate_dims(dims, true);
     if (rc != SS_OK) return rc;
     if (!launch || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
@@ -296,7 +315,7 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
         return SS_OK;
     }
     if (!u || !delta || !A || !B || !C || !y) return SS_ERR_INVALID_ARG;
-    const void* ptrs[] = {u, delta, delta_bias, A, B, C, D, z, y, last_state};
+    const void* ptrs[] = {u, delta, delta_bias, A, B, C, D, z, y, last_state, conv_w, conv_b};
     for (const void* q : ptrs)
         if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
 
@@ -313,12 +332,13 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
     FwdParams p{};
     p.u = u; p.delta = delta; p.bias = delta_bias; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
     p.y = y; p.last_state = last_state;
+    p.conv_w = conv_w; p.conv_b = conv_b;
     p.L = L; p.batch = static_cast<int>(batch); p.d = static_cast<int>(d);
     p.chunk_len = static_cast<int>(pl.chunk_len > 0 ? pl.chunk_len : L);
     p.nchunks = static_cast<int>(pl.nchunks); p.nblk = static_cast<int>(pl.nblk);
     p.pflags = ((flags & SS_DELTA_SOFTPLUS) ? kPfSoftplus : 0u) | ((flags & SS_FORCE_GENERAL_A) ? kPfForceGeneral : 0u) |
                ((flags & SS_TEST_DROP_CARRY) ? kPfTestDrop : 0u) | (z ? kPfHasZ : 0u) |
-               (delta_bias ? kPfHasBias : 0u) | (D ? kPfHasD : 0u);
+               (delta_bias ? kPfHasBias : 0u) | (D ? kPfHasD : 0u) | (conv ? kPfConv : 0u);
     p.hdr = reinterpret_cast<uint32_t*>(ws);
     p.status = reinterpret_cast<uint32_t*>(ws + pl.status_off);
     p.rec = reinterpret_cast<float*>(ws + pl.rec_off);
@@ -330,7 +350,7 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
     CUtensorMap maps[6];
     std::memset(maps, 0, sizeof(maps));
     if (tma) {
-        bool ok = make_map(&maps[0], u, bf16, d, L, batch, kCB, kTT) &&
+        bool ok = make_map(&maps[0], u, bf16, d, L, batch, kCB, kTT + (conv ? kHalo : 0)) &&
                   make_map(&maps[1], delta, bf16, d, L, batch, kCB, kTT) &&
                   make_map(&maps[2], z ? z : u, bf16, d, L, batch, kCB, kTT) &&
                   make_map(&maps[3], B, bf16, kN, L, batch, kN, kTT) &&
@@ -338,51 +358,95 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
                   make_map(&maps[5], y, bf16, d, L, batch, kCB, kTT);
         if (!ok) return SS_ERR_CUDA;
     }
-    if (bf16) {
-        if (choose(dims, flags).v == kNarrow)
-            rc = tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 4, false>(p, items, maps, stream)
-                     : launch_fwd<__nv_bfloat16, false, 1, 2, 4, false>(p, items, maps, stream);
-        else
-            rc = tma ? launch_fwd<__nv_bfloat16, true, 4, 1, 8, true>(p, items, maps, stream)
-                     : launch_fwd<__nv_bfloat16, false, 1, 1, 8, true>(p, items, maps, stream);
-    } else {
-        rc = tma ? launch_fwd<float, true, 2, 1, 8, false>(p, items, maps, stream)
-                 : launch_fwd<float, false, 1, 1, 8, false>(p, items, maps, stream);
-    }
+    const Variant v = choose(dims, flags).v;
+    rc = conv ? launch_variant<true>(bf16, tma, v, p, items, maps, stream)
+              : launch_variant<false>(bf16, tma, v, p, items, maps, stream);
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) return ss_check(launch);
     return SS_OK;
 }
 
-int ss_step(float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
-            const float* D, const void* z, void* y, const float* delta_bias, uint32_t flags, const ss_dims* dims,
-            const ss_launch* launch) {
+int ss_fwd(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+           const void* C, const float* D, const void* z, void* y, float* last_state, uint32_t flags,
+           const ss_dims* dims, const ss_launch* launch) {
+    return fwd_impl(u, delta, delta_bias, A, B, C, D, z, y, last_state, nullptr, nullptr, flags, dims, launch);
+}
+
+int ss_fwd_conv(const void* x, const float* conv_w, const float* conv_b, const void* delta, const float* delta_bias,
+                const float* A, const void* B, const void* C, const float* D, const void* z, void* y,
+                float* last_state, float* conv_state, uint32_t flags, const ss_dims* dims, const ss_launch* launch) {
+    if (!conv_w) return SS_ERR_INVALID_ARG;
+    if (conv_state && !aligned16(conv_state)) return SS_ERR_INVALID_ARG;
+    int rc = fwd_impl(x, delta, delta_bias, A, B, C, D, z, y, last_state, conv_w, conv_b,
+                      flags & ~static_cast<uint32_t>(SS_SYNC_CHECK), dims, launch);
+    if (rc != SS_OK) return rc;
+    const int64_t n = dims->batch * dims->d_inner;
+    if (conv_state && n > 0) {
+        if (!x && dims->seqlen > 0) return SS_ERR_INVALID_ARG;
+        cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
+        const unsigned blocks = static_cast<unsigned>(std::min<int64_t>(ceil_div(n, 256), 4096));
+        if (flags & SS_BF16)
+            ss_conv_tail_kernel<__nv_bfloat16><<<blocks, 256, 0, stream>>>(
+                static_cast<const __nv_bfloat16*>(x), conv_state, dims->batch, dims->seqlen, dims->d_inner);
+        else
+            ss_conv_tail_kernel<float><<<blocks, 256, 0, stream>>>(static_cast<const float*>(x), conv_state,
+                                                                   dims->batch, dims->seqlen, dims->d_inner);
+        if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+    }
+    if (flags & SS_SYNC_CHECK) return ss_check(launch);
+    return SS_OK;
+}
+
+// ss_step and ss_step_conv (conv_w non-null: the token's input `u` is x, and
+// u = silu(conv) over conv_state, which shifts in x).
+static int step_impl(float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
+                     const float* D, const void* z, void* y, const float* delta_bias, float* conv_state,
+                     const float* conv_w, const float* conv_b, uint32_t flags, const ss_dims* dims,
+                     const ss_launch* launch) {
     int rc = validate_dims(dims, false);
     if (rc != SS_OK) return rc;
     if (!launch || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
+    const bool conv = conv_w != nullptr;
     const int64_t batch = dims->batch, d = dims->d_inner;
     if (batch == 0 || d == 0) return SS_OK;
-    if (!state || !u || !delta || !A || !B || !C || !y) return SS_ERR_INVALID_ARG;
-    const void* ptrs[] = {state, u, delta, A, B, C, D, z, y, delta_bias};
+    if (!state || !u || !delta || !A || !B || !C || !y || (conv && !conv_state)) return SS_ERR_INVALID_ARG;
+    const void* ptrs[] = {state, u, delta, A, B, C, D, z, y, delta_bias, conv_state, conv_w, conv_b};
     for (const void* q : ptrs)
         if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
     const bool bf16 = (flags & SS_BF16) != 0;
     StepParams p{};
     p.state = state; p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z; p.y = y;
     p.bias = delta_bias; p.batch = batch; p.d = static_cast<int>(d);
+    p.conv_state = conv_state; p.conv_w = conv_w; p.conv_b = conv_b;
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
     const dim3 grid(static_cast<unsigned>(ceil_div(d, kStepChanPerBlock)),
                     static_cast<unsigned>(std::min<int64_t>(ceil_div(batch, 2), 65535)));
     cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
-    if (bf16)
-        ss_step_kernel<__nv_bfloat16><<<grid, kStepThreads, 0, stream>>>(p);
-    else
-        ss_step_kernel<float><<<grid, kStepThreads, 0, stream>>>(p);
+    if (bf16) {
+        if (conv) ss_step_kernel<__nv_bfloat16, true><<<grid, kStepThreads, 0, stream>>>(p);
+        else      ss_step_kernel<__nv_bfloat16, false><<<grid, kStepThreads, 0, stream>>>(p);
+    } else {
+        if (conv) ss_step_kernel<float, true><<<grid, kStepThreads, 0, stream>>>(p);
+        else      ss_step_kernel<float, false><<<grid, kStepThreads, 0, stream>>>(p);
+    }
     if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
     }
     return SS_OK;
+}
+
+int ss_step(float* state, const void* u, const void* delta, const float* A, const void* B, const void* C,
+            const float* D, const void* z, void* y, const float* delta_bias, uint32_t flags, const ss_dims* dims,
+            const ss_launch* launch) {
+    return step_impl(state, u, delta, A, B, C, D, z, y, delta_bias, nullptr, nullptr, nullptr, flags, dims, launch);
+}
+
+int ss_step_conv(float* state, float* conv_state, const void* x, const float* conv_w, const float* conv_b,
+                 const void* delta, const float* A, const void* B, const void* C, const float* D, const void* z,
+                 void* y, const float* delta_bias, uint32_t flags, const ss_dims* dims, const ss_launch* launch) {
+    if (!conv_w) return SS_ERR_INVALID_ARG;
+    return step_impl(state, x, delta, A, B, C, D, z, y, delta_bias, conv_state, conv_w, conv_b, flags, dims, launch);
 }
 
 size_t ss_bwd_workspace_bytes(const ss_dims* dims, uint32_t flags) {

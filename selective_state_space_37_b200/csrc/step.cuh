@@ -10,6 +10,10 @@
 // readout Σ_n C_n h_n is finished with two butterfly shuffles.  A block
 // covers kStepChanPerBlock channels of one batch row, so a thread finds its
 // (batch, channel) without integer division.
+// With the conv prologue (CONV) the token's input is x and u = silu(cb +
+// w0 s0 + w1 s1 + w2 s2 + w3 x) over the conv state s (the previous three x
+// of the channel, fp32, oldest first), which then shifts in x ("Understanding
+// Mamba and Selective State Space Models (SSMs)" §3.3, causal conv of width 4).
 #pragma once
 
 #include <type_traits>
@@ -32,10 +36,30 @@ struct StepParams {
     const void* z;
     void* y;
     const float* bias;
+    float* conv_state;     // [batch, d, 3] fp32, read and shifted (conv prologue only)
+    const float* conv_w;   // [d, 4]
+    const float* conv_b;   // [d] or null
     int64_t batch;
     int d;
     int softplus;
 };
+
+// x[b, L-3 .. L-1, ch] of a sequence as fp32 (zero before its start): the conv
+// state a decode step continues from after a forward pass with the prologue.
+template <typename IO>
+__global__ void ss_conv_tail_kernel(const IO* __restrict__ x, float* __restrict__ conv_state, int64_t batch,
+                                    int64_t L, int64_t d) {
+    const int64_t n = batch * d;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t b = i / d, ch = i % d;
+#pragma unroll
+        for (int k = 0; k < 3; ++k) {
+            const int64_t t = L - 3 + k;
+            conv_state[i * 3 + k] = t >= 0 ? to_f32(x[(b * L + t) * d + ch]) : 0.0f;
+        }
+    }
+}
 
 template <typename IO>
 __device__ __forceinline__ void load4(const IO* p, float (&v)[4]);
@@ -53,7 +77,7 @@ __device__ __forceinline__ void load4<__nv_bfloat16>(const __nv_bfloat16* p, flo
 
 // Grid: x over blocks of kStepChanPerBlock channels of one batch row,
 // y over batch rows (strided when batch exceeds the grid's y extent).
-template <typename IO>
+template <typename IO, bool CONV>
 __global__ void __launch_bounds__(kStepThreads) ss_step_kernel(const __grid_constant__ StepParams p) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
     const int q = threadIdx.x & 3;   // states 4q .. 4q+3
@@ -64,13 +88,19 @@ __global__ void __launch_bounds__(kStepThreads) ss_step_kernel(const __grid_cons
     load4<float>(p.A + static_cast<int64_t>(chs) * 16 + 4 * q, Av);
     const float Dv = (valid && p.D) ? __ldg(p.D + chs) : 0.f;
     const float bv = (valid && p.bias) ? __ldg(p.bias + chs) : 0.f;
+    float cw[4] = {0.f, 0.f, 0.f, 0.f};
+    float cb = 0.f;
+    if (CONV) {
+        load4<float>(p.conv_w + static_cast<int64_t>(chs) * 4, cw);
+        cb = (valid && p.conv_b) ? __ldg(p.conv_b + chs) : 0.f;
+    }
     // Two batch rows per iteration, all their loads issued before the math.
     constexpr int R = 2;
     for (int64_t b0 = blockIdx.y; b0 < p.batch; b0 += static_cast<int64_t>(R) * gridDim.y) {
         int64_t cs[R];
         bool ok[R];
         float4 h4[R];
-        float uu[R], xr[R], zz[R], Bv[R][4], Cv[R][4];
+        float uu[R], xr[R], zz[R], Bv[R][4], Cv[R][4], cs3[R][3];
 #pragma unroll
         for (int r = 0; r < R; ++r) {
             const int64_t b = b0 + static_cast<int64_t>(r) * gridDim.y;
@@ -84,9 +114,24 @@ __global__ void __launch_bounds__(kStepThreads) ss_step_kernel(const __grid_cons
             zz[r] = (ok[r] && p.z) ? to_f32(static_cast<const IO*>(p.z)[cs[r]]) : 0.f;
             load4<IO>(static_cast<const IO*>(p.B) + bs * 16 + 4 * q, Bv[r]);
             load4<IO>(static_cast<const IO*>(p.C) + bs * 16 + 4 * q, Cv[r]);
+            if (CONV) {
+#pragma unroll
+                for (int k = 0; k < 3; ++k) cs3[r][k] = ok[r] ? p.conv_state[cs[r] * 3 + k] : 0.f;
+            }
         }
+        if (CONV) __syncwarp();   // every lane of a channel has read its conv state before it shifts
 #pragma unroll
         for (int r = 0; r < R; ++r) {
+            if (CONV) {
+                const float xv = uu[r];
+                const float c = fmaf(cw[3], xv, fmaf(cw[2], cs3[r][2], fmaf(cw[1], cs3[r][1], fmaf(cw[0], cs3[r][0], cb))));
+                uu[r] = FAST ? silu_tanh(c) : silu_accurate(c);
+                if (ok[r] && q == 0) {
+                    p.conv_state[cs[r] * 3 + 0] = cs3[r][1];
+                    p.conv_state[cs[r] * 3 + 1] = cs3[r][2];
+                    p.conv_state[cs[r] * 3 + 2] = xv;
+                }
+            }
             // λ = Δ / ln 2 on the fast path (decay 2^(λ A), Δ u = λ (ln 2 u)); Δ itself otherwise.
             float lam, dscale;
             if (FAST) {

@@ -20,11 +20,13 @@ table, d_state = 16 as in the README usage example and the deep-dive article
   I/O dtype     : fp32 for the tiny case, bf16 otherwise; A, D, bias fp32.
   Backward upstream gradients: dy ~ N(0, 1) in the I/O dtype and
   dlast_state ~ N(0, 1) fp32.
+  Conv prologue (deep-dive §3.3): conv_w [d, 4] Kaiming-normal, std sqrt(2/4);
+  conv_b = 0 (or N(0, 0.1^2) where a test covers the bias); x takes u's recipe.
 """
 from .configs import CONFIGS, FwdConfig, StepConfig, get_config
-from .gen import (bwd_upstream, fwd_inputs, step_inputs, step_sequence_inputs, general_A,
+from .gen import (bwd_upstream, conv_params, fwd_inputs, step_inputs, step_sequence_inputs, general_A,
                   to_f64, sample_channels)
 
-__all__ = ["CONFIGS", "FwdConfig", "StepConfig", "get_config", "fwd_inputs", "bwd_upstream",
+__all__ = ["CONFIGS", "FwdConfig", "StepConfig", "get_config", "fwd_inputs", "bwd_upstream", "conv_params",
            "step_inputs", "step_sequence_inputs", "general_A", "to_f64",
            "sample_channels"]

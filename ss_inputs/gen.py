@@ -11,7 +11,7 @@ import numpy as np
 import torch
 
 _TAGS = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "bias": 6, "D": 7, "A": 8, "state": 9,
-         "dy": 10, "dlast": 11}
+         "dy": 10, "dlast": 11, "conv_w": 12, "conv_b": 13}
 _SLICE = 1 << 26  # elements drawn per slice when filling a large tensor
 
 
@@ -97,6 +97,20 @@ def bwd_upstream(batch, seqlen, d_inner, d_state=16, dtype="bf16", seed=0, devic
     dy = _normal((batch, seqlen, d_inner), 1.0, _torch_dtype(dtype), device, seed, "dy")
     dl = _normal((batch, d_inner, d_state), 1.0, torch.float32, device, seed, "dlast") if dlast else None
     return dy, dl
+
+
+def conv_params(d_inner, seed=0, device="cpu", bias="zero", width=4):
+    """Weights of the causal conv1d prologue: conv_w [d_inner, width] fp32 drawn
+    Kaiming-normal for a depthwise kernel (std sqrt(2 / width)), conv_b zero
+    (the deep-dive's initialisation, §3.3) or N(0, 0.1^2) with bias="normal"."""
+    w = _normal((d_inner, width), math.sqrt(2.0 / width), torch.float32, device, seed, "conv_w")
+    if bias == "zero":
+        b = torch.zeros(d_inner, dtype=torch.float32, device=device)
+    elif bias == "normal":
+        b = _normal((d_inner,), 0.1, torch.float32, device, seed, "conv_b")
+    else:
+        b = None
+    return w, b
 
 
 def step_inputs(batch, d_inner, d_state=16, dtype="bf16", seed=0, device="cpu", gate=True,
