@@ -277,6 +277,39 @@ def time_e2e(ss, torch, cfg, device, inp, steps):
     return ms, h2d, d2h
 
 
+def time_fwd_conv(ss, torch, cfg, device, steps, warmup):
+    """ss_fwd_conv (conv1d + SiLU prologue fused) on a forward workload, x in
+    place of u, timed back to back with CUDA events."""
+    from ss_inputs import conv_params, fwd_inputs
+    inp = fwd_inputs(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.d_state, cfg.dtype, cfg.seed, device,
+                     gate=cfg.gate, D_kind=cfg.D_kind)
+    w, cb = conv_params(cfg.d_inner, cfg.seed, device)
+    y = torch.empty_like(inp["u"])
+    st = torch.empty((cfg.batch, cfg.d_inner, cfg.d_state), dtype=torch.float32, device=device)
+    ws = torch.empty(ss.fwd_workspace_bytes(cfg.batch, cfg.seqlen, cfg.d_inner, cfg.dtype == "bf16"),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def one():
+        ss.ss_fwd_conv(inp["u"], w, inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"], z=inp["z"],
+                       delta_bias=inp["delta_bias"], conv_b=cb, y=y, last_state=st, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    del inp, y, st, ws
+    torch.cuda.empty_cache()
+    return ms
+
+
 def time_bwd(ss, torch, cfg, device, steps, warmup):
     """The backward (ss_bwd) of a forward workload: `steps` calls timed
     back to back with CUDA events, inputs and upstream gradients resident."""
@@ -473,6 +506,15 @@ def run_ours(args):
                             "graph_back_to_back_ms_per_step": dms_warm,
                             "graph_back_to_back_steps_per_s": 1e3 / dms_warm}
         torch.cuda.empty_cache()
+        for name in ("mamba2p8b", "mamba130m"):
+            c = CONFIGS[name]
+            cms = time_fwd_conv(ss, torch, c, device, 20, 3)
+            gbs = c.compulsory_bytes(conv=True) / (cms * 1e-3) / 1e9
+            fwd_ms = step_ms if name == cfg.name else extras.get(name, {}).get("ms_per_step")
+            extras["conv_fwd_" + name] = {"ms_per_step": cms, "GB_s": gbs, "frac_of_hbm": gbs / hbm,
+                                          "ratio_to_fwd": (cms / fwd_ms) if fwd_ms else None,
+                                          "note": "ss_fwd_conv: causal conv1d (width 4) + SiLU prologue "
+                                                  "fused; x read in place of u"}
         for name in ("mamba2p8b", "mamba130m"):
             c = CONFIGS[name]
             bms = time_bwd(ss, torch, c, device, 5, 2)

@@ -20,14 +20,15 @@ class FwdConfig:
         """Channel-timesteps: one (batch, t, channel) element of u."""
         return self.batch * self.seqlen * self.d_inner
 
-    def compulsory_bytes(self) -> int:
-        """Bytes every forward pass must move at least once: u, delta_raw, z
-        read and y written (one element each per channel-timestep), B and C
-        read, A/D/bias read and the final state written."""
+    def compulsory_bytes(self, conv=False) -> int:
+        """Bytes every forward pass must move at least once: u (or, with the
+        conv prologue, x), delta_raw, z read and y written (one element each
+        per channel-timestep), B and C read, A/D/bias (and conv weights) read
+        and the final state written."""
         e = 4 if self.dtype == "fp32" else 2
         per_chts = (4 if self.gate else 3) * e
         bc = 2 * self.batch * self.seqlen * self.d_state * e
-        params = self.d_inner * (self.d_state * 4 + 8)
+        params = self.d_inner * (self.d_state * 4 + 8 + (20 if conv else 0))
         state = self.batch * self.d_inner * self.d_state * 4
         return self.ch_ts * per_chts + bc + params + state
 
