@@ -50,7 +50,7 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--mode", choices=["fwd", "decode", "bwd"], default="fwd",
+    ap.add_argument("--mode", choices=["fwd", "decode", "bwd", "block"], default="fwd",
                     help="decode: time only the decode workload, --steps single-token steps; "
                          "bwd: time only ss_bwd on --workload")
     return ap.parse_args()
@@ -310,6 +310,40 @@ def time_fwd_conv(ss, torch, cfg, device, steps, warmup):
     return ms
 
 
+BLOCK_SHAPES = {   # Mamba-block inner path: (batch, L, d_model), d_inner = 2 d_model
+    "block_mamba130m": (8, 2048, 768),
+    "block_mamba2p8b": (4, 8192, 2560),
+}
+
+
+def time_block(ss, torch, name, device, steps, warmup):
+    """ss_block_fwd (projections on cuBLAS, conv, scan, out_proj) on random-init
+    weights, timed back to back with CUDA events.  Returns (ms, tokens,
+    projection FLOPs per call)."""
+    from ss_inputs import block_inputs
+    b, L, dm = BLOCK_SHAPES[name]
+    hidden, w = block_inputs(b, L, dm, seed=9, device=device)
+    out = torch.empty_like(hidden)
+    scratch = torch.empty(ss.block_scratch_bytes(w, b, L), dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+    for _ in range(warmup):
+        ss.ss_block_fwd(hidden, w, out=out, scratch=scratch, stream=stream)
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        ss.ss_block_fwd(hidden, w, out=out, scratch=scratch, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    di, rk = 2 * dm, w["x_proj_dt"].shape[0]
+    flops = 2 * b * L * (2 * di * dm + di * (rk + 32) + rk * di + dm * di)
+    del hidden, w, out, scratch
+    torch.cuda.empty_cache()
+    return ms, b * L, flops
+
+
 def time_bwd(ss, torch, cfg, device, steps, warmup):
     """The backward (ss_bwd) of a forward workload: `steps` calls timed
     back to back with CUDA events, inputs and upstream gradients resident."""
@@ -515,6 +549,13 @@ def run_ours(args):
                                           "ratio_to_fwd": (cms / fwd_ms) if fwd_ms else None,
                                           "note": "ss_fwd_conv: causal conv1d (width 4) + SiLU prologue "
                                                   "fused; x read in place of u"}
+        for name in BLOCK_SHAPES:
+            kms, toks, flops = time_block(ss, torch, name, device, 10, 3)
+            extras[name] = {"ms_per_step": kms, "tokens_per_s": toks / (kms * 1e-3),
+                            "projection_TFLOP_s": flops / (kms * 1e-3) / 1e12,
+                            "shape": dict(zip(("batch", "seq_len", "d_model"), BLOCK_SHAPES[name])),
+                            "note": "ss_block_fwd, random-init bf16 weights: in_proj, x_proj, dt_proj, "
+                                    "out_proj on cuBLAS; conv1d + SiLU and the scan in this library"}
         for name in ("mamba2p8b", "mamba130m"):
             c = CONFIGS[name]
             bms = time_bwd(ss, torch, c, device, 5, 2)
@@ -651,6 +692,22 @@ def run_bwd_only(args):
                       "ch_ts_per_s": c.ch_ts / (ms * 1e-3)}), flush=True)
 
 
+def run_block_only(args):
+    """Mamba-block inner path alone (for profiling): --steps ss_block_fwd calls
+    on the 2.8B-shaped block (or the 130M one with --workload mamba130m)."""
+    import torch
+
+    import selective_state_space_37_b200 as ss
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    ss.lib()
+    name = "block_" + args.workload
+    ms, toks, flops = time_block(ss, torch, name, device, max(args.steps, 1), args.warmup)
+    print(json.dumps({"metric": "Mamba block inner path tokens/s", "value": toks / (ms * 1e-3),
+                      "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "ms_per_step": ms,
+                      "workload": name, "projection_TFLOP_s": flops / (ms * 1e-3) / 1e12}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -659,6 +716,8 @@ def main():
         run_decode_only(args)
     elif args.mode == "bwd":
         run_bwd_only(args)
+    elif args.mode == "block":
+        run_block_only(args)
     else:
         run_ours(args)
 

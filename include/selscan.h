@@ -19,6 +19,8 @@
  *   ss_fwd_conv / ss_step_conv  the same with the causal conv1d + SiLU
  *            prologue of the Mamba block fused in ("Understanding Mamba and
  *            Selective State Space Models (SSMs)" §3.3).
+ *   ss_block_fwd  the Mamba block's inner forward path around the scan
+ *            (projections on cuBLAS, conv, scan, gate, output projection).
  *   ss_bwd   the gradients of ss_fwd's inputs from the gradient of its outputs
  *            (the models are trained and fine-tuned with gradient
  *            checkpointing: "Mamba 7.9.1" article §5.3-5.4; model-architecture
@@ -175,6 +177,49 @@ SS_API int ss_step_conv(float* state, float* conv_state, const void* x, const fl
                         const void* delta, const float* A, const void* B, const void* C, const float* D,
                         const void* z, void* y, const float* delta_bias, uint32_t flags, const ss_dims* dims,
                         const ss_launch* launch);
+
+/* Weights of one Mamba block (bf16 matrices row-major [out, in]; fp32 vectors).
+ * The block's interface is the README's Usage > Mamba (d_model, d_state = 16,
+ * d_conv = 4, expand = 2 so d_inner = 2 d_model; output shaped like the input;
+ * "roughly 3 · expand · d_model^2 parameters"); Δ comes from a linear
+ * projection whose bias sets its range (README, Initialization). */
+typedef struct ss_block_weights {
+    const void* in_proj_x;   /* [d_inner, d_model] bf16: x = hidden · in_proj_xᵀ */
+    const void* in_proj_z;   /* [d_inner, d_model] bf16: z = hidden · in_proj_zᵀ (the gate input) */
+    const float* conv_w;     /* [d_inner, 4] causal conv1d taps, tap 3 on the current token */
+    const float* conv_b;     /* [d_inner] or NULL */
+    const void* x_proj_dt;   /* [dt_rank, d_inner] bf16: Δ's low-rank input = u · x_proj_dtᵀ */
+    const void* x_proj_B;    /* [16, d_inner] bf16: B = u · x_proj_Bᵀ */
+    const void* x_proj_C;    /* [16, d_inner] bf16: C = u · x_proj_Cᵀ */
+    const void* dt_proj;     /* [d_inner, dt_rank] bf16: Δraw = (u · x_proj_dtᵀ) · dt_projᵀ */
+    const float* dt_bias;    /* [d_inner] Δ's projection bias (added before the softplus) */
+    const float* A;          /* [d_inner, 16] (negative; A = -exp(A_log)) */
+    const float* D;          /* [d_inner] or NULL */
+    const void* out_proj;    /* [d_model, d_inner] bf16: out = y · out_projᵀ */
+    int64_t d_model, d_inner, dt_rank;
+} ss_block_weights;
+
+/* ss_block_fwd -- forward of one Mamba block's inner path, bf16 activations:
+ *   x, z = hidden · in_proj_xᵀ, hidden · in_proj_zᵀ
+ *   u    = silu(conv_b + causal_conv4(x))                  (deep-dive §3.3)
+ *   Δraw = (u · x_proj_dtᵀ) · dt_projᵀ,  B = u · x_proj_Bᵀ,  C = u · x_proj_Cᵀ
+ *   y    = ss_fwd(u, Δraw, A, B, C, D, z, dt_bias, softplus on)
+ *   out  = y · out_projᵀ
+ *   hidden, out  [batch, seqlen, d_model] bf16 (device)
+ *   scratch      device buffer of at least ss_block_scratch_bytes() bytes,
+ *                16-byte aligned: the bf16 intermediates, the scan's
+ *                workspace and cuBLAS's workspace (nothing is allocated)
+ *   stream       cudaStream_t
+ * The projections run on cuBLAS (bf16 operands, fp32 accumulation); the conv
+ * and the scan are this library's kernels.  Errors: SS_ERR_INVALID_ARG for
+ * NULL/misaligned pointers or sizes (d_inner and d_model multiples of 8),
+ * SS_ERR_WORKSPACE for a small scratch, SS_ERR_CUDA for a CUDA or cuBLAS
+ * failure. */
+SS_API int ss_block_fwd(const void* hidden, void* out, const ss_block_weights* w, int64_t batch, int64_t seqlen,
+                        void* scratch, size_t scratch_bytes, void* stream);
+
+/* Scratch bytes ss_block_fwd needs (0 for invalid sizes). */
+SS_API size_t ss_block_scratch_bytes(const ss_block_weights* w, int64_t batch, int64_t seqlen);
 
 /* ss_bwd -- backward of ss_fwd: given dy = dJ/dy and optionally
  * dlast_state = dJ/dlast_state for a scalar J, writes dJ/d(input) for every

@@ -7,7 +7,8 @@ sm_100a in csrc/).  Three operations:
   ss_step  one decode step on a carried fp32 state;
   ss_bwd   gradients of ss_fwd's inputs from the gradients of its outputs;
   ss_fwd_conv / ss_step_conv  the same with the causal conv1d + SiLU
-           prologue fused in.
+           prologue fused in;
+  ss_block_fwd  the Mamba block's inner forward path around the scan.
 
 Build the library with ``python -m selective_state_space_37_b200.csrc.build``
 (``__graft_entry__.build()`` does the same).
@@ -15,11 +16,13 @@ Build the library with ``python -m selective_state_space_37_b200.csrc.build``
 from ._binding import (D_STATE, EXPORTED, LIB_PATH, SS_BF16, SS_DELTA_SOFTPLUS,
                        SS_ERR_CUDA, SS_ERR_INVALID_ARG, SS_ERR_TIMEOUT, SS_ERR_UNSUPPORTED,
                        SS_ERR_WORKSPACE, SS_FORCE_GENERAL_A, SS_OK, SS_SYNC_CHECK,
-                       SS_TEST_DROP_CARRY, SelscanError, bwd_workspace_bytes, fwd_chunk_len,
+                       SS_TEST_DROP_CARRY, SelscanError, block_scratch_bytes, bwd_workspace_bytes,
+                       fwd_chunk_len, ss_block_fwd,
                        fwd_workspace_bytes, lib, ss_bwd, ss_check, ss_dims, ss_fwd, ss_fwd_conv,
                        ss_launch, ss_step, ss_step_conv, status_string, workspace_for)
 
-__all__ = ["ss_fwd", "ss_step", "ss_bwd", "ss_fwd_conv", "ss_step_conv", "ss_check", "fwd_workspace_bytes", "fwd_chunk_len",
+__all__ = ["ss_fwd", "ss_step", "ss_bwd", "ss_fwd_conv", "ss_step_conv", "ss_block_fwd",
+           "block_scratch_bytes", "ss_check", "fwd_workspace_bytes", "fwd_chunk_len",
            "bwd_workspace_bytes",
            "status_string", "lib", "SelscanError", "ss_dims", "ss_launch", "workspace_for",
            "D_STATE", "EXPORTED", "LIB_PATH", "SS_OK", "SS_ERR_INVALID_ARG",

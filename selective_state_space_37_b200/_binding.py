@@ -34,7 +34,7 @@ D_STATE = 16
 # Every symbol include/selscan.h declares.
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
             "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
-            "ss_fwd_conv", "ss_step_conv")
+            "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_block_scratch_bytes")
 
 
 class ss_dims(ctypes.Structure):
@@ -46,6 +46,23 @@ class ss_launch(ctypes.Structure):
     _fields_ = [("stream", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("timeout_iters", ctypes.c_uint32),
                 ("chunk_len", ctypes.c_int32)]
+
+
+class ss_block_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("in_proj_x", "in_proj_z", "conv_w", "conv_b", "x_proj_dt",
+                                                "x_proj_B", "x_proj_C", "dt_proj", "dt_bias", "A", "D",
+                                                "out_proj")] + \
+               [("d_model", ctypes.c_int64), ("d_inner", ctypes.c_int64), ("dt_rank", ctypes.c_int64)]
+
+
+BLOCK_WEIGHT_SHAPES = {   # name: (shape as a function of (d_model, d_inner, dt_rank), dtype tag)
+    "in_proj_x": (lambda m, i, r: (i, m), "bf16"), "in_proj_z": (lambda m, i, r: (i, m), "bf16"),
+    "conv_w": (lambda m, i, r: (i, 4), "f32"), "conv_b": (lambda m, i, r: (i,), "f32"),
+    "x_proj_dt": (lambda m, i, r: (r, i), "bf16"), "x_proj_B": (lambda m, i, r: (D_STATE, i), "bf16"),
+    "x_proj_C": (lambda m, i, r: (D_STATE, i), "bf16"), "dt_proj": (lambda m, i, r: (i, r), "bf16"),
+    "dt_bias": (lambda m, i, r: (i,), "f32"), "A": (lambda m, i, r: (i, D_STATE), "f32"),
+    "D": (lambda m, i, r: (i,), "f32"), "out_proj": (lambda m, i, r: (m, i), "bf16"),
+}
 
 
 class SelscanError(RuntimeError):
@@ -103,6 +120,11 @@ def lib():
         L.ss_step_conv.argtypes = [f32p, f32p, vp, f32p, f32p, vp, f32p, vp, vp, f32p, vp, vp, f32p,
                                    ctypes.c_uint32, ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch)]
         L.ss_step_conv.restype = ctypes.c_int
+        L.ss_block_fwd.argtypes = [vp, vp, ctypes.POINTER(ss_block_weights), ctypes.c_int64, ctypes.c_int64,
+                                   vp, ctypes.c_size_t, vp]
+        L.ss_block_fwd.restype = ctypes.c_int
+        L.ss_block_scratch_bytes.argtypes = [ctypes.POINTER(ss_block_weights), ctypes.c_int64, ctypes.c_int64]
+        L.ss_block_scratch_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -349,6 +371,53 @@ def ss_step_conv(state, conv_state, x, conv_w, delta, A, B, C, D=None, z=None, d
     if rc != SS_OK:
         raise SelscanError(rc, "ss_step_conv")
     return y
+
+
+def _block_struct(weights, device):
+    d_inner, d_model = weights["in_proj_x"].shape
+    dt_rank = weights["x_proj_dt"].shape[0]
+    st = ss_block_weights()
+    for name, (shape_fn, tag) in BLOCK_WEIGHT_SHAPES.items():
+        t = weights.get(name)
+        if t is None and name in ("conv_b", "D"):
+            continue
+        _check(t, name, shape_fn(d_model, d_inner, dt_rank), torch.bfloat16 if tag == "bf16" else torch.float32,
+               device)
+        setattr(st, name, t.data_ptr())
+    st.d_model, st.d_inner, st.dt_rank = d_model, d_inner, dt_rank
+    return st
+
+
+def block_scratch_bytes(weights, batch, seqlen):
+    st = _block_struct(weights, weights["in_proj_x"].device)
+    return int(lib().ss_block_scratch_bytes(ctypes.byref(st), batch, seqlen))
+
+
+def ss_block_fwd(hidden, weights, *, out=None, scratch=None, stream=None):
+    """Forward of one Mamba block's inner path through libselscan's
+    ss_block_fwd.  hidden [batch, L, d_model] bf16; weights: a dict of
+    tensors named as the fields of ss_block_weights (bf16 matrices, fp32
+    vectors).  Returns out [batch, L, d_model] bf16."""
+    batch, L, d_model = hidden.shape
+    dev = hidden.device
+    st = _block_struct(weights, dev)
+    if st.d_model != d_model:
+        raise ValueError("hidden's last dimension must equal d_model")
+    _check(hidden, "hidden", (batch, L, d_model), torch.bfloat16, dev)
+    if out is None:
+        out = torch.empty_like(hidden)
+    _check(out, "out", (batch, L, d_model), torch.bfloat16, dev)
+    sh = _stream_handle(stream, dev)
+    need = int(lib().ss_block_scratch_bytes(ctypes.byref(st), batch, L))
+    if need == 0:
+        raise SelscanError(SS_ERR_INVALID_ARG, "ss_block_fwd")
+    if scratch is None:
+        scratch = workspace_for(need, dev, sh)
+    rc = lib().ss_block_fwd(_ptr(hidden), _ptr(out), ctypes.byref(st), batch, L, scratch.data_ptr(),
+                            scratch.numel() * scratch.element_size(), sh)
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_block_fwd")
+    return out
 
 
 def ss_check(workspace, stream=None, device=None):

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(os.path.dirname(HERE))
 LIB = os.path.join(HERE, "libselscan.so")
 SOURCES = ["selscan.cu"]
-HEADERS = ["common.cuh", "fwd.cuh", "bwd.cuh", "step.cuh"]
+HEADERS = ["common.cuh", "fwd.cuh", "bwd.cuh", "step.cuh", "block.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [
@@ -22,6 +22,7 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
     "--expt-relaxed-constexpr",
     "-cudart", "static",
+    "-lcublas", "-Xlinker", "-rpath", "-Xlinker", "/usr/local/cuda/lib64",
 ]
 
 

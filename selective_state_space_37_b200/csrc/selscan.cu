@@ -2,6 +2,7 @@
 // argument validation, work decomposition, workspace layout, TMA descriptor
 // set-up and kernel launches.  No allocation happens here: every buffer,
 // including the workspace, belongs to the caller.
+#include <cublas_v2.h>
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -10,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/selscan.h"
+#include "block.cuh"
 #include "bwd.cuh"
 #include "fwd.cuh"
 #include "step.cuh"
@@ -232,6 +234,61 @@ int launch_bwd_flags(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
     const bool hz = p.z != nullptr;
     if (p.softplus) return hz ? launch_bwd<IO, true, true>(p, ctas, stream) : launch_bwd<IO, true, false>(p, ctas, stream);
     return hz ? launch_bwd<IO, false, true>(p, ctas, stream) : launch_bwd<IO, false, false>(p, ctas, stream);
+}
+
+// ------------------------------------------------------------- Mamba block
+// One cuBLAS handle per (host thread, device): a handle binds one stream at a
+// time, so threads never share one.
+cublasHandle_t cublas_handle() {
+    thread_local cublasHandle_t handles[kMaxDevices] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!handles[dev] && cublasCreate(&handles[dev]) != CUBLAS_STATUS_SUCCESS) handles[dev] = nullptr;
+    return handles[dev];
+}
+
+// Row-major Y[M, N] = X[M, K] · W[N, K]ᵀ in bf16 with fp32 accumulation (a
+// column-major cuBLAS call computing Yᵀ = W · Xᵀ).
+bool gemm_bf16(cublasHandle_t h, const void* X, const void* W, void* Y, int64_t M, int64_t N, int64_t K) {
+    const float alpha = 1.0f, beta = 0.0f;
+    return cublasGemmEx(h, CUBLAS_OP_T, CUBLAS_OP_N, static_cast<int>(N), static_cast<int>(M), static_cast<int>(K),
+                        &alpha, W, CUDA_R_16BF, static_cast<int>(K), X, CUDA_R_16BF, static_cast<int>(K), &beta, Y,
+                        CUDA_R_16BF, static_cast<int>(N), CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) ==
+           CUBLAS_STATUS_SUCCESS;
+}
+
+constexpr size_t kCublasWorkspace = size_t(32) << 20;
+
+// Scratch layout of ss_block_fwd: bf16 x, z, u, Δraw, y [M, d_inner], the
+// Δ input [M, dt_rank], B, C [M, 16], then the scan's workspace and cuBLAS's.
+struct BlockPlan {
+    size_t x, z, u, delta, y, dtl, B, C, fwd_ws, fwd_ws_bytes, cublas_ws, total;
+};
+
+bool block_plan(const ss_block_weights* w, int64_t batch, int64_t seqlen, BlockPlan* pl) {
+    if (!w || batch < 0 || seqlen < 0 || w->d_model <= 0 || w->d_inner <= 0 || w->dt_rank <= 0) return false;
+    if (w->d_inner % 8 || w->d_model % 8 || w->dt_rank >= (int64_t(1) << 20)) return false;
+    const int64_t M = batch * seqlen;
+    const int64_t lim = int64_t(1) << 31;
+    if (M >= lim || w->d_inner >= lim || w->d_model >= lim) return false;
+    auto al = [](size_t v) { return (v + 255) / 256 * 256; };
+    size_t off = 0;
+    auto take = [&](size_t bytes) { const size_t o = off; off = al(off + bytes); return o; };
+    const size_t act = static_cast<size_t>(M) * w->d_inner * 2;
+    pl->x = take(act);
+    pl->z = take(act);
+    pl->u = take(act);
+    pl->delta = take(act);
+    pl->y = take(act);
+    pl->dtl = take(static_cast<size_t>(M) * w->dt_rank * 2);
+    pl->B = take(static_cast<size_t>(M) * kN * 2);
+    pl->C = take(static_cast<size_t>(M) * kN * 2);
+    ss_dims dims{batch, seqlen, w->d_inner, kN};
+    pl->fwd_ws_bytes = make_plan(&dims, SS_BF16 | SS_DELTA_SOFTPLUS, 0).total;
+    pl->fwd_ws = take(pl->fwd_ws_bytes);
+    pl->cublas_ws = take(kCublasWorkspace);
+    pl->total = off;
+    return true;
 }
 
 // ------------------------------------------------ allocation-free entry point
@@ -505,6 +562,66 @@ int ss_bwd(const void* u, const void* delta, const float* delta_bias, const floa
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
     }
+    return SS_OK;
+}
+
+size_t ss_block_scratch_bytes(const ss_block_weights* w, int64_t batch, int64_t seqlen) {
+    BlockPlan pl{};
+    return block_plan(w, batch, seqlen, &pl) ? pl.total : 0;
+}
+
+int ss_block_fwd(const void* hidden, void* out, const ss_block_weights* w, int64_t batch, int64_t seqlen,
+                 void* scratch, size_t scratch_bytes, void* stream_v) {
+    BlockPlan pl{};
+    if (!block_plan(w, batch, seqlen, &pl)) return SS_ERR_INVALID_ARG;
+    const int64_t M = batch * seqlen, di = w->d_inner, dm = w->d_model, rk = w->dt_rank;
+    if (M == 0) return SS_OK;
+    const void* need[] = {hidden, out, w->in_proj_x, w->in_proj_z, w->conv_w, w->x_proj_dt, w->x_proj_B,
+                          w->x_proj_C, w->dt_proj, w->dt_bias, w->A, w->out_proj};
+    for (const void* q : need)
+        if (!q || !aligned16(q)) return SS_ERR_INVALID_ARG;
+    if ((w->conv_b && !aligned16(w->conv_b)) || (w->D && !aligned16(w->D))) return SS_ERR_INVALID_ARG;
+    if (!scratch || scratch_bytes < pl.total || !aligned16(scratch)) return SS_ERR_WORKSPACE;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    cublasHandle_t h = cublas_handle();
+    if (!h) return SS_ERR_CUDA;
+    unsigned char* base = static_cast<unsigned char*>(scratch);
+    if (cublasSetStream(h, stream) != CUBLAS_STATUS_SUCCESS ||
+        cublasSetWorkspace(h, base + pl.cublas_ws, kCublasWorkspace) != CUBLAS_STATUS_SUCCESS)
+        return SS_ERR_CUDA;
+    void* x = base + pl.x;
+    void* z = base + pl.z;
+    void* u = base + pl.u;
+    void* delta = base + pl.delta;
+    void* y = base + pl.y;
+    void* dtl = base + pl.dtl;
+    void* Bm = base + pl.B;
+    void* Cm = base + pl.C;
+    // in_proj
+    if (!gemm_bf16(h, hidden, w->in_proj_x, x, M, di, dm) || !gemm_bf16(h, hidden, w->in_proj_z, z, M, di, dm))
+        return SS_ERR_CUDA;
+    // causal conv1d + SiLU
+    const dim3 grid(static_cast<unsigned>(ceil_div(di, kConvThreads)),
+                    static_cast<unsigned>(ceil_div(seqlen, kConvSteps)), static_cast<unsigned>(batch));
+    if (grid.y > 65535u || grid.z > 65535u) return SS_ERR_INVALID_ARG;
+    ss_conv_silu_kernel<__nv_bfloat16><<<grid, kConvThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(x), w->conv_w, w->conv_b, static_cast<__nv_bfloat16*>(u), seqlen, di);
+    if (cudaGetLastError() != cudaSuccess) return SS_ERR_CUDA;
+    // selection projections and Δ's projection
+    if (!gemm_bf16(h, u, w->x_proj_dt, dtl, M, rk, di) || !gemm_bf16(h, u, w->x_proj_B, Bm, M, kN, di) ||
+        !gemm_bf16(h, u, w->x_proj_C, Cm, M, kN, di) || !gemm_bf16(h, dtl, w->dt_proj, delta, M, di, rk))
+        return SS_ERR_CUDA;
+    // the selective scan, gated by z
+    ss_dims dims{batch, seqlen, di, kN};
+    ss_launch launch{};
+    launch.stream = stream;
+    launch.workspace = base + pl.fwd_ws;
+    launch.workspace_bytes = pl.fwd_ws_bytes;
+    int rc = ss_fwd(u, delta, w->dt_bias, w->A, Bm, Cm, w->D, z, y, nullptr, SS_BF16 | SS_DELTA_SOFTPLUS, &dims,
+                    &launch);
+    if (rc != SS_OK) return rc;
+    // out_proj
+    if (!gemm_bf16(h, y, w->out_proj, out, M, dm, di)) return SS_ERR_CUDA;
     return SS_OK;
 }
 

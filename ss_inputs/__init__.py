@@ -22,11 +22,14 @@ table, d_state = 16 as in the README usage example and the deep-dive article
   dlast_state ~ N(0, 1) fp32.
   Conv prologue (deep-dive §3.3): conv_w [d, 4] Kaiming-normal, std sqrt(2/4);
   conv_b = 0 (or N(0, 0.1^2) where a test covers the bias); x takes u's recipe.
+  Mamba block (README Usage > Mamba: expand 2, d_conv 4): hidden ~ N(0, 1) bf16,
+  projection matrices N(0, 1/fan_in) bf16, dt_rank = ceil(d_model / 16).
 """
 from .configs import CONFIGS, FwdConfig, StepConfig, get_config
-from .gen import (bwd_upstream, conv_params, fwd_inputs, step_inputs, step_sequence_inputs, general_A,
+from .gen import (block_inputs, bwd_upstream, conv_params, fwd_inputs, step_inputs, step_sequence_inputs, general_A,
                   to_f64, sample_channels)
 
 __all__ = ["CONFIGS", "FwdConfig", "StepConfig", "get_config", "fwd_inputs", "bwd_upstream", "conv_params",
+           "block_inputs",
            "step_inputs", "step_sequence_inputs", "general_A", "to_f64",
            "sample_channels"]

@@ -11,7 +11,8 @@ import numpy as np
 import torch
 
 _TAGS = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "bias": 6, "D": 7, "A": 8, "state": 9,
-         "dy": 10, "dlast": 11, "conv_w": 12, "conv_b": 13}
+         "dy": 10, "dlast": 11, "conv_w": 12, "conv_b": 13, "hidden": 14, "w_in_x": 15,
+         "w_in_z": 16, "w_x_dt": 17, "w_x_B": 18, "w_x_C": 19, "w_dt": 20, "w_out": 21}
 _SLICE = 1 << 26  # elements drawn per slice when filling a large tensor
 
 
@@ -111,6 +112,36 @@ def conv_params(d_inner, seed=0, device="cpu", bias="zero", width=4):
     else:
         b = None
     return w, b
+
+
+def block_inputs(batch, seqlen, d_model, d_state=16, seed=0, device="cpu", expand=2):
+    """One Mamba block's input and random-init weights (the block's interface:
+    d_inner = expand · d_model, d_conv = 4; dt_rank = ceil(d_model / 16)).
+    hidden ~ N(0, 1) bf16; projection matrices N(0, 1/fan_in) bf16; conv taps
+    Kaiming-normal, conv bias 0; dt_bias as delta_bias_init; A = -(n+1); D = 1.
+    Returns (hidden, weights dict named as ss_block_weights' fields)."""
+    d_inner = expand * d_model
+    rank = -(-d_model // 16)
+    bf = torch.bfloat16
+
+    def mat(tag, rows, cols):
+        return _normal((rows, cols), 1.0 / math.sqrt(cols), bf, device, seed, tag)
+
+    w = {
+        "in_proj_x": mat("w_in_x", d_inner, d_model),
+        "in_proj_z": mat("w_in_z", d_inner, d_model),
+        "x_proj_dt": mat("w_x_dt", rank, d_inner),
+        "x_proj_B": mat("w_x_B", d_state, d_inner),
+        "x_proj_C": mat("w_x_C", d_state, d_inner),
+        "dt_proj": mat("w_dt", d_inner, rank),
+        "out_proj": mat("w_out", d_model, d_inner),
+        "dt_bias": delta_bias_init(d_inner, seed, "cpu").to(device),
+        "A": structured_A(d_inner, d_state, device),
+        "D": torch.ones(d_inner, dtype=torch.float32, device=device),
+    }
+    w["conv_w"], w["conv_b"] = conv_params(d_inner, seed, device)
+    hidden = _normal((batch, seqlen, d_model), 1.0, bf, device, seed, "hidden")
+    return hidden, w
 
 
 def step_inputs(batch, d_inner, d_state=16, dtype="bf16", seed=0, device="cpu", gate=True,

@@ -67,3 +67,65 @@ def test_causality():
     np.testing.assert_array_equal(u0[:, :11], u1[:, :11])
     assert np.all(np.abs(u0[:, 11:15] - u1[:, 11:15]) > 0)
     np.testing.assert_array_equal(u0[:, 15:], u1[:, 15:])
+
+
+# --------------------------------------------------------- block composition
+from oracle.block import block_fwd, round_bf16  # noqa: E402
+
+
+def block_weights(rng, d_model=12, d_inner=24, N=16, rank=3):
+    return {
+        "in_proj_x": rng.normal(size=(d_inner, d_model)) * 0.3,
+        "in_proj_z": rng.normal(size=(d_inner, d_model)) * 0.3,
+        "conv_w": rng.normal(size=(d_inner, 4)) * 0.7,
+        "conv_b": np.zeros(d_inner),
+        "x_proj_dt": rng.normal(size=(rank, d_inner)) * 0.2,
+        "x_proj_B": rng.normal(size=(N, d_inner)) * 0.2,
+        "x_proj_C": rng.normal(size=(N, d_inner)) * 0.2,
+        "dt_proj": rng.normal(size=(d_inner, rank)) * 0.3,
+        "dt_bias": rng.normal(size=d_inner) * 0.3 - 2.0,
+        "A": -np.tile(np.arange(1, N + 1, dtype=np.float64), (d_inner, 1)),
+        "D": rng.normal(size=d_inner),
+        "out_proj": rng.normal(size=(d_model, d_inner)) * 0.2,
+    }
+
+
+def test_round_bf16_matches_torch():
+    rng = np.random.default_rng(5)
+    a = rng.normal(size=4096) * 10.0 ** rng.integers(-6, 6, size=4096)
+    ref = torch.from_numpy(a).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(round_bf16(a), ref)
+
+
+def test_block_zero_input_gives_zero_output():
+    """With zero conv bias, zero hidden makes x = u = 0, so every SSM input
+    term vanishes and out = 0 exactly."""
+    rng = np.random.default_rng(6)
+    w = block_weights(rng)
+    out = block_fwd(np.zeros((2, 9, 12)), w, store_bf16=False)
+    np.testing.assert_array_equal(out, 0.0)
+
+
+def test_block_is_linear_in_out_proj_and_shape_preserving():
+    rng = np.random.default_rng(7)
+    w = block_weights(rng)
+    h = rng.normal(size=(2, 10, 12))
+    o1 = block_fwd(h, w, store_bf16=False)
+    assert o1.shape == h.shape                       # README: y.shape == x.shape
+    w2 = dict(w)
+    w2["out_proj"] = 2.5 * w["out_proj"]
+    np.testing.assert_allclose(block_fwd(h, w2, store_bf16=False), 2.5 * o1, rtol=1e-12, atol=1e-14)
+
+
+def test_block_matches_its_steps_by_hand():
+    """The composition equals the steps run one by one with the pinned
+    conv and scan oracles (catches a swapped projection or a wrong gate input)."""
+    rng = np.random.default_rng(8)
+    w = block_weights(rng)
+    h = rng.normal(size=(1, 7, 12))
+    x = h @ w["in_proj_x"].T
+    z = h @ w["in_proj_z"].T
+    u = oracle.conv_silu(x, w["conv_w"], w["conv_b"])
+    y, _ = oracle.fwd(u, (u @ w["x_proj_dt"].T) @ w["dt_proj"].T, w["A"], u @ w["x_proj_B"].T,
+                      u @ w["x_proj_C"].T, D=w["D"], z=z, delta_bias=w["dt_bias"])
+    np.testing.assert_allclose(block_fwd(h, w, store_bf16=False), y @ w["out_proj"].T, rtol=1e-12, atol=1e-13)
