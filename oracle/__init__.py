@@ -50,6 +50,8 @@ def _lib():
         lib.ss_oracle_bwd_f64.restype = ctypes.c_int
         lib.ss_oracle_conv_silu_f64.argtypes = [_DP, _DP, _DP, _DP, _I64, _I64, _I64, _I64]
         lib.ss_oracle_conv_silu_f64.restype = ctypes.c_int
+        lib.ss_oracle_ssd_f64.argtypes = [_DP] * 9 + [_I64, _I64, _I64, _I64, _I64, ctypes.c_int]
+        lib.ss_oracle_ssd_f64.restype = ctypes.c_int
         lib.ss_oracle_set_mutation.argtypes = [ctypes.c_int]
         lib.ss_oracle_get_mutation.restype = ctypes.c_int
         lib.ss_oracle_max_threads.restype = ctypes.c_int
@@ -195,6 +197,31 @@ def conv_silu(x, w, bias=None):
     return u
 
 
+def ssd(x, dt, A, B, C, D=None, dt_bias=None, softplus=True):
+    """Multi-head scan with a scalar decay per head, float64, plain recurrence.
+    x [b, L, H, P]; dt [b, L, H]; A, D, dt_bias [H]; B, C [b, L, N].
+    Returns (y [b, L, H, P], final_state [b, H, P, N])."""
+    xa = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+    batch, L, H, P = xa.shape
+    N = np.asarray(B).shape[-1]
+    keep = []
+    ptrs = []
+    for v, shp in ((dt, (batch, L, H)), (dt_bias, (H,)), (A, (H,)), (B, (batch, L, N)), (C, (batch, L, N)),
+                   (D, (H,))):
+        a, pp = _arr(v, shp)
+        keep.append(a)
+        ptrs.append(_ptr(pp))
+    y = np.empty_like(xa)
+    st = np.empty((batch, H, P, N))
+    rc = _lib().ss_oracle_ssd_f64(xa.ctypes.data_as(_DP), ptrs[0], ptrs[1], ptrs[2], ptrs[3], ptrs[4], ptrs[5],
+                                  y.ctypes.data_as(_DP), st.ctypes.data_as(_DP), batch, L, H, P, N,
+                                  int(bool(softplus)))
+    if rc != 0:
+        raise ValueError(f"oracle ssd rejected sizes (rc={rc})")
+    del keep
+    return y, st
+
+
 def set_mutation(m: int) -> None:
     """Test-only: plant deliberate mistake number m (0 restores the oracle)."""
     _lib().ss_oracle_set_mutation(int(m))
@@ -216,7 +243,7 @@ def library_path() -> str:
     return _build.LIB
 
 
-__all__ = ["fwd", "fwd_chunked", "step", "bwd", "conv_silu", "set_mutation", "get_mutation",
+__all__ = ["fwd", "fwd_chunked", "step", "bwd", "conv_silu", "ssd", "set_mutation", "get_mutation",
            "max_threads", "set_threads", "library_path"]
 
 if os.environ.get("SS_ORACLE_THREADS"):

@@ -523,3 +523,55 @@ int ss_oracle_conv_silu_f64(const double* x, const double* w, const double* bias
     }
     return 0;
 }
+
+/* ---------------------------------------------------------------------------
+ * Multi-head scan with a scalar decay per head (the Mamba-2 / SSD model of
+ * the mamba README's Mamba-2 section and the model-architecture page's
+ * "Mamba-2 (multi-head, larger state)": headdim P, d_state N, ngroups = 1),
+ * double precision, plain recurrence.  For each (b, head h), with the head's
+ * P channels sharing Δ, B and C:
+ *   Δ_t     = softplus(dt_t,h + dt_bias_h)        (or dt + bias without softplus)
+ *   H_t[p,n] = exp(Δ_t A_h) H_{t-1}[p,n] + Δ_t B_t,n x_t,h,p
+ *   y_t,h,p = Σ_n C_t,n H_t[p,n] + D_h x_t,h,p
+ * starting from H = 0.  Layouts: x, y [batch, L, H, P]; dt [batch, L, H];
+ * A, dt_bias, D [H]; B, C [batch, L, N]; final_state [batch, H, P, N].
+ * ------------------------------------------------------------------------- */
+int ss_oracle_ssd_f64(const double* x, const double* dt, const double* dt_bias, const double* A,
+                      const double* B, const double* C, const double* D, double* y, double* final_state,
+                      int64_t batch, int64_t L, int64_t H, int64_t P, int64_t N, int softplus)
+{
+    if (batch < 0 || L < 0 || H < 0 || P < 1 || N < 1 || P * N > (1 << 20)) return -1;
+    int failed = 0;
+#pragma omp parallel for collapse(2) schedule(dynamic, 1)
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+            double* st = (double*)calloc((size_t)(P * N), sizeof(double));
+            if (!st) {
+#pragma omp atomic write
+                failed = 1;
+                continue;
+            }
+            for (int64_t t = 0; t < L; ++t) {
+                const double xr = dt[(b * L + t) * H + h] + (dt_bias ? dt_bias[h] : 0.0);
+                const double delta = softplus ? softplus_d(xr) : xr;
+                const double a = exp(delta * A[h]);
+                const double* Bt = B + (b * L + t) * N;
+                const double* Ct = C + (b * L + t) * N;
+                const double* xt = x + ((b * L + t) * H + h) * P;
+                double* yt = y + ((b * L + t) * H + h) * P;
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) {
+                        st[p * N + n] = a * st[p * N + n] + delta * Bt[n] * xt[p];
+                        acc += Ct[n] * st[p * N + n];
+                    }
+                    yt[p] = acc + (D ? D[h] * xt[p] : 0.0);
+                }
+            }
+            if (final_state)
+                for (int64_t i = 0; i < P * N; ++i) final_state[(b * H + h) * P * N + i] = st[i];
+            free(st);
+        }
+    }
+    return failed ? -1 : 0;
+}
