@@ -21,6 +21,8 @@
  *            Selective State Space Models (SSMs)" §3.3).
  *   ss_block_fwd  the Mamba block's inner forward path around the scan
  *            (projections on cuBLAS, conv, scan, gate, output projection).
+ *   ss_ssd_fwd  the multi-head scan with a scalar decay per head (Mamba-2's
+ *            SSD model) on the tensor cores.
  *   ss_bwd   the gradients of ss_fwd's inputs from the gradient of its outputs
  *            (the models are trained and fine-tuned with gradient
  *            checkpointing: "Mamba 7.9.1" article §5.3-5.4; model-architecture
@@ -220,6 +222,37 @@ SS_API int ss_block_fwd(const void* hidden, void* out, const ss_block_weights* w
 
 /* Scratch bytes ss_block_fwd needs (0 for invalid sizes). */
 SS_API size_t ss_block_scratch_bytes(const ss_block_weights* w, int64_t batch, int64_t seqlen);
+
+/* Sizes of a multi-head scalar-decay scan (ss_ssd_fwd). */
+typedef struct ss_ssd_dims {
+    int64_t batch;
+    int64_t seqlen;
+    int64_t nheads;
+    int64_t headdim;   /* must be 64 */
+    int64_t d_state;   /* 64 or 128 */
+} ss_ssd_dims;
+
+/* ss_ssd_fwd -- the multi-head scan with one scalar decay per head and step
+ * (the Mamba-2 / "State Space Dual" model of the mamba README's Mamba-2
+ * section and the model-architecture page's "Mamba-2 (multi-head, larger
+ * state)": headdim 64, d_state 64 or 128, ngroups 1 -- B and C shared by all
+ * heads).  For each (b, head h), with the head's channels p sharing Δ, B, C:
+ *   Δ_t = softplus(dt_t,h + dt_bias_h)   (dt + bias without SS_DELTA_SOFTPLUS)
+ *   H_t[p, n] = exp(Δ_t A_h) H_{t-1}[p, n] + Δ_t B_t,n x_t,h,p,   H_{-1} = 0
+ *   y_t,h,p = Σ_n C_t,n H_t[p, n] + D_h x_t,h,p
+ *   x, y         [batch, seqlen, nheads, headdim] bf16
+ *   dt           [batch, seqlen, nheads] bf16
+ *   A            [nheads] fp32 (negative); dt_bias, D [nheads] fp32 or NULL
+ *   B, C         [batch, seqlen, d_state] bf16
+ *   final_state  [batch, nheads, headdim, d_state] fp32 or NULL
+ *   flags        SS_DELTA_SOFTPLUS, SS_SYNC_CHECK (bf16 only; SS_BF16 ignored)
+ * Computed chunk by chunk (64 steps) as dense bf16 products with fp32
+ * accumulation on the tensor cores; the carried state stays on chip.
+ * Errors: SS_ERR_INVALID_ARG for NULL/misaligned pointers or sizes,
+ * SS_ERR_UNSUPPORTED for headdim != 64 or d_state not 64 or 128. */
+SS_API int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float* A, const void* B,
+                      const void* C, const float* D, void* y, float* final_state, uint32_t flags,
+                      const ss_ssd_dims* dims, void* stream);
 
 /* ss_bwd -- backward of ss_fwd: given dy = dJ/dy and optionally
  * dlast_state = dJ/dlast_state for a scalar J, writes dJ/d(input) for every

@@ -34,7 +34,7 @@ D_STATE = 16
 # Every symbol include/selscan.h declares.
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
             "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
-            "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_block_scratch_bytes")
+            "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_block_scratch_bytes", "ss_ssd_fwd")
 
 
 class ss_dims(ctypes.Structure):
@@ -63,6 +63,11 @@ BLOCK_WEIGHT_SHAPES = {   # name: (shape as a function of (d_model, d_inner, dt_
     "dt_bias": (lambda m, i, r: (i,), "f32"), "A": (lambda m, i, r: (i, D_STATE), "f32"),
     "D": (lambda m, i, r: (i,), "f32"), "out_proj": (lambda m, i, r: (m, i), "bf16"),
 }
+
+
+class ss_ssd_dims(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int64), ("seqlen", ctypes.c_int64), ("nheads", ctypes.c_int64),
+                ("headdim", ctypes.c_int64), ("d_state", ctypes.c_int64)]
 
 
 class SelscanError(RuntimeError):
@@ -125,6 +130,9 @@ def lib():
         L.ss_block_fwd.restype = ctypes.c_int
         L.ss_block_scratch_bytes.argtypes = [ctypes.POINTER(ss_block_weights), ctypes.c_int64, ctypes.c_int64]
         L.ss_block_scratch_bytes.restype = ctypes.c_size_t
+        L.ss_ssd_fwd.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, f32p, ctypes.c_uint32,
+                                 ctypes.POINTER(ss_ssd_dims), vp]
+        L.ss_ssd_fwd.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -418,6 +426,39 @@ def ss_block_fwd(hidden, weights, *, out=None, scratch=None, stream=None):
     if rc != SS_OK:
         raise SelscanError(rc, "ss_block_fwd")
     return out
+
+
+def ss_ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, *, softplus=True, y=None, final_state=None,
+               return_final_state=True, stream=None, sync_check=False):
+    """Multi-head scan with a scalar decay per head (Mamba-2's SSD model).
+    x [batch, L, nheads, 64] bf16; dt [batch, L, nheads] bf16; A [nheads] fp32;
+    B, C [batch, L, d_state] bf16 (d_state 64 or 128); D, dt_bias [nheads] fp32
+    or None.  Returns (y [batch, L, nheads, 64] bf16, final_state
+    [batch, nheads, 64, d_state] fp32 or None)."""
+    batch, L, H, P = x.shape
+    N = B.shape[-1]
+    dev = x.device
+    bf = torch.bfloat16
+    _check(x, "x", (batch, L, H, P), bf, dev)
+    _check(dt, "dt", (batch, L, H), bf, dev)
+    _check(B, "B", (batch, L, N), bf, dev)
+    _check(C, "C", (batch, L, N), bf, dev)
+    _check(A, "A", (H,), torch.float32, dev)
+    _check(D, "D", (H,), torch.float32, dev)
+    _check(dt_bias, "dt_bias", (H,), torch.float32, dev)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, "y", (batch, L, H, P), bf, dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
+    _check(final_state, "final_state", (batch, H, P, N), torch.float32, dev)
+    flags = (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
+    dims = ss_ssd_dims(batch, L, H, P, N)
+    rc = lib().ss_ssd_fwd(_ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+                          _ptr(final_state), flags, ctypes.byref(dims), _stream_handle(stream, dev))
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_ssd_fwd")
+    return y, final_state
 
 
 def ss_check(workspace, stream=None, device=None):

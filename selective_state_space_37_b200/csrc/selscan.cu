@@ -14,6 +14,7 @@
 #include "block.cuh"
 #include "bwd.cuh"
 #include "fwd.cuh"
+#include "ssd.cuh"
 #include "step.cuh"
 
 using namespace selscan;
@@ -558,6 +559,56 @@ int ss_bwd(const void* u, const void* delta, const float* delta_bias, const floa
     p.nseg = static_cast<int>(ceil_div(L, kSeg)); p.nblk = static_cast<int>(nblk);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
     rc = (flags & SS_BF16) ? launch_bwd_flags<__nv_bfloat16>(p, ctas, stream) : launch_bwd_flags<float>(p, ctas, stream);
+    if (rc != SS_OK) return rc;
+    if (flags & SS_SYNC_CHECK) {
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
+    }
+    return SS_OK;
+}
+
+int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float* A, const void* B, const void* C,
+               const float* D, void* y, float* final_state, uint32_t flags, const ss_ssd_dims* dims,
+               void* stream_v) {
+    if (!dims || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, H = dims->nheads;
+    if (batch < 0 || L < 0 || H < 0) return SS_ERR_INVALID_ARG;
+    if (dims->headdim != kSsdP || (dims->d_state != 64 && dims->d_state != 128)) return SS_ERR_UNSUPPORTED;
+    const int64_t lim = int64_t(1) << 31;
+    if (batch * H >= lim || L >= lim || double(batch) * double(L) * double(H) * kSsdP > 4.0e18)
+        return SS_ERR_INVALID_ARG;
+    if (batch == 0 || H == 0) return SS_OK;
+    if (!A || (L > 0 && (!x || !dt || !B || !C || !y))) return SS_ERR_INVALID_ARG;
+    const void* ptrs[] = {x, dt, dt_bias, A, B, C, D, y, final_state};
+    for (const void* q : ptrs)
+        if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    SsdParams p{};
+    p.x = static_cast<const __nv_bfloat16*>(x);
+    p.dt = static_cast<const __nv_bfloat16*>(dt);
+    p.dt_bias = dt_bias; p.A = A;
+    p.B = static_cast<const __nv_bfloat16*>(B);
+    p.C = static_cast<const __nv_bfloat16*>(C);
+    p.D = D;
+    p.y = static_cast<__nv_bfloat16*>(y);
+    p.final_state = final_state;
+    p.L = L; p.batch = static_cast<int>(batch); p.H = static_cast<int>(H);
+    p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
+    auto go = [&](auto kern, size_t smem) -> int {
+        static bool attr_set[2][kMaxDevices] = {{false}};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        const int which = smem > 50000 ? 1 : 0;
+        if (dev < 0 || dev >= kMaxDevices || !attr_set[which][dev]) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+                cudaSuccess)
+                return SS_ERR_CUDA;
+            if (dev >= 0 && dev < kMaxDevices) attr_set[which][dev] = true;
+        }
+        kern<<<static_cast<unsigned>(batch * H), kSsdThreads, smem, stream>>>(p);
+        return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+    };
+    const int rc = dims->d_state == 128 ? go(ss_ssd_kernel<128>, sizeof(SsdSmem<128>))
+                                        : go(ss_ssd_kernel<64>, sizeof(SsdSmem<64>));
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;

@@ -24,12 +24,14 @@ table, d_state = 16 as in the README usage example and the deep-dive article
   conv_b = 0 (or N(0, 0.1^2) where a test covers the bias); x takes u's recipe.
   Mamba block (README Usage > Mamba: expand 2, d_conv 4): hidden ~ N(0, 1) bf16,
   projection matrices N(0, 1/fan_in) bf16, dt_rank = ceil(d_model / 16).
+  Mamba-2 SSD scan (model-architecture page: headdim 64, d_state 128, one
+  group): x, B, C ~ N(0, 1) bf16, dt ~ N(0, 0.5^2), A_h = -U[1, 16], D = 1.
 """
 from .configs import CONFIGS, FwdConfig, StepConfig, get_config
-from .gen import (block_inputs, bwd_upstream, conv_params, fwd_inputs, step_inputs, step_sequence_inputs, general_A,
+from .gen import (block_inputs, ssd_inputs, bwd_upstream, conv_params, fwd_inputs, step_inputs, step_sequence_inputs, general_A,
                   to_f64, sample_channels)
 
 __all__ = ["CONFIGS", "FwdConfig", "StepConfig", "get_config", "fwd_inputs", "bwd_upstream", "conv_params",
-           "block_inputs",
+           "block_inputs", "ssd_inputs",
            "step_inputs", "step_sequence_inputs", "general_A", "to_f64",
            "sample_channels"]

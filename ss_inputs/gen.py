@@ -12,7 +12,8 @@ import torch
 
 _TAGS = {"u": 1, "delta": 2, "z": 3, "B": 4, "C": 5, "bias": 6, "D": 7, "A": 8, "state": 9,
          "dy": 10, "dlast": 11, "conv_w": 12, "conv_b": 13, "hidden": 14, "w_in_x": 15,
-         "w_in_z": 16, "w_x_dt": 17, "w_x_B": 18, "w_x_C": 19, "w_dt": 20, "w_out": 21}
+         "w_in_z": 16, "w_x_dt": 17, "w_x_B": 18, "w_x_C": 19, "w_dt": 20, "w_out": 21,
+         "ssd_x": 22, "ssd_dt": 23, "ssd_B": 24, "ssd_C": 25, "ssd_A": 26}
 _SLICE = 1 << 26  # elements drawn per slice when filling a large tensor
 
 
@@ -142,6 +143,25 @@ def block_inputs(batch, seqlen, d_model, d_state=16, seed=0, device="cpu", expan
     w["conv_w"], w["conv_b"] = conv_params(d_inner, seed, device)
     hidden = _normal((batch, seqlen, d_model), 1.0, bf, device, seed, "hidden")
     return hidden, w
+
+
+def ssd_inputs(batch, seqlen, nheads, d_state=128, headdim=64, seed=0, device="cpu"):
+    """Inputs of the multi-head scalar-decay scan (Mamba-2 SSD model): x ~ N(0,1)
+    [batch, L, nheads, headdim] bf16; dt ~ N(0, 0.5^2) [batch, L, nheads] bf16;
+    B, C ~ N(0,1) [batch, L, d_state] bf16 (one group); A_h = -U[1, 16] (one
+    negative decay rate per head); dt_bias as delta_bias_init; D = 1."""
+    bf = torch.bfloat16
+    g = _gen("cpu", seed, "ssd_A")
+    A = -(1.0 + 15.0 * torch.rand(nheads, generator=g, dtype=torch.float32)).to(device)
+    return {
+        "x": _normal((batch, seqlen, nheads, headdim), 1.0, bf, device, seed, "ssd_x"),
+        "dt": _normal((batch, seqlen, nheads), 0.5, bf, device, seed, "ssd_dt"),
+        "B": _normal((batch, seqlen, d_state), 1.0, bf, device, seed, "ssd_B"),
+        "C": _normal((batch, seqlen, d_state), 1.0, bf, device, seed, "ssd_C"),
+        "A": A,
+        "dt_bias": delta_bias_init(nheads, seed, "cpu").to(device),
+        "D": torch.ones(nheads, dtype=torch.float32, device=device),
+    }
 
 
 def step_inputs(batch, d_inner, d_state=16, dtype="bf16", seed=0, device="cpu", gate=True,

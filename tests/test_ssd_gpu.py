@@ -1,0 +1,56 @@
+"""GPU parity of ss_ssd_fwd (multi-head scalar-decay scan, tensor cores)
+against oracle.ssd (fp64 recurrence, pinned in test_oracle_ssd_pins.py).
+Bound: max|y - y_ref| <= 2e-2 · max|y_ref| and the same for the final state
+-- the kernel rounds the decay-weighted C Bᵀ, the scaled B and the carried
+state's copy to bf16 (2^-9 relative each) before the tensor-core products."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import selective_state_space_37_b200 as ss
+from gpu_util import rel_max_err
+from ss_inputs import ssd_inputs, to_f64
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+TOL = 2e-2
+
+
+def run_and_ref(inp, softplus=True):
+    y, st = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
+                          softplus=softplus, sync_check=True)
+    yr, sr = oracle.ssd(to_f64(inp["x"]), to_f64(inp["dt"]), to_f64(inp["A"]), to_f64(inp["B"]),
+                        to_f64(inp["C"]), D=to_f64(inp["D"]), dt_bias=to_f64(inp["dt_bias"]), softplus=softplus)
+    return y, st, yr, sr
+
+
+SHAPES = [(2, 100, 3, 64), (1, 64, 2, 128), (2, 257, 4, 128), (1, 1, 2, 64), (3, 130, 1, 128)]
+
+
+@pytest.mark.parametrize("shape", SHAPES, ids=[f"b{b}_L{l}_H{h}_N{n}" for b, l, h, n in SHAPES])
+def test_ssd_matches_oracle(shape):
+    b, L, H, N = shape
+    inp = ssd_inputs(b, L, H, N, seed=600 + L + H + N, device=DEV)
+    y, st, yr, sr = run_and_ref(inp)
+    assert rel_max_err(to_f64(y), yr) <= TOL
+    assert rel_max_err(to_f64(st), sr) <= TOL
+
+
+def test_ssd_softplus_off_and_no_skip():
+    inp = ssd_inputs(2, 150, 2, 64, seed=7, device=DEV)
+    inp["dt"] = (inp["dt"].float().abs() * 0.05 + 0.01).to(torch.bfloat16)
+    inp["D"] = None
+    inp["dt_bias"] = None
+    y, st, yr, sr = run_and_ref(inp, softplus=False)
+    assert rel_max_err(to_f64(y), yr) <= TOL
+    assert rel_max_err(to_f64(st), sr) <= TOL
+
+
+def test_ssd_zero_length_and_bad_sizes():
+    inp = ssd_inputs(2, 0, 3, 64, seed=1, device=DEV)
+    y, st = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], sync_check=True)
+    assert torch.count_nonzero(st).item() == 0
+    dims = ss.ss_ssd_dims(1, 8, 2, 32, 64)        # headdim 32: unsupported
+    rc = ss.lib().ss_ssd_fwd(None, None, None, inp["A"].data_ptr(), None, None, None, None, None, 0, dims, None)
+    assert rc == ss.SS_ERR_UNSUPPORTED
