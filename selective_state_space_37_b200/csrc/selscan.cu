@@ -191,6 +191,23 @@ int launch_variant(bool bf16, bool tma, Variant v, const FwdParams& p, int64_t i
                : launch_fwd<float, false, 1, 1, 8, false, CONV>(p, items, maps, stream);
 }
 
+template <int N>
+int launch_ssd(const SsdParams& p, int64_t ctas, cudaStream_t stream) {
+    auto kern = ss_ssd_kernel<N>;
+    const size_t smem = sizeof(SsdSmem<N>);
+    static bool attr_set[kMaxDevices] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+            return SS_ERR_CUDA;
+        if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
+    }
+    kern<<<static_cast<unsigned>(ctas), kSsdThreads, smem, stream>>>(p);
+    return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
+}
+
 int validate_dims(const ss_dims* dims, bool need_seqlen) {
     if (!dims) return SS_ERR_INVALID_ARG;
     if (dims->batch < 0 || dims->d_inner < 0 || dims->d_state <= 0) return SS_ERR_INVALID_ARG;
@@ -593,22 +610,7 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
     p.final_state = final_state;
     p.L = L; p.batch = static_cast<int>(batch); p.H = static_cast<int>(H);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
-    auto go = [&](auto kern, size_t smem) -> int {
-        static bool attr_set[2][kMaxDevices] = {{false}};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        const int which = smem > 50000 ? 1 : 0;
-        if (dev < 0 || dev >= kMaxDevices || !attr_set[which][dev]) {
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-                cudaSuccess)
-                return SS_ERR_CUDA;
-            if (dev >= 0 && dev < kMaxDevices) attr_set[which][dev] = true;
-        }
-        kern<<<static_cast<unsigned>(batch * H), kSsdThreads, smem, stream>>>(p);
-        return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
-    };
-    const int rc = dims->d_state == 128 ? go(ss_ssd_kernel<128>, sizeof(SsdSmem<128>))
-                                        : go(ss_ssd_kernel<64>, sizeof(SsdSmem<64>));
+    const int rc = dims->d_state == 128 ? launch_ssd<128>(p, batch * H, stream) : launch_ssd<64>(p, batch * H, stream);
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;

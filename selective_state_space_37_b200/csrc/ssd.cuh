@@ -43,15 +43,28 @@ struct SsdParams {
 };
 
 template <int N>
-struct SsdSmem {
+struct SsdTiles {
     __nv_bfloat16 X[kSsdQ][kSsdP + kSsdPad];    // x of the chunk [t][p]
     __nv_bfloat16 Bt[kSsdQ][N + kSsdPad];       // B [s][n]; then scaled by e^{cum_end - cum_s} Δ_s
     __nv_bfloat16 Ct[kSsdQ][N + kSsdPad];       // C [t][n]
+};
+
+template <int N>
+struct SsdSmem {
+    SsdTiles<N> tile[2];                        // this chunk's tiles and the next one's, in flight
     __nv_bfloat16 G[kSsdP][N + kSsdPad];        // carried state, bf16 copy [p][n]
-    float a[kSsdQ];                             // Δ_t A
     float cum[kSsdQ];                           // inclusive prefix of Δ A
     float dlt[kSsdQ];                           // Δ_t
 };
+
+// 16-byte asynchronous copy global -> shared; zero fill when !valid.
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -95,38 +108,66 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
     for (int i = tid; i < kSsdP * (N + kSsdPad) / 2; i += kSsdThreads)
         reinterpret_cast<uint32_t*>(&S.G[0][0])[i] = 0u;
 
-    for (int64_t t0 = 0; t0 < p.L; t0 += kSsdQ) {
+    // Copies of one chunk's x, B, C tiles (rows past the sequence read as zero).
+    auto issue_tiles = [&](int64_t t0, SsdTiles<N>& T) {
         const int q = static_cast<int>(p.L - t0 < kSsdQ ? p.L - t0 : kSsdQ);
-        __syncthreads();   // the previous chunk is done with every tile
-        // ---------------------------------------------------------- tiles
-        const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
         for (int i = tid; i < kSsdQ * (kSsdP / 8); i += kSsdThreads) {
             const int r = i / (kSsdP / 8), k = (i % (kSsdP / 8)) * 8;
-            const __nv_bfloat16* src = p.x + ((static_cast<int64_t>(b) * p.L + t0 + r) * p.H + h) * kSsdP + k;
-            *reinterpret_cast<uint4*>(&S.X[r][k]) = r < q ? *reinterpret_cast<const uint4*>(src) : zero4;
+            const int rr = r < q ? r : 0;
+            cp_async16(&T.X[r][k], p.x + ((static_cast<int64_t>(b) * p.L + t0 + rr) * p.H + h) * kSsdP + k, r < q);
         }
         for (int i = tid; i < kSsdQ * (N / 8); i += kSsdThreads) {
             const int r = i / (N / 8), k = (i % (N / 8)) * 8;
-            const int64_t off = (static_cast<int64_t>(b) * p.L + t0 + r) * N + k;
-            *reinterpret_cast<uint4*>(&S.Bt[r][k]) = r < q ? *reinterpret_cast<const uint4*>(p.B + off) : zero4;
-            *reinterpret_cast<uint4*>(&S.Ct[r][k]) = r < q ? *reinterpret_cast<const uint4*>(p.C + off) : zero4;
+            const int rr = r < q ? r : 0;
+            const int64_t off = (static_cast<int64_t>(b) * p.L + t0 + rr) * N + k;
+            cp_async16(&T.Bt[r][k], p.B + off, r < q);
+            cp_async16(&T.Ct[r][k], p.C + off, r < q);
         }
-        if (tid < kSsdQ) {
-            float dl = 0.0f;
-            if (tid < q) {
-                const float xr = __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t0 + tid) * p.H + h]) + bias;
-                dl = p.softplus ? softplus_accurate(xr) : xr;
+    };
+    // Warp 0 holds Δraw of the next chunk's steps 2·lane and 2·lane + 1.
+    float dtn[2] = {0.0f, 0.0f};
+    auto load_dt = [&](int64_t t0) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int64_t t = t0 + 2 * lane + e;
+            dtn[e] = t < p.L ? __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t) * p.H + h]) : 0.0f;
+        }
+    };
+    if (p.L > 0) issue_tiles(0, S.tile[0]);
+    cp_async_commit();
+    if (w == 0) load_dt(0);
+
+    int cb = 0;   // tile buffer of the current chunk
+    for (int64_t t0 = 0; t0 < p.L; t0 += kSsdQ, cb ^= 1) {
+        const int q = static_cast<int>(p.L - t0 < kSsdQ ? p.L - t0 : kSsdQ);
+        __syncthreads();   // the previous chunk is done with every tile and with cum / dlt
+        if (t0 + kSsdQ < p.L) issue_tiles(t0 + kSsdQ, S.tile[cb ^ 1]);
+        cp_async_commit();
+        if (w == 0) {
+            // Δ and the inclusive prefix of Δ A over the chunk: each lane takes two
+            // consecutive steps, then one scan over the 32 pair sums.
+            float dl[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                const float xr = dtn[e] + bias;
+                dl[e] = (2 * lane + e < q) ? (p.softplus ? softplus_accurate(xr) : xr) : 0.0f;
             }
-            S.dlt[tid] = dl;
-            S.a[tid] = dl * Ah;
+            const float a1 = dl[1] * Ah;
+            float sc = fmaf(dl[0], Ah, a1);
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, sc, o);
+                if (lane >= o) sc += v;
+            }
+            S.cum[2 * lane + 1] = sc;
+            S.cum[2 * lane] = sc - a1;
+            S.dlt[2 * lane] = dl[0];
+            S.dlt[2 * lane + 1] = dl[1];
+            if (t0 + kSsdQ < p.L) load_dt(t0 + kSsdQ);
         }
+        cp_async_wait_one();   // this thread's copies of the current chunk have landed
         __syncthreads();
-        if (tid < kSsdQ) {   // inclusive prefix of Δ A, in time order
-            float s = 0.0f;
-            for (int r = 0; r <= tid; ++r) s += S.a[r];
-            S.cum[tid] = s;
-        }
-        __syncthreads();
+        auto& T = S.tile[cb];
         const float cum_end = S.cum[kSsdQ - 1];
 
         // ------------------------------------------ S = C Bᵀ, causal tiles only
@@ -137,12 +178,12 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
 #pragma unroll
         for (int k = 0; k < N; k += 16) {
             uint32_t af[4];
-            ldsm_x4(af, &S.Ct[16 * w + (lane & 7) + ((lane >> 3) & 1) * 8][k + (lane >> 4) * 8]);
+            ldsm_x4(af, &T.Ct[16 * w + (lane & 7) + ((lane >> 3) & 1) * 8][k + (lane >> 4) * 8]);
 #pragma unroll
             for (int j = 0; j < 8; j += 2) {
                 if (j < nS) {
                     uint32_t bf[4];
-                    ldsm_x4(bf, &S.Bt[8 * j + (lane & 7) + (lane >> 4) * 8][k + ((lane >> 3) & 1) * 8]);
+                    ldsm_x4(bf, &T.Bt[8 * j + (lane & 7) + (lane >> 4) * 8][k + ((lane >> 3) & 1) * 8]);
                     mma_bf16(accS[j], af, bf[0], bf[1]);
                     mma_bf16(accS[j + 1], af, bf[2], bf[3]);
                 }
@@ -152,7 +193,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
         for (int i = tid; i < kSsdQ * (N / 2); i += kSsdThreads) {
             const int r = i / (N / 2), k = (i % (N / 2)) * 2;
             const float sc = __expf(cum_end - S.cum[r]) * S.dlt[r];
-            __nv_bfloat162* v = reinterpret_cast<__nv_bfloat162*>(&S.Bt[r][k]);
+            __nv_bfloat162* v = reinterpret_cast<__nv_bfloat162*>(&T.Bt[r][k]);
             const float2 f = __bfloat1622float2(*v);
             *v = __floats2bfloat162_rn(f.x * sc, f.y * sc);
         }
@@ -190,7 +231,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
 #pragma unroll
             for (int k = 0; k < N; k += 16) {
                 uint32_t af[4];
-                ldsm_x4(af, &S.Ct[16 * w + (lane & 7) + ((lane >> 3) & 1) * 8][k + (lane >> 4) * 8]);
+                ldsm_x4(af, &T.Ct[16 * w + (lane & 7) + ((lane >> 3) & 1) * 8][k + (lane >> 4) * 8]);
 #pragma unroll
                 for (int j = 0; j < 8; j += 2) {
                     uint32_t bf[4];
@@ -212,7 +253,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
 #pragma unroll
                 for (int j = 0; j < 8; j += 2) {
                     uint32_t bf[4];
-                    ldsm_x4_t(bf, &S.X[16 * kb + (lane & 7) + ((lane >> 3) & 1) * 8][8 * j + (lane >> 4) * 8]);
+                    ldsm_x4_t(bf, &T.X[16 * kb + (lane & 7) + ((lane >> 3) & 1) * 8][8 * j + (lane >> 4) * 8]);
                     mma_bf16(accY[j], mf[kb], bf[0], bf[1]);
                     mma_bf16(accY[j + 1], mf[kb], bf[2], bf[3]);
                 }
@@ -225,7 +266,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 const int t = half ? t_hi : t_lo;
-                const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&S.X[t][pc]));
+                const float2 xv = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&T.X[t][pc]));
                 const float y0 = fmaf(Dh, xv.x, accY[j][2 * half]);
                 const float y1 = fmaf(Dh, xv.y, accY[j][2 * half + 1]);
                 if (t < q)
@@ -245,11 +286,11 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
 #pragma unroll
         for (int ks = 0; ks < kSsdQ; ks += 16) {
             uint32_t af[4];   // Xᵀ rows p = 16w.., k = s
-            ldsm_x4_t(af, &S.X[ks + (lane & 7) + (lane >> 4) * 8][16 * w + ((lane >> 3) & 1) * 8]);
+            ldsm_x4_t(af, &T.X[ks + (lane & 7) + (lane >> 4) * 8][16 * w + ((lane >> 3) & 1) * 8]);
 #pragma unroll
             for (int j = 0; j < NT; j += 2) {
                 uint32_t bf[4];
-                ldsm_x4_t(bf, &S.Bt[ks + (lane & 7) + ((lane >> 3) & 1) * 8][8 * j + (lane >> 4) * 8]);
+                ldsm_x4_t(bf, &T.Bt[ks + (lane & 7) + ((lane >> 3) & 1) * 8][8 * j + (lane >> 4) * 8]);
                 mma_bf16(accG[j], af, bf[0], bf[1]);
                 mma_bf16(accG[j + 1], af, bf[2], bf[3]);
             }
