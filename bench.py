@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "selective-scan fwd effective HBM GB/s (% of B200 peak); decode steps/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 # device code of the forward kernel (the profile's traffic figure is used only
 # while these files are unchanged)
 KERNEL_SOURCES = ["selective_state_space_37_b200/csrc/fwd.cuh",
@@ -64,6 +65,17 @@ def peaks():
         return float(pk["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """(burst, sustained) dense bf16 TFLOP/s from MEASURED_PEAKS.json, with its kind."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return "measured", float(pk["bf16_tflops"]), float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"]))
+    except Exception:
+        return "fallback", FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS
 
 
 def kernel_source_hash():
@@ -344,6 +356,51 @@ def time_block(ss, torch, name, device, steps, warmup):
     return ms, b * L, flops
 
 
+SSD_SHAPES = {   # multi-head scalar-decay scan: (batch, L, nheads, d_state), headdim 64
+    "ssd_mamba2_2p7b": (4, 8192, 80, 128),    # d_model 2560, expand 2: 5120 = 80 heads x 64
+    "ssd_mamba2_130m": (8, 2048, 24, 128),    # d_model 768: 1536 = 24 heads x 64
+}
+
+
+def ssd_useful_flops(b, L, H, N, Q=64, P=64):
+    """Dense-equivalent FLOPs of the chunked form per call: the causal half of
+    C Bᵀ (Q/2 · N per step) and of the masked product with x (Q/2 · P), the
+    carried state into the outputs (N · P) and the state update (N · P)."""
+    return 2 * (Q // 2 * N + Q // 2 * P + 2 * N * P) * b * L * H
+
+
+def ssd_compulsory_bytes(b, L, H, N, P=64):
+    return 2 * (2 * b * L * H * P + 2 * b * L * N + b * L * H) + 4 * b * H * P * N + 12 * H
+
+
+def time_ssd(ss, torch, name, device, steps, warmup):
+    from ss_inputs import ssd_inputs
+    b, L, H, N = SSD_SHAPES[name]
+    inp = ssd_inputs(b, L, H, N, seed=3, device=device)
+    y = torch.empty_like(inp["x"])
+    st = torch.empty((b, H, 64, N), dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def one():
+        ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
+                      y=y, final_state=st, stream=stream)
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / steps
+    del inp, y, st
+    torch.cuda.empty_cache()
+    return ms
+
+
 def time_bwd(ss, torch, cfg, device, steps, warmup):
     """The backward (ss_bwd) of a forward workload: `steps` calls timed
     back to back with CUDA events, inputs and upstream gradients resident."""
@@ -549,6 +606,16 @@ def run_ours(args):
                                           "ratio_to_fwd": (cms / fwd_ms) if fwd_ms else None,
                                           "note": "ss_fwd_conv: causal conv1d (width 4) + SiLU prologue "
                                                   "fused; x read in place of u"}
+        _, bf16_peak, _ = tensor_peak()
+        for name, (b, L, H, N) in SSD_SHAPES.items():
+            sms = time_ssd(ss, torch, name, device, 10, 3)
+            tf = ssd_useful_flops(b, L, H, N) / (sms * 1e-3) / 1e12
+            gbs = ssd_compulsory_bytes(b, L, H, N) / (sms * 1e-3) / 1e9
+            extras[name] = {"ms_per_step": sms, "TFLOP_s": tf, "frac_of_bf16_peak": tf / bf16_peak,
+                            "GB_s": gbs, "frac_of_hbm": gbs / hbm,
+                            "shape": {"batch": b, "seq_len": L, "nheads": H, "headdim": 64, "d_state": N},
+                            "note": "ss_ssd_fwd: chunked matrix form on mma.sync bf16 tensor-core "
+                                    "instructions; TFLOP_s counts the causal-half products"}
         for name in BLOCK_SHAPES:
             kms, toks, flops = time_block(ss, torch, name, device, 10, 3)
             extras[name] = {"ms_per_step": kms, "tokens_per_s": toks / (kms * 1e-3),
