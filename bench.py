@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--mode", choices=["fwd", "decode", "bwd", "block"], default="fwd",
+    ap.add_argument("--mode", choices=["fwd", "decode", "bwd", "block", "ssd"], default="fwd",
                     help="decode: time only the decode workload, --steps single-token steps; "
                          "bwd: time only ss_bwd on --workload")
     return ap.parse_args()
@@ -775,6 +775,25 @@ def run_block_only(args):
                       "workload": name, "projection_TFLOP_s": flops / (ms * 1e-3) / 1e12}), flush=True)
 
 
+def run_ssd_only(args):
+    """SSD scan alone (for profiling): --steps ss_ssd_fwd calls on the
+    2.7B-shaped Mamba-2 layer (or the 130M one with --workload mamba130m)."""
+    import torch
+
+    import selective_state_space_37_b200 as ss
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    ss.lib()
+    name = "ssd_mamba2_130m" if args.workload == "mamba130m" else "ssd_mamba2_2p7b"
+    b, L, H, N = SSD_SHAPES[name]
+    ms = time_ssd(ss, torch, name, device, max(args.steps, 1), args.warmup)
+    _, peak, _ = tensor_peak()
+    tf = ssd_useful_flops(b, L, H, N) / (ms * 1e-3) / 1e12
+    print(json.dumps({"metric": "SSD scan useful TFLOP/s", "value": tf, "unit": "TFLOP/s", "n_gpus": 1,
+                      "steps": args.steps, "ms_per_step": ms, "workload": name, "frac_of_bf16_peak": tf / peak,
+                      "GB_s": ssd_compulsory_bytes(b, L, H, N) / (ms * 1e-3) / 1e9}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
@@ -785,6 +804,8 @@ def main():
         run_bwd_only(args)
     elif args.mode == "block":
         run_block_only(args)
+    elif args.mode == "ssd":
+        run_ssd_only(args)
     else:
         run_ours(args)
 
