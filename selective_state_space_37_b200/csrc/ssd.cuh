@@ -16,6 +16,8 @@
 // chunks never leaves the SM.  The products use the warp-level mma.sync
 // m16n8k16 bf16 instructions with ldmatrix fragment loads from padded shared
 // tiles; warp w owns rows 16w..16w+15 of S and Y (time) and of G (channel).
+// Three CTAs share an SM (62 KB of shared memory and <= 168 registers each),
+// so one CTA's tile copies (cp.async) and barriers overlap the others' products.
 #pragma once
 
 #include "common.cuh"
@@ -51,7 +53,7 @@ struct SsdTiles {
 
 template <int N>
 struct SsdSmem {
-    SsdTiles<N> tile[2];                        // this chunk's tiles and the next one's, in flight
+    SsdTiles<N> tile[1];                        // this chunk's tiles
     __nv_bfloat16 G[kSsdP][N + kSsdPad];        // carried state, bf16 copy [p][n]
     float cum[kSsdQ];                           // inclusive prefix of Δ A
     float dlt[kSsdQ];                           // Δ_t
@@ -64,7 +66,7 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src, bool vali
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p) {
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
@@ -90,7 +92,7 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }
 
 template <int N>
-__global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_constant__ SsdParams p) {
+__global__ void __launch_bounds__(kSsdThreads, 3) ss_ssd_kernel(const __grid_constant__ SsdParams p) {
     constexpr int NT = N / 8;          // n8 tiles of the state width
     extern __shared__ __align__(16) unsigned char ssd_smem_raw[];
     auto& S = *reinterpret_cast<SsdSmem<N>*>(ssd_smem_raw);
@@ -133,15 +135,12 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
             dtn[e] = t < p.L ? __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t) * p.H + h]) : 0.0f;
         }
     };
-    if (p.L > 0) issue_tiles(0, S.tile[0]);
-    cp_async_commit();
     if (w == 0) load_dt(0);
 
-    int cb = 0;   // tile buffer of the current chunk
-    for (int64_t t0 = 0; t0 < p.L; t0 += kSsdQ, cb ^= 1) {
+    for (int64_t t0 = 0; t0 < p.L; t0 += kSsdQ) {
         const int q = static_cast<int>(p.L - t0 < kSsdQ ? p.L - t0 : kSsdQ);
         __syncthreads();   // the previous chunk is done with every tile and with cum / dlt
-        if (t0 + kSsdQ < p.L) issue_tiles(t0 + kSsdQ, S.tile[cb ^ 1]);
+        issue_tiles(t0, S.tile[0]);
         cp_async_commit();
         if (w == 0) {
             // Δ and the inclusive prefix of Δ A over the chunk: each lane takes two
@@ -165,16 +164,20 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
             S.dlt[2 * lane + 1] = dl[1];
             if (t0 + kSsdQ < p.L) load_dt(t0 + kSsdQ);
         }
-        cp_async_wait_one();   // this thread's copies of the current chunk have landed
+        cp_async_wait_all();   // this thread's copies of the chunk have landed
         __syncthreads();
-        auto& T = S.tile[cb];
+        auto& T = S.tile[0];
         const float cum_end = S.cum[kSsdQ - 1];
 
-        // ------------------------------------------ S = C Bᵀ, causal tiles only
+        // ----------- S = C Bᵀ (causal tiles only) and C G_inᵀ, sharing C's fragments
         const int nS = 2 * (w + 1);                 // s-tiles 0 .. 16w+15
-        float accS[8][4];
+        const bool carry = t0 > 0;                  // G_in is zero before the first chunk
+        float accS[8][4], accY[8][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) accS[j][0] = accS[j][1] = accS[j][2] = accS[j][3] = 0.0f;
+        for (int j = 0; j < 8; ++j) {
+            accS[j][0] = accS[j][1] = accS[j][2] = accS[j][3] = 0.0f;
+            accY[j][0] = accY[j][1] = accY[j][2] = accY[j][3] = 0.0f;
+        }
 #pragma unroll
         for (int k = 0; k < N; k += 16) {
             uint32_t af[4];
@@ -186,6 +189,12 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
                     ldsm_x4(bf, &T.Bt[8 * j + (lane & 7) + (lane >> 4) * 8][k + ((lane >> 3) & 1) * 8]);
                     mma_bf16(accS[j], af, bf[0], bf[1]);
                     mma_bf16(accS[j + 1], af, bf[2], bf[3]);
+                }
+                if (carry) {
+                    uint32_t gf[4];
+                    ldsm_x4(gf, &S.G[8 * j + (lane & 7) + (lane >> 4) * 8][k + ((lane >> 3) & 1) * 8]);
+                    mma_bf16(accY[j], af, gf[0], gf[1]);
+                    mma_bf16(accY[j + 1], af, gf[2], gf[3]);
                 }
             }
         }
@@ -224,22 +233,7 @@ __global__ void __launch_bounds__(kSsdThreads, 2) ss_ssd_kernel(const __grid_con
         }
 
         // ---------------------------------------- Y = e^{cum} (C G_inᵀ) + M X
-        float accY[8][4];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) accY[j][0] = accY[j][1] = accY[j][2] = accY[j][3] = 0.0f;
-        if (t0 > 0) {
-#pragma unroll
-            for (int k = 0; k < N; k += 16) {
-                uint32_t af[4];
-                ldsm_x4(af, &T.Ct[16 * w + (lane & 7) + ((lane >> 3) & 1) * 8][k + (lane >> 4) * 8]);
-#pragma unroll
-                for (int j = 0; j < 8; j += 2) {
-                    uint32_t bf[4];
-                    ldsm_x4(bf, &S.G[8 * j + (lane & 7) + (lane >> 4) * 8][k + ((lane >> 3) & 1) * 8]);
-                    mma_bf16(accY[j], af, bf[0], bf[1]);
-                    mma_bf16(accY[j + 1], af, bf[2], bf[3]);
-                }
-            }
+        if (carry) {
             const float e_lo = __expf(cum_lo), e_hi = __expf(cum_hi);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
