@@ -253,14 +253,15 @@ def bwd_workspace_bytes(batch, seqlen, d_inner, bf16=True, d_state=D_STATE):
 
 
 def ss_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, dlast_state=None, *,
-           softplus=True, grads=None, workspace=None, stream=None, sync_check=False):
+           softplus=True, grads=None, chunk_len=0, workspace=None, stream=None, sync_check=False):
     """Backward of ss_fwd through libselscan's ss_bwd.
 
     Same inputs as ss_fwd plus dy [batch, L, d_inner] (the element type of u)
     and dlast_state [batch, d_inner, 16] fp32 or None.  Returns a dict with
     du, ddelta, dz (element type of u; dz only with z), dA [d_inner, 16],
     dB, dC [batch, L, 16], dD and ddelta_bias [d_inner] (fp32; only with D /
-    delta_bias).  `grads` may supply preallocated output tensors by name.
+    delta_bias).  `grads` may supply preallocated output tensors by name;
+    chunk_len > 0 fixes the time-chunk length (0: the library's choice).
     """
     if u.dim() != 3:
         raise ValueError("u must be [batch, L, d_inner]")
@@ -296,7 +297,7 @@ def ss_bwd(u, delta, A, B, C, dy, D=None, z=None, delta_bias=None, dlast_state=N
     need = int(lib().ss_bwd_workspace_bytes(ctypes.byref(dims), flags))
     if workspace is None:
         workspace = workspace_for(need, dev, sh)
-    launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(), 0, 0)
+    launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(), 0, int(chunk_len))
     rc = lib().ss_bwd(_ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
                       _ptr(dy), _ptr(dlast_state), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]),
                       _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g.get("dD")), _ptr(g.get("dz")),

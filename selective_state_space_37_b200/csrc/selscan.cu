@@ -224,34 +224,110 @@ int validate_dims(const ss_dims* dims, bool need_seqlen) {
     return SS_OK;
 }
 
-// Backward: forward-state checkpoints, [batch][ceil(L / kSeg)][d][kN] fp32.
-size_t bwd_workspace(const ss_dims* dims) {
-    const int64_t nseg = ceil_div(std::max<int64_t>(dims->seqlen, 1), kSeg);
-    return static_cast<size_t>(dims->batch * nseg * dims->d_inner) * kN * sizeof(float);
+// Backward workspace: local checkpoints [batch][nseg][d][kN], their Σ Δ
+// [batch][nseg][d], then chunk records for up to kBwdMaxChunks chunks:
+// h_loc and g_loc [batch][kmax][d][kN], Σ Δ [batch][kmax][d]; each region
+// 256-byte aligned.
+constexpr int64_t kBwdMaxChunks = 16;
+struct BwdLayout {
+    size_t ckpt, sck, hloc, gloc, send, total;
+    int64_t nseg, kmax;
+};
+BwdLayout bwd_layout(const ss_dims* dims) {
+    BwdLayout w{};
+    const int64_t b = dims->batch, d = dims->d_inner;
+    w.nseg = ceil_div(std::max<int64_t>(dims->seqlen, 1), kSeg);
+    w.kmax = std::min(kBwdMaxChunks, w.nseg);
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    size_t off = 0;
+    w.ckpt = off; off += al(static_cast<size_t>(b * w.nseg * d) * kN * sizeof(float));
+    w.sck = off;  off += al(static_cast<size_t>(b * w.nseg * d) * sizeof(float));
+    w.hloc = off; off += al(static_cast<size_t>(b * w.kmax * d) * kN * sizeof(float));
+    w.gloc = off; off += al(static_cast<size_t>(b * w.kmax * d) * kN * sizeof(float));
+    w.send = off; off += al(static_cast<size_t>(b * w.kmax * d) * sizeof(float));
+    w.total = off;
+    return w;
+}
+size_t bwd_workspace(const ss_dims* dims) { return bwd_layout(dims).total; }
+
+// Time chunks for `items` (batch, channel-block) items of nseg segments on
+// `slots` resident CTAs: the count whose waves x segments per chunk is
+// smallest, charging chunking 10 % for its extra pass (adjoint-only
+// recurrence).  A positive chunk_len fixes the chunk length instead.
+void bwd_chunks(int64_t items, int64_t nseg, int64_t kmax, int64_t slots, int32_t chunk_len, int& nchunk,
+                int& cseg) {
+    if (chunk_len > 0) {
+        int64_t cs = std::max<int64_t>(1, ceil_div(chunk_len, kSeg));
+        if (ceil_div(nseg, cs) > kmax) cs = ceil_div(nseg, kmax);
+        cseg = static_cast<int>(cs);
+        nchunk = static_cast<int>(ceil_div(nseg, cs));
+        return;
+    }
+    double best = 0.0;
+    nchunk = 1;
+    cseg = static_cast<int>(nseg);
+    for (int64_t k = 1; k <= kmax; ++k) {
+        const int64_t cs = ceil_div(nseg, k);
+        if (ceil_div(nseg, cs) != k) continue;
+        const double waves = static_cast<double>(ceil_div(items * k, std::max<int64_t>(slots, 1)));
+        const double cost = waves * static_cast<double>(cs) * (k > 1 ? 1.1 : 1.0);
+        if (k == 1 || cost < best - 1e-9) {
+            best = cost;
+            nchunk = static_cast<int>(k);
+            cseg = static_cast<int>(cs);
+        }
+    }
 }
 
-template <typename IO, bool SP, bool HZ>
-int launch_bwd(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
-    auto kern = ss_bwd_kernel<IO, SP, HZ>;
-    const size_t smem = sizeof(BwdSmem<IO>);
-    static bool attr_set[kMaxDevices] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
+template <typename Kern>
+int set_bwd_smem(Kern kern, size_t smem, bool (&attr_set)[kMaxDevices], int dev) {
     if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
             cudaSuccess)
             return SS_ERR_CUDA;
         if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
     }
-    kern<<<static_cast<unsigned>(ctas), kBwdThreads, smem, stream>>>(p);
+    return SS_OK;
+}
+
+// Plans the chunks (needs the kernels' occupancy) and launches the chunk pass
+// then the gradient pass.
+template <typename IO, bool SP, bool HZ>
+int launch_bwd(BwdParams& p, int64_t items, int64_t kmax, int32_t chunk_len, cudaStream_t stream) {
+    auto kchunk = ss_bwd_chunk_kernel<IO, SP, HZ>;
+    auto kgrad = ss_bwd_kernel<IO, SP, HZ>;
+    const size_t smem = sizeof(BwdSmem<IO>);
+    static bool attr_chunk[kMaxDevices] = {false};
+    static bool attr_grad[kMaxDevices] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
+    const size_t smem_chunk = sizeof(ChunkSmem<IO>);
+    if (set_bwd_smem(kchunk, smem_chunk, attr_chunk, dev) != SS_OK ||
+        set_bwd_smem(kgrad, smem, attr_grad, dev) != SS_OK)
+        return SS_ERR_CUDA;
+    int per_sm = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kgrad, kBwdThreads, smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return SS_ERR_CUDA;
+    bwd_chunks(items, p.nseg, kmax, static_cast<int64_t>(per_sm) * sms, chunk_len, p.nchunk, p.cseg);
+    const int64_t ctas = items * p.nchunk;
+    if (ctas >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    kchunk<<<static_cast<unsigned>(ctas), kBwdThreads, smem_chunk, stream>>>(p);
+    const int64_t states = static_cast<int64_t>(p.batch) * p.d * kN;
+    const int64_t cblocks = std::min<int64_t>(ceil_div(states, 256), int64_t(sms) * 16);
+    ss_bwd_combine_kernel<<<static_cast<unsigned>(cblocks), 256, 0, stream>>>(p);
+    kgrad<<<static_cast<unsigned>(ctas), kBwdThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
 template <typename IO>
-int launch_bwd_flags(const BwdParams& p, int64_t ctas, cudaStream_t stream) {
+int launch_bwd_flags(BwdParams& p, int64_t items, int64_t kmax, int32_t chunk_len, cudaStream_t stream) {
     const bool hz = p.z != nullptr;
-    if (p.softplus) return hz ? launch_bwd<IO, true, true>(p, ctas, stream) : launch_bwd<IO, true, false>(p, ctas, stream);
-    return hz ? launch_bwd<IO, false, true>(p, ctas, stream) : launch_bwd<IO, false, false>(p, ctas, stream);
+    if (p.softplus)
+        return hz ? launch_bwd<IO, true, true>(p, items, kmax, chunk_len, stream)
+                  : launch_bwd<IO, true, false>(p, items, kmax, chunk_len, stream);
+    return hz ? launch_bwd<IO, false, true>(p, items, kmax, chunk_len, stream)
+              : launch_bwd<IO, false, false>(p, items, kmax, chunk_len, stream);
 }
 
 // ------------------------------------------------------------- Mamba block
@@ -560,22 +636,29 @@ int ss_bwd(const void* u, const void* delta, const float* delta_bias, const floa
     // With no tokens, last_state = h_{-1} = 0 depends on nothing: every gradient is zero.
     if (L == 0) return (flags & SS_SYNC_CHECK) ? (cudaStreamSynchronize(stream) == cudaSuccess ? SS_OK : SS_ERR_CUDA)
                                               : SS_OK;
-    const size_t need = bwd_workspace(dims);
-    if (!launch->workspace || launch->workspace_bytes < need || !aligned16(launch->workspace))
+    const BwdLayout w = bwd_layout(dims);
+    if (!launch->workspace || launch->workspace_bytes < w.total || !aligned16(launch->workspace))
         return SS_ERR_WORKSPACE;
     const int64_t nblk = ceil_div(d, kBwdCh);
-    const int64_t ctas = batch * nblk;
-    if (ctas >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    const int64_t items = batch * nblk;
+    if (items >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
 
     BwdParams p{};
     p.u = u; p.delta = delta; p.bias = delta_bias; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
     p.dy = dy; p.dlast = dlast_state;
     p.du = du; p.ddelta = ddelta; p.dz = dz; p.dA = dA; p.dB = dB; p.dC = dC; p.dD = dD; p.dbias = ddelta_bias;
-    p.ckpt = static_cast<float*>(launch->workspace);
+    unsigned char* ws = static_cast<unsigned char*>(launch->workspace);
+    p.ckpt = reinterpret_cast<float*>(ws + w.ckpt);
+    p.sck = reinterpret_cast<float*>(ws + w.sck);
+    p.hloc = reinterpret_cast<float*>(ws + w.hloc);
+    p.gloc = reinterpret_cast<float*>(ws + w.gloc);
+    p.send = reinterpret_cast<float*>(ws + w.send);
     p.L = L; p.batch = static_cast<int>(batch); p.d = static_cast<int>(d);
-    p.nseg = static_cast<int>(ceil_div(L, kSeg)); p.nblk = static_cast<int>(nblk);
+    p.nseg = static_cast<int>(w.nseg); p.nblk = static_cast<int>(nblk);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
-    rc = (flags & SS_BF16) ? launch_bwd_flags<__nv_bfloat16>(p, ctas, stream) : launch_bwd_flags<float>(p, ctas, stream);
+    p.vec = (d * static_cast<int64_t>((flags & SS_BF16) ? 2 : 4)) % 16 == 0 ? 1 : 0;
+    rc = (flags & SS_BF16) ? launch_bwd_flags<__nv_bfloat16>(p, items, w.kmax, launch->chunk_len, stream)
+                           : launch_bwd_flags<float>(p, items, w.kmax, launch->chunk_len, stream);
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;

@@ -114,6 +114,23 @@ def test_workspace_layout(L):
     assert L.ss_fwd_workspace_bytes(ctypes.byref(ss.ss_dims(1, 8, 256, 32)), ss.SS_BF16, 0) == 0
 
 
+def test_bwd_workspace_layout(L):
+    """Checkpoints [b][nseg][d][16] and their Σ Δ [b][nseg][d], then records
+    for min(16, nseg) time chunks (h_loc, g_loc [b][k][d][16], Σ Δ [b][k][d]),
+    each region rounded up to 256 bytes."""
+    al = lambda x: (x + 255) // 256 * 256
+
+    def expect(b, L_, d):
+        nseg = max(1, -(-L_ // 32))
+        k = min(16, nseg)
+        return (al(b * nseg * d * 64) + al(b * nseg * d * 4) + 2 * al(b * k * d * 64) + al(b * k * d * 4))
+
+    for b, L_, d in ((1, 32, 64), (2, 1000, 130), (4, 8192, 5120), (3, 1, 10), (1, 0, 64)):
+        got = L.ss_bwd_workspace_bytes(ctypes.byref(ss.ss_dims(b, L_, d, 16)), ss.SS_BF16)
+        assert got == expect(b, L_, d), (b, L_, d)
+    assert L.ss_bwd_workspace_bytes(ctypes.byref(ss.ss_dims(1, 8, 64, 32)), ss.SS_BF16) == 0
+
+
 def test_auto_chunking_is_a_tile_multiple(L):
     for (b, l, d) in ((4, 8192, 5120), (8, 2048, 1536), (1, 1 << 20, 1536), (1, 64, 32)):
         dims = ss.ss_dims(b, l, d, 16)

@@ -32,9 +32,10 @@ def tols(dtype):
     return 1e-2, 2e-3
 
 
-def run_both(inp, dy, dl, softplus=True):
+def run_both(inp, dy, dl, softplus=True, chunk_len=0):
     got = ss.ss_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"], z=inp["z"],
-                    delta_bias=inp["delta_bias"], dlast_state=dl, softplus=softplus, sync_check=True)
+                    delta_bias=inp["delta_bias"], dlast_state=dl, softplus=softplus, chunk_len=chunk_len,
+                    sync_check=True)
     ref = oracle.bwd(to_f64(inp["u"]), to_f64(inp["delta"]), to_f64(inp["A"]), to_f64(inp["B"]),
                      to_f64(inp["C"]), to_f64(dy), D=to_f64(inp["D"]), z=to_f64(inp["z"]),
                      delta_bias=to_f64(inp["delta_bias"]), dlast=to_f64(dl), softplus=softplus)
@@ -71,6 +72,43 @@ def test_bwd_fp32(shape):
     dy, dl = bwd_upstream(b, L, d, 16, "fp32", 7 + L + d, DEV)
     got, ref = run_both(inp, dy, dl)
     check(got, ref, torch.float32)
+
+
+# Forced time chunks: the chunk length is rounded up to whole 32-step
+# segments, so these give 2 .. 10 chunks with a ragged last chunk and a
+# ragged last segment; the chunks' carried state and adjoint must be exact.
+CHUNKED = [((2, 300, 96), 64), ((1, 333, 64), 32), ((3, 200, 130), 96), ((1, 1000, 64), 100)]
+
+
+@pytest.mark.parametrize("shape,chunk", CHUNKED, ids=[f"b{b}_L{l}_d{d}_c{c}" for (b, l, d), c in CHUNKED])
+def test_bwd_time_chunks_bf16(shape, chunk):
+    b, L, d = shape
+    seed = 900 + L + chunk
+    inp = fwd_inputs(b, L, d, 16, "bf16", seed, DEV, gate=True, D_kind="normal")
+    dy, dl = bwd_upstream(b, L, d, 16, "bf16", seed, DEV)
+    got, ref = run_both(inp, dy, dl, chunk_len=chunk)
+    check(got, ref, torch.bfloat16)
+
+
+def test_bwd_time_chunks_fp32_general_A():
+    inp = fwd_inputs(2, 260, 70, 16, "fp32", 77, DEV, gate=True, D_kind="normal", A_kind="general")
+    dy, dl = bwd_upstream(2, 260, 70, 16, "fp32", 77, DEV)
+    got, ref = run_both(inp, dy, dl, chunk_len=64)
+    check(got, ref, torch.float32)
+
+
+def test_bwd_chunked_matches_unchunked():
+    """Chunking re-associates exact linear recurrences: the chunked and the
+    one-chunk gradients agree to fp32 rounding."""
+    inp = fwd_inputs(2, 640, 128, 16, "bf16", 81, DEV, gate=True, D_kind="normal")
+    dy, dl = bwd_upstream(2, 640, 128, 16, "bf16", 81, DEV)
+    one = ss.ss_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"], z=inp["z"],
+                    delta_bias=inp["delta_bias"], dlast_state=dl, chunk_len=640, sync_check=True)
+    many = ss.ss_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"], z=inp["z"],
+                     delta_bias=inp["delta_bias"], dlast_state=dl, chunk_len=32, sync_check=True)
+    for k in one:
+        e = rel_max_err(to_f64(many[k]), to_f64(one[k]))
+        assert e <= (1e-2 if k in IO_GRADS else 1e-4), f"{k}: {e:.3g}"
 
 
 def test_bwd_general_A_bf16():
@@ -114,7 +152,9 @@ def test_bwd_rejects_bad_arguments():
     dims = ss.ss_dims(1, 32, 64, 16)
     flags = ss.SS_BF16 | ss.SS_DELTA_SOFTPLUS
     need = int(ss.lib().ss_bwd_workspace_bytes(dims, flags))
-    assert need == 1 * 1 * 64 * 16 * 4
+    # one 32-step segment, one chunk: checkpoints 64 x 16 fp32, their Σ Δ (64
+    # floats -> 256 B), h_loc and g_loc records 64 x 16 each, Σ Δ record 256 B
+    assert need == 4096 + 256 + 4096 + 4096 + 256
     g = {k: torch.empty_like(inp["u"]) for k in ("du", "ddelta", "dz")}
     f = {k: torch.empty(s, device=DEV) for k, s in (("dA", (64, 16)), ("dB", (1, 32, 16)), ("dC", (1, 32, 16)))}
     ws = torch.empty(need, dtype=torch.uint8, device=DEV)
