@@ -632,7 +632,8 @@ def run_ours(args):
                                      "ch_ts_per_s": c.ch_ts / (bms * 1e-3),
                                      "ratio_to_fwd": (bms / fwd_ms) if fwd_ms else None,
                                      "note": "ss_bwd (all input gradients), upstream dy and dlast_state "
-                                             "resident; one kernel launch plus the zeroing memsets"}
+                                             "resident; three kernel launches (chunk pass, record fold, gradient pass) "
+                                                     "plus the zeroing memsets"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

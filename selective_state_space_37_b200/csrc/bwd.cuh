@@ -54,6 +54,7 @@
 #include <type_traits>
 
 #include "common.cuh"
+#include "cp_async.cuh"
 #include "fwd.cuh"
 
 namespace selscan {
@@ -269,7 +270,10 @@ __device__ __forceinline__ void adjoint_step(BwdSmem<IO>& S, const BwdParams& p,
                                              float& dD_acc, float& dbias_acc) {
     const int lane = threadIdx.x & 31;
     const int hp = kBH * cp.p;
-    const bool writer = cp.valid && cp.p == 0;   // stores the per-channel outputs
+    // Both threads of a channel hold the same per-channel outputs (their sums
+    // over the two halves commute exactly) and both store them: the same value
+    // to the same address, without a divergent branch.
+    const bool writer = cp.valid;
     const float4 pr = S.pre[r][cp.c];
     const float dt = pr.x, sig = pr.w;
     const float uv = to_f32(S.tu[r][cp.c]);

@@ -21,6 +21,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "cp_async.cuh"
 
 namespace selscan {
 
