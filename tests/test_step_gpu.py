@@ -35,6 +35,33 @@ def test_step_small(dtype, shape, A_kind):
         assert rel_max_err(to_f64(inp["state"]), sr) <= tol
 
 
+# Options and shapes of the bf16 step: one batch row, many rows, a few
+# channels, d_inner not a multiple of the 64-channel block, gate / softplus /
+# D / bias on and off.
+OPTS = [(1, 8, True, True, True), (37, 4096, True, True, True), (300, 24, False, True, False), (512, 4096, True, True, True),
+        (4, 136, True, False, True), (2, 2048, False, False, False)]
+
+
+@pytest.mark.parametrize("b,d,gate,softplus,opts", OPTS,
+                         ids=[f"b{b}_d{d}_g{int(g)}_sp{int(s)}_o{int(o)}" for b, d, g, s, o in OPTS])
+def test_step_options(b, d, gate, softplus, opts):
+    inp = step_inputs(b, d, 16, "bf16", 70 + b + d, DEV, gate=gate, bias=opts)
+    if not opts:
+        inp["D"] = None
+    if not softplus:   # Δ is used as given: keep it positive (and without the negative bias)
+        inp["delta"] = (inp["delta"].float().abs() * 0.1 + 0.01).to(torch.bfloat16)
+        inp["delta_bias"] = None
+    st0 = to_f64(inp["state"])
+    y = ss.ss_step(inp["state"], inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], D=inp["D"],
+                   z=inp["z"], delta_bias=inp["delta_bias"], softplus=softplus, sync_check=True)
+    sr, yr = oracle.step(st0, to_f64(inp["u"]), to_f64(inp["delta"]), to_f64(inp["A"]), to_f64(inp["B"]),
+                         to_f64(inp["C"]), D=to_f64(inp["D"]), z=to_f64(inp["z"]),
+                         delta_bias=to_f64(inp["delta_bias"]), softplus=softplus, precision="f32")
+    tol = tol_for(inp["u"].dtype)
+    assert rel_max_err(to_f64(y), yr) <= tol
+    assert rel_max_err(to_f64(inp["state"]), sr) <= tol
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "fp32"])
 def test_step_loop_equals_scan(dtype):
     """L decode steps from a zero state reproduce ss_fwd (y at every step and
