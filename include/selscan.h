@@ -23,6 +23,8 @@
  *            (projections on cuBLAS, conv, scan, gate, output projection).
  *   ss_ssd_fwd  the multi-head scan with a scalar decay per head (Mamba-2's
  *            SSD model) on the tensor cores.
+ *   ss_fwd_host  ss_fwd on activations in host memory, with uploads, scans
+ *            and downloads of batch slices overlapped.
  *   ss_bwd   the gradients of ss_fwd's inputs from the gradient of its outputs
  *            (the models are trained and fine-tuned with gradient
  *            checkpointing: "Mamba 7.9.1" article §5.3-5.4; model-architecture
@@ -287,6 +289,32 @@ SS_API int ss_bwd(const void* u, const void* delta, const float* delta_bias, con
                   const void* C, const float* D, const void* z, const void* dy, const float* dlast_state,
                   void* du, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
                   float* ddelta_bias, uint32_t flags, const ss_dims* dims, const ss_launch* launch);
+
+/* ss_fwd_host -- ss_fwd on activations in HOST memory (an engineering
+ * addition: the pages have no counterpart).  u, delta, z, B, C (inputs) and
+ * y, last_state (outputs) are host pointers, same layouts and element types
+ * as ss_fwd; page-locked (pinned) memory lets the copies run asynchronously,
+ * pageable memory works but copies synchronously.  A, D and delta_bias are
+ * DEVICE pointers (parameters stay resident).  The batch is cut into slices
+ * of rows_per_slice rows (0 or less: 1); slice s is uploaded on a copy
+ * stream, scanned on launch->stream and downloaded on a second copy stream,
+ * through two device staging slots, so uploads, scans and downloads of
+ * neighbouring slices overlap.  The results equal ss_fwd applied to each
+ * slice.  launch->workspace is the staging: at least
+ * ss_fwd_host_workspace_bytes(dims, flags, rows_per_slice) bytes, 16-byte
+ * aligned, else SS_ERR_WORKSPACE; it must stay untouched until the call's
+ * work on launch->stream completes.  The copy streams and their events are
+ * created on the first call of each host thread on each device and kept.
+ * The call is asynchronous on launch->stream: y and last_state are complete
+ * once launch->stream has been synchronized (SS_SYNC_CHECK does it and
+ * returns the device status).  Errors: as ss_fwd. */
+SS_API int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+                       const void* C, const float* D, const void* z, void* y, float* last_state, uint32_t flags,
+                       const ss_dims* dims, const ss_launch* launch, int32_t rows_per_slice);
+
+/* Staging bytes ss_fwd_host needs (two slices' activations and states plus
+ * one slice's ss_fwd workspace); 0 for sizes it would reject. */
+SS_API size_t ss_fwd_host_workspace_bytes(const ss_dims* dims, uint32_t flags, int32_t rows_per_slice);
 
 /* Workspace bytes ss_bwd needs for these sizes (0 for invalid dims). */
 SS_API size_t ss_bwd_workspace_bytes(const ss_dims* dims, uint32_t flags);

@@ -34,7 +34,8 @@ D_STATE = 16
 # Every symbol include/selscan.h declares.
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
             "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
-            "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_block_scratch_bytes", "ss_ssd_fwd")
+            "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_block_scratch_bytes", "ss_ssd_fwd",
+            "ss_fwd_host", "ss_fwd_host_workspace_bytes")
 
 
 class ss_dims(ctypes.Structure):
@@ -102,6 +103,11 @@ def lib():
         L.ss_step.restype = ctypes.c_int
         L.ss_fwd_workspace_bytes.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32, ctypes.c_int32]
         L.ss_fwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ss_fwd_host.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, vp, f32p, ctypes.c_uint32,
+                                  ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch), ctypes.c_int32]
+        L.ss_fwd_host.restype = ctypes.c_int
+        L.ss_fwd_host_workspace_bytes.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32, ctypes.c_int32]
+        L.ss_fwd_host_workspace_bytes.restype = ctypes.c_size_t
         L.ss_fwd_chunk_len.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32]
         L.ss_fwd_chunk_len.restype = ctypes.c_int32
         L.ss_check.argtypes = [ctypes.POINTER(ss_launch)]
@@ -245,6 +251,60 @@ def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, y=None, last_s
     if rc != SS_OK:
         raise SelscanError(rc, "ss_fwd")
     return y, last_state
+
+
+def ss_fwd_host(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, y=None, last_state=None,
+                return_last_state=True, softplus=True, rows_per_slice=1, workspace=None, stream=None,
+                sync_check=False):
+    """ss_fwd on activations in host memory through libselscan's ss_fwd_host.
+
+    u, delta, z, B, C (and y, last_state if given) are CPU tensors -- pinned
+    for overlapped copies -- with ss_fwd's shapes; A, D, delta_bias are CUDA
+    tensors on the device that runs the scan.  Batch slices of rows_per_slice
+    rows are uploaded, scanned and downloaded with the three overlapped.
+    Returns (y, last_state) as CPU tensors, complete once the stream is
+    synchronized (sync_check=True does it).
+    """
+    if u.dim() != 3:
+        raise ValueError("u must be [batch, L, d_inner]")
+    batch, L, d = u.shape
+    host = torch.device("cpu")
+    dev = A.device
+    if dev.type != "cuda":
+        raise ValueError("A, D and delta_bias must be CUDA tensors")
+    io = u.dtype
+    for t, nm, shp in ((u, "u", (batch, L, d)), (delta, "delta", (batch, L, d)),
+                       (z, "z", (batch, L, d)), (B, "B", (batch, L, D_STATE)),
+                       (C, "C", (batch, L, D_STATE))):
+        _check(t, nm, shp, io, host)
+    _check(A, "A", (d, D_STATE), torch.float32, dev)
+    _check(D, "D", (d,), torch.float32, dev)
+    _check(delta_bias, "delta_bias", (d,), torch.float32, dev)
+    pin = u.is_pinned()
+    if y is None:
+        y = torch.empty((batch, L, d), dtype=io, pin_memory=pin)
+    _check(y, "y", (batch, L, d), io, host)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, d, D_STATE), dtype=torch.float32, pin_memory=pin)
+    _check(last_state, "last_state", (batch, d, D_STATE), torch.float32, host)
+    flags = _io_flag(u) | (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
+    sh = _stream_handle(stream, dev)
+    dims = ss_dims(batch, L, d, D_STATE)
+    need = int(lib().ss_fwd_host_workspace_bytes(ctypes.byref(dims), flags, int(rows_per_slice)))
+    if workspace is None:
+        workspace = workspace_for(need, dev, sh)
+    launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(), 0, 0)
+    rc = lib().ss_fwd_host(_ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                           _ptr(z), _ptr(y), _ptr(last_state), flags, ctypes.byref(dims),
+                           ctypes.byref(launch), int(rows_per_slice))
+    if rc != SS_OK:
+        raise SelscanError(rc, "ss_fwd_host")
+    return y, last_state
+
+
+def fwd_host_workspace_bytes(batch, seqlen, d_inner, bf16=True, rows_per_slice=1, d_state=D_STATE):
+    dims = ss_dims(batch, seqlen, d_inner, d_state)
+    return int(lib().ss_fwd_host_workspace_bytes(ctypes.byref(dims), SS_BF16 if bf16 else 0, int(rows_per_slice)))
 
 
 def bwd_workspace_bytes(batch, seqlen, d_inner, bf16=True, d_state=D_STATE):

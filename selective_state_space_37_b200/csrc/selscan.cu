@@ -523,6 +523,152 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
     return fwd_impl(u, delta, delta_bias, A, B, C, D, z, y, last_state, nullptr, nullptr, flags, dims, launch);
 }
 
+// ------------------------------------------------------------- host-buffer forward
+// Staging of ss_fwd_host: two slots, each holding one batch slice's u, Δraw,
+// z, y [rows, L, d], B, C [rows, L, 16] and last_state [rows, d, 16], then
+// the forward workspace for one slice; every region 256-byte aligned.
+struct HostPlan {
+    size_t act, bc, st, slot, ws_off, ws, total;
+    int64_t rows;
+};
+static HostPlan host_plan(const ss_dims* dims, uint32_t flags, int32_t rows_per_slice) {
+    HostPlan h{};
+    const size_t es = (flags & SS_BF16) ? 2 : 4;
+    const int64_t L = dims->seqlen, d = dims->d_inner;
+    h.rows = std::max<int64_t>(1, std::min<int64_t>(rows_per_slice > 0 ? rows_per_slice : 1, dims->batch));
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    h.act = al(static_cast<size_t>(h.rows * L * d) * es);
+    h.bc = al(static_cast<size_t>(h.rows * L * kN) * es);
+    h.st = al(static_cast<size_t>(h.rows * d * kN) * sizeof(float));
+    h.slot = 4 * h.act + 2 * h.bc + h.st;
+    ss_dims sd = *dims;
+    sd.batch = h.rows;
+    h.ws_off = 2 * h.slot;
+    h.ws = al(ss_fwd_workspace_bytes(&sd, flags, 0));
+    h.total = h.ws_off + h.ws;
+    return h;
+}
+
+// Copy streams and events of the host pipeline, one set per (host thread,
+// device), created on first use and kept (like the cuBLAS handle).
+struct HostPipe {
+    cudaStream_t up = nullptr, down = nullptr;
+    cudaEvent_t start = nullptr, end = nullptr, in_ready[2] = {}, done[2] = {}, out_free[2] = {};
+    bool ok = false;
+};
+static HostPipe* host_pipe() {
+    thread_local HostPipe pipes[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    HostPipe& h = pipes[dev];
+    if (!h.ok) {
+        bool ok = cudaStreamCreateWithFlags(&h.up, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&h.down, cudaStreamNonBlocking) == cudaSuccess;
+        cudaEvent_t* evs[] = {&h.start, &h.end, &h.in_ready[0], &h.in_ready[1], &h.done[0], &h.done[1],
+                              &h.out_free[0], &h.out_free[1]};
+        for (cudaEvent_t* e : evs) ok = ok && cudaEventCreateWithFlags(e, cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) return nullptr;
+        h.ok = true;
+    }
+    return &h;
+}
+
+size_t ss_fwd_host_workspace_bytes(const ss_dims* dims, uint32_t flags, int32_t rows_per_slice) {
+    if (validate_dims(dims, true) != SS_OK || (flags & ~kKnownFlags) || dims->batch == 0 || dims->d_inner == 0)
+        return 0;
+    return host_plan(dims, flags, rows_per_slice).total;
+}
+
+int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+                const void* C, const float* D, const void* z, void* y, float* last_state, uint32_t flags,
+                const ss_dims* dims, const ss_launch* launch, int32_t rows_per_slice) {
+    int rc = validate_dims(dims, true);
+    if (rc != SS_OK) return rc;
+    if (!launch || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
+    const int64_t batch = dims->batch, L = dims->seqlen, d = dims->d_inner;
+    if (batch == 0 || d == 0) return SS_OK;
+    if (!A || (L > 0 && (!u || !delta || !B || !C || !y))) return SS_ERR_INVALID_ARG;
+    const void* dev_ptrs[] = {A, D, delta_bias};
+    for (const void* q : dev_ptrs)
+        if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
+    const HostPlan h = host_plan(dims, flags, rows_per_slice);
+    if (!launch->workspace || launch->workspace_bytes < h.total || !aligned16(launch->workspace))
+        return SS_ERR_WORKSPACE;
+    cudaStream_t cs = static_cast<cudaStream_t>(launch->stream);
+    if (L == 0) {   // last_state = h_{-1} = 0, nothing else to do
+        if (last_state) {
+            if (cudaStreamSynchronize(cs) != cudaSuccess) return SS_ERR_CUDA;
+            std::memset(last_state, 0, static_cast<size_t>(batch * d * kN) * sizeof(float));
+        }
+        return SS_OK;
+    }
+    HostPipe* hp = host_pipe();
+    if (!hp) return SS_ERR_CUDA;
+    const size_t es = (flags & SS_BF16) ? 2 : 4;
+    unsigned char* base = static_cast<unsigned char*>(launch->workspace);
+    ss_launch sl = *launch;   // the slices' forward: workspace after the two slots
+    sl.workspace = base + h.ws_off;
+    sl.workspace_bytes = h.ws;
+    const uint32_t fflags = flags & ~static_cast<uint32_t>(SS_SYNC_CHECK);
+    auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    // the copy streams start after the work already queued on the caller's stream
+    if (!ok(cudaEventRecord(hp->start, cs)) || !ok(cudaStreamWaitEvent(hp->up, hp->start, 0)) ||
+        !ok(cudaStreamWaitEvent(hp->down, hp->start, 0)))
+        return SS_ERR_CUDA;
+    const int64_t nslices = ceil_div(batch, h.rows);
+    for (int64_t s = 0; s < nslices; ++s) {
+        const int slot = static_cast<int>(s & 1);
+        const int64_t r0 = s * h.rows, nr = std::min(h.rows, batch - r0);
+        unsigned char* sp = base + slot * h.slot;
+        void* su = sp;
+        void* sd = sp + h.act;
+        void* sz = sp + 2 * h.act;
+        void* sy = sp + 3 * h.act;
+        void* sB = sp + 4 * h.act;
+        void* sC = sp + 4 * h.act + h.bc;
+        float* sst = reinterpret_cast<float*>(sp + 4 * h.act + 2 * h.bc);
+        const size_t act_bytes = static_cast<size_t>(nr * L * d) * es, act_off = static_cast<size_t>(r0 * L * d) * es;
+        const size_t bc_bytes = static_cast<size_t>(nr * L * kN) * es, bc_off = static_cast<size_t>(r0 * L * kN) * es;
+        // upload (after the forward of slice s - 2 has read this slot)
+        if (s >= 2 && !ok(cudaStreamWaitEvent(hp->up, hp->done[slot], 0))) return SS_ERR_CUDA;
+        if (!ok(cudaMemcpyAsync(su, static_cast<const unsigned char*>(u) + act_off, act_bytes, cudaMemcpyHostToDevice,
+                                hp->up)) ||
+            !ok(cudaMemcpyAsync(sd, static_cast<const unsigned char*>(delta) + act_off, act_bytes,
+                                cudaMemcpyHostToDevice, hp->up)) ||
+            (z && !ok(cudaMemcpyAsync(sz, static_cast<const unsigned char*>(z) + act_off, act_bytes,
+                                      cudaMemcpyHostToDevice, hp->up))) ||
+            !ok(cudaMemcpyAsync(sB, static_cast<const unsigned char*>(B) + bc_off, bc_bytes, cudaMemcpyHostToDevice,
+                                hp->up)) ||
+            !ok(cudaMemcpyAsync(sC, static_cast<const unsigned char*>(C) + bc_off, bc_bytes, cudaMemcpyHostToDevice,
+                                hp->up)) ||
+            !ok(cudaEventRecord(hp->in_ready[slot], hp->up)))
+            return SS_ERR_CUDA;
+        // forward of the slice (after its upload, and after slice s - 2's y left this slot)
+        if (!ok(cudaStreamWaitEvent(cs, hp->in_ready[slot], 0)) ||
+            (s >= 2 && !ok(cudaStreamWaitEvent(cs, hp->out_free[slot], 0))))
+            return SS_ERR_CUDA;
+        ss_dims sdims = *dims;
+        sdims.batch = nr;
+        rc = fwd_impl(su, sd, delta_bias, A, sB, sC, D, z ? sz : nullptr, sy, last_state ? sst : nullptr, nullptr,
+                      nullptr, fflags, &sdims, &sl);
+        if (rc != SS_OK) return rc;
+        if (!ok(cudaEventRecord(hp->done[slot], cs))) return SS_ERR_CUDA;
+        // download
+        if (!ok(cudaStreamWaitEvent(hp->down, hp->done[slot], 0)) ||
+            !ok(cudaMemcpyAsync(static_cast<unsigned char*>(y) + act_off, sy, act_bytes, cudaMemcpyDeviceToHost,
+                                hp->down)) ||
+            (last_state && !ok(cudaMemcpyAsync(last_state + r0 * d * kN, sst,
+                                               static_cast<size_t>(nr * d * kN) * sizeof(float),
+                                               cudaMemcpyDeviceToHost, hp->down))) ||
+            !ok(cudaEventRecord(hp->out_free[slot], hp->down)))
+            return SS_ERR_CUDA;
+    }
+    // the caller's stream continues after the last download
+    if (!ok(cudaEventRecord(hp->end, hp->down)) || !ok(cudaStreamWaitEvent(cs, hp->end, 0))) return SS_ERR_CUDA;
+    if (flags & SS_SYNC_CHECK) return ss_check(&sl);
+    return SS_OK;
+}
+
 int ss_fwd_conv(const void* x, const float* conv_w, const float* conv_b, const void* delta, const float* delta_bias,
                 const float* A, const void* B, const void* C, const float* D, const void* z, void* y,
                 float* last_state, float* conv_state, uint32_t flags, const ss_dims* dims, const ss_launch* launch) {
