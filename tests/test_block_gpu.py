@@ -40,3 +40,20 @@ def test_block_rejects_bad_sizes():
     st = ss._binding._block_struct(w, DEV)
     st.d_inner = 100                                                          # not a multiple of 8
     assert int(ss.lib().ss_block_scratch_bytes(st, 1, 16)) == 0
+
+
+def test_block_full_size_prefix():
+    """The Mamba-2.8B-shaped block (batch 4, L 8192, d_model 2560) on the whole
+    input, as the bench times it; the block is causal, so the oracle on the
+    first 256 tokens of two batch rows gives those rows' exact outputs."""
+    b, L, dm = 4, 8192, 2560
+    hidden, w = block_inputs(b, L, dm, seed=9, device=DEV)
+    out = ss.ss_block_fwd(hidden, w)
+    torch.cuda.synchronize()
+    wn = np_weights(w)
+    T = 256
+    for bi in (0, 3):
+        ref = block_fwd(to_f64(hidden[bi:bi + 1, :T]), wn, store_bf16=True)
+        assert rel_max_err(to_f64(out[bi:bi + 1, :T]), ref) <= 2e-2, bi
+    del hidden, w, out
+    torch.cuda.empty_cache()

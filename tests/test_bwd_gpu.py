@@ -185,3 +185,36 @@ def test_bwd_config_mamba130m_full():
     check(got, ref, torch.bfloat16)
     del inp, dy, dl, got
     torch.cuda.empty_cache()
+
+
+def test_bwd_config_mamba2p8b_sampled():
+    """The 2.8B-shaped layer (batch 4, L 8192, d_inner 5120) in the bench's
+    launch configuration (4 time chunks).  du, dΔraw, dz, dB and dC of batch
+    entry 0 against the oracle run on that entry (all channels, full L; dB and
+    dC sum over its channels); dA, dD and dbias (sums over batch and time) on
+    48 sampled channels against the oracle run on those channels of every
+    entry."""
+    c = CONFIGS["mamba2p8b"]
+    inp = fwd_inputs(c.batch, c.seqlen, c.d_inner, c.d_state, c.dtype, c.seed, DEV, gate=c.gate,
+                     D_kind=c.D_kind)
+    dy, dl = bwd_upstream(c.batch, c.seqlen, c.d_inner, c.d_state, c.dtype, c.seed, DEV)
+    got = ss.ss_bwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], dy, D=inp["D"], z=inp["z"],
+                    delta_bias=inp["delta_bias"], dlast_state=dl, sync_check=True)
+    tol_io, tol_acc = tols(torch.bfloat16)
+    one = slice(0, 1)
+    ref = oracle.bwd(to_f64(inp["u"][one]), to_f64(inp["delta"][one]), to_f64(inp["A"]), to_f64(inp["B"][one]),
+                     to_f64(inp["C"][one]), to_f64(dy[one]), D=to_f64(inp["D"]), z=to_f64(inp["z"][one]),
+                     delta_bias=to_f64(inp["delta_bias"]), dlast=to_f64(dl[one]))
+    for k in ("du", "ddelta", "dz", "dB", "dC"):
+        e = rel_max_err(to_f64(got[k][one]), ref[k])
+        assert e <= (tol_io if k in IO_GRADS else tol_acc), f"{k}: {e:.3g}"
+    chs = torch.from_numpy(np.sort(np.random.default_rng(11).choice(c.d_inner, size=48, replace=False))).to(DEV)
+    pick = lambda t: t.index_select(-1, chs)
+    ref = oracle.bwd(to_f64(pick(inp["u"])), to_f64(pick(inp["delta"])), to_f64(inp["A"][chs]), to_f64(inp["B"]),
+                     to_f64(inp["C"]), to_f64(pick(dy)), D=to_f64(inp["D"][chs]), z=to_f64(pick(inp["z"])),
+                     delta_bias=to_f64(inp["delta_bias"][chs]), dlast=to_f64(dl[:, chs]))
+    for k, rk in (("dA", "dA"), ("dD", "dD"), ("ddelta_bias", "dbias")):
+        e = rel_max_err(to_f64(got[k][chs]), ref[rk])
+        assert e <= tol_acc, f"{k}: {e:.3g}"
+    del inp, dy, dl, got
+    torch.cuda.empty_cache()

@@ -54,3 +54,24 @@ def test_ssd_zero_length_and_bad_sizes():
     dims = ss.ss_ssd_dims(1, 8, 2, 32, 64)        # headdim 32: unsupported
     rc = ss.lib().ss_ssd_fwd(None, None, None, inp["A"].data_ptr(), None, None, None, None, None, 0, dims, None)
     assert rc == ss.SS_ERR_UNSUPPORTED
+
+
+def test_ssd_full_size_sampled_heads():
+    """The Mamba-2-2.7B-shaped layer (batch 4, L 8192, 80 heads, d_state 128)
+    in the bench's launch configuration; the oracle recomputes a sample of
+    (batch, head) pairs alone (heads are independent), every step and every
+    channel of each."""
+    b, L, H, N = 4, 8192, 80, 128
+    inp = ssd_inputs(b, L, H, N, seed=3, device=DEV)
+    y, st = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
+                          sync_check=True)
+    rng = np.random.default_rng(5)
+    picks = [(int(rng.integers(b)), int(h)) for h in rng.choice(H, size=6, replace=False)]
+    for bi, h in picks:
+        yr, sr = oracle.ssd(to_f64(inp["x"][bi:bi + 1, :, h:h + 1]), to_f64(inp["dt"][bi:bi + 1, :, h:h + 1]),
+                            to_f64(inp["A"][h:h + 1]), to_f64(inp["B"][bi:bi + 1]), to_f64(inp["C"][bi:bi + 1]),
+                            D=to_f64(inp["D"][h:h + 1]), dt_bias=to_f64(inp["dt_bias"][h:h + 1]))
+        assert rel_max_err(to_f64(y[bi:bi + 1, :, h:h + 1]), yr) <= TOL, (bi, h)
+        assert rel_max_err(to_f64(st[bi:bi + 1, h:h + 1]), sr) <= TOL, (bi, h)
+    del inp, y, st
+    torch.cuda.empty_cache()
