@@ -263,9 +263,11 @@ __device__ __forceinline__ void load_state(const float4 (&src)[kNP4][kBwdCh], co
 // One adjoint step (row r of the segment): given h_t (hc) and h_{t-1}
 // (hprev), advances g from ∂J/∂h_t to ∂J/∂h_{t-1} and emits every gradient
 // of step t.
+// i is the step's (b, t, channel) element index; dst its dB or dC entry for
+// this lane's value of the transpose.
 template <typename IO, bool FAST, bool STRUCT, bool HZ>
 __device__ __forceinline__ void adjoint_step(BwdSmem<IO>& S, const BwdParams& p, const BwdChan& cp, int r,
-                                             int64_t row, int64_t ch, const float (&hc)[kBH],
+                                             int64_t i, float* dst, const float (&hc)[kBH],
                                              const float (&hprev)[kBH], float (&g)[kBH], float (&dA_acc)[kBH],
                                              float& dD_acc, float& dbias_acc) {
     const int lane = threadIdx.x & 31;
@@ -285,7 +287,6 @@ __device__ __forceinline__ void adjoint_step(BwdSmem<IO>& S, const BwdParams& p,
     const float4 b0 = Bq[0], b1 = Bq[1], c0 = Cq[0], c1 = Cq[1];
     const float Bh[kBH] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
     const float Ch[kBH] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    const int64_t i = row * p.d + ch;
 
     // s_t = Σ_n C h_t + D u (both halves), then the gate
     f32x2 acc = mul2(pk2(Ch[0], Ch[1]), pk2(hc[0], hc[1]));
@@ -346,7 +347,6 @@ __device__ __forceinline__ void adjoint_step(BwdSmem<IO>& S, const BwdParams& p,
     const f32x2 s01 = add2(add2(pk2(v0.x, v0.y), pk2(v0.z, v0.w)), add2(pk2(v1.x, v1.y), pk2(v1.z, v1.w)));
     const f32x2 s23 = add2(add2(pk2(v2.x, v2.y), pk2(v2.z, v2.w)), add2(pk2(v3.x, v3.y), pk2(v3.z, v3.w)));
     const f32x2 sum = add2(s01, s23);
-    float* dst = (j16 < kBH ? p.dB : p.dC) + row * kN + kBH * (lane >> 4) + (j16 & (kBH - 1));
     atomicAdd(dst, sum.x + sum.y);
 }
 
@@ -597,6 +597,11 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
         for (int s = nsub - 1; s >= 0; --s) {
             const int ns = min(kSub, nt - s * kSub);   // uniform over the CTA
             float hs[kSub][kBH];                        // h_t of the sub-segment's steps, in registers
+            // element index and dB / dC entry of the sub-segment's first step
+            const int64_t rs = row0 + t0 + s * kSub;
+            const int64_t ib = rs * d + ch;
+            float* dstb = ((threadIdx.x & 15) < kBH ? p.dB : p.dC) + rs * kN + kBH * ((threadIdx.x >> 4) & 1) +
+                          (threadIdx.x & (kBH - 1));
             load_state(S.hsub[s], cp, h);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
@@ -614,8 +619,8 @@ __device__ __forceinline__ void bwd_item(BwdSmem<IO>& S, const BwdParams& p, con
                 } else {
                     load_state(S.hsub[s], cp, hprev);
                 }
-                adjoint_step<IO, FAST, STRUCT, HZ>(S, p, cp, s * kSub + j, row0 + t0 + s * kSub + j, ch, hs[j],
-                                                   hprev, g, dA_acc, dD_acc, dbias_acc);
+                adjoint_step<IO, FAST, STRUCT, HZ>(S, p, cp, s * kSub + j, ib + static_cast<int64_t>(j) * p.d,
+                                                   dstb + j * kN, hs[j], hprev, g, dA_acc, dD_acc, dbias_acc);
             }
         }
     }

@@ -256,9 +256,10 @@ BwdLayout bwd_layout(const ss_dims* dims) {
 size_t bwd_workspace(const ss_dims* dims) { return bwd_layout(dims).total; }
 
 // Time chunks for `items` (batch, channel-block) items of nseg segments on
-// `slots` resident CTAs: the count whose waves x segments per chunk is
-// smallest, charging chunking 10 % for its extra pass (adjoint-only
-// recurrence).  A positive chunk_len fixes the chunk length instead.
+// `slots` resident CTAs: the count whose waves x (segments per chunk + a
+// fixed cost of two segments per item: staging, records) is smallest,
+// charging chunking 10 % for its extra pass (adjoint-only recurrence).  A
+// positive chunk_len fixes the chunk length instead.
 void bwd_chunks(int64_t items, int64_t nseg, int64_t kmax, int64_t slots, int32_t chunk_len, int& nchunk,
                 int& cseg) {
     if (chunk_len > 0) {
@@ -275,7 +276,7 @@ void bwd_chunks(int64_t items, int64_t nseg, int64_t kmax, int64_t slots, int32_
         const int64_t cs = ceil_div(nseg, k);
         if (ceil_div(nseg, cs) != k) continue;
         const double waves = static_cast<double>(ceil_div(items * k, std::max<int64_t>(slots, 1)));
-        const double cost = waves * static_cast<double>(cs) * (k > 1 ? 1.1 : 1.0);
+        const double cost = waves * static_cast<double>(cs + 2) * (k > 1 ? 1.1 : 1.0);
         if (k == 1 || cost < best - 1e-9) {
             best = cost;
             nchunk = static_cast<int>(k);
