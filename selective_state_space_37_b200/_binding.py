@@ -35,7 +35,7 @@ D_STATE = 16
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
             "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
             "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_block_scratch_bytes", "ss_ssd_fwd",
-            "ss_fwd_host", "ss_fwd_host_workspace_bytes")
+            "ss_fwd_host", "ss_fwd_host_workspace_bytes", "ss_ssd_fwd_workspace_bytes")
 
 
 class ss_dims(ctypes.Structure):
@@ -137,8 +137,10 @@ def lib():
         L.ss_block_scratch_bytes.argtypes = [ctypes.POINTER(ss_block_weights), ctypes.c_int64, ctypes.c_int64]
         L.ss_block_scratch_bytes.restype = ctypes.c_size_t
         L.ss_ssd_fwd.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, f32p, ctypes.c_uint32,
-                                 ctypes.POINTER(ss_ssd_dims), vp]
+                                 ctypes.POINTER(ss_ssd_dims), ctypes.POINTER(ss_launch)]
         L.ss_ssd_fwd.restype = ctypes.c_int
+        L.ss_ssd_fwd_workspace_bytes.argtypes = [ctypes.POINTER(ss_ssd_dims), ctypes.c_uint32]
+        L.ss_ssd_fwd_workspace_bytes.restype = ctypes.c_size_t
         _lib = L
     return _lib
 
@@ -490,12 +492,13 @@ def ss_block_fwd(hidden, weights, *, out=None, scratch=None, stream=None):
 
 
 def ss_ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, *, softplus=True, y=None, final_state=None,
-               return_final_state=True, stream=None, sync_check=False):
+               return_final_state=True, chunk_len=0, split=True, workspace=None, stream=None, sync_check=False):
     """Multi-head scan with a scalar decay per head (Mamba-2's SSD model).
     x [batch, L, nheads, 64] bf16; dt [batch, L, nheads] bf16; A [nheads] fp32;
     B, C [batch, L, d_state] bf16 (d_state 64 or 128); D, dt_bias [nheads] fp32
     or None.  Returns (y [batch, L, nheads, 64] bf16, final_state
-    [batch, nheads, 64, d_state] fp32 or None)."""
+    [batch, nheads, 64, d_state] fp32 or None).  split=False runs every
+    sequence whole (no workspace); chunk_len > 0 fixes the segment length."""
     batch, L, H, P = x.shape
     N = B.shape[-1]
     dev = x.device
@@ -515,8 +518,16 @@ def ss_ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, *, softplus=True, y=None, f
     _check(final_state, "final_state", (batch, H, P, N), torch.float32, dev)
     flags = (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
     dims = ss_ssd_dims(batch, L, H, P, N)
+    sh = _stream_handle(stream, dev)
+    if split:
+        if workspace is None:
+            workspace = workspace_for(int(lib().ss_ssd_fwd_workspace_bytes(ctypes.byref(dims), flags)), dev, sh)
+        launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(), 0,
+                           int(chunk_len))
+    else:
+        launch = ss_launch(sh, None, 0, 0, int(chunk_len))
     rc = lib().ss_ssd_fwd(_ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
-                          _ptr(final_state), flags, ctypes.byref(dims), _stream_handle(stream, dev))
+                          _ptr(final_state), flags, ctypes.byref(dims), ctypes.byref(launch))
     if rc != SS_OK:
         raise SelscanError(rc, "ss_ssd_fwd")
     return y, final_state

@@ -196,20 +196,98 @@ int launch_variant(bool bf16, bool tma, Variant v, const FwdParams& p, int64_t i
                : launch_fwd<float, false, 1, 1, 8, false, CONV>(p, items, maps, stream);
 }
 
-template <int N>
-int launch_ssd(const SsdParams& p, int64_t ctas, cudaStream_t stream) {
-    auto kern = ss_ssd_kernel<N>;
-    const size_t smem = sizeof(SsdSmem<N>);
-    static bool attr_set[kMaxDevices] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
+// SSD time segments: workspace for up to kSsdMaxSeg segments per sequence --
+// the segment end-state records [batch, H, kmax - 1, P, N] fp32, then Σ Δ A
+// per segment [batch, H, kmax]; each region 256-byte aligned.
+constexpr int64_t kSsdMaxSeg = 8;
+struct SsdLayout {
+    size_t rec, esum, total;
+    int64_t nchunks, kmax;
+};
+SsdLayout ssd_layout(const ss_ssd_dims* d) {
+    SsdLayout w{};
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    w.nchunks = ceil_div(std::max<int64_t>(d->seqlen, 1), kSsdQ);
+    w.kmax = std::min(kSsdMaxSeg, w.nchunks);
+    const int64_t bh = d->batch * d->nheads;
+    w.rec = 0;
+    w.esum = al(static_cast<size_t>(bh * (w.kmax - 1) * kSsdP * d->d_state) * sizeof(float));
+    w.total = w.esum + al(static_cast<size_t>(bh * w.kmax) * sizeof(float));
+    return w;
+}
+
+// Segments for `items` (batch x heads) sequences of nchunks chunks on `slots`
+// resident CTAs: the count with the smallest waves x chunks per segment, the
+// state pass (about 0.3 of the main pass's work per chunk) added, and
+// splitting charged 10 %.  chunk_len > 0 fixes the segment length instead.
+void ssd_segments(int64_t items, int64_t nchunks, int64_t kmax, int64_t slots, int32_t chunk_len, int& nseg,
+                  int& cseg) {
+    slots = std::max<int64_t>(slots, 1);
+    if (chunk_len > 0) {
+        int64_t cs = std::max<int64_t>(1, ceil_div(chunk_len, kSsdQ));
+        if (ceil_div(nchunks, cs) > kmax) cs = ceil_div(nchunks, kmax);
+        cseg = static_cast<int>(cs);
+        nseg = static_cast<int>(ceil_div(nchunks, cs));
+        return;
+    }
+    double best = 0.0;
+    nseg = 1;
+    cseg = static_cast<int>(nchunks);
+    for (int64_t k = 1; k <= kmax; ++k) {
+        const int64_t cs = ceil_div(nchunks, k);
+        if (ceil_div(nchunks, cs) != k) continue;
+        double cost = static_cast<double>(ceil_div(items * k, slots) * cs);
+        if (k > 1) cost = 1.1 * (cost + 0.3 * static_cast<double>(ceil_div(items * (k - 1), slots) * cs));
+        if (k == 1 || cost < best - 1e-9) {
+            best = cost;
+            nseg = static_cast<int>(k);
+            cseg = static_cast<int>(cs);
+        }
+    }
+}
+
+template <typename Kern>
+int ssd_smem_attr(Kern kern, size_t smem, bool (&attr_set)[kMaxDevices], int dev) {
     if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
             cudaSuccess)
             return SS_ERR_CUDA;
         if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
     }
-    kern<<<static_cast<unsigned>(ctas), kSsdThreads, smem, stream>>>(p);
+    return SS_OK;
+}
+
+// Plans the segments (split only with a workspace) and launches the state
+// pass, the fold and the main pass.
+template <int N>
+int launch_ssd(SsdParams& p, int64_t items, const SsdLayout& w, int32_t chunk_len, bool have_ws,
+               cudaStream_t stream) {
+    auto kmain = ss_ssd_kernel<N, false>;
+    auto kstate = ss_ssd_kernel<N, true>;
+    const size_t smem = sizeof(SsdSmem<N>);
+    static bool attr_main[kMaxDevices] = {false};
+    static bool attr_state[kMaxDevices] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
+    if (ssd_smem_attr(kmain, smem, attr_main, dev) != SS_OK || ssd_smem_attr(kstate, smem, attr_state, dev) != SS_OK)
+        return SS_ERR_CUDA;
+    p.nseg = 1;
+    p.cseg = static_cast<int>(w.nchunks);
+    if (have_ws) {
+        int per_sm = 0, sms = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kmain, kSsdThreads, smem) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return SS_ERR_CUDA;
+        ssd_segments(items, w.nchunks, w.kmax, static_cast<int64_t>(per_sm) * sms, chunk_len, p.nseg, p.cseg);
+    }
+    if (items * p.nseg >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    if (p.nseg > 1) {
+        kstate<<<static_cast<unsigned>(items * (p.nseg - 1)), kSsdThreads, smem, stream>>>(p);
+        const int64_t total = items * kSsdP * N;
+        const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), 4096);
+        ss_ssd_fold_kernel<N><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(p);
+    }
+    kmain<<<static_cast<unsigned>(items * p.nseg), kSsdThreads, smem, stream>>>(p);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
@@ -818,10 +896,16 @@ int ss_bwd(const void* u, const void* delta, const float* delta_bias, const floa
     return SS_OK;
 }
 
+size_t ss_ssd_fwd_workspace_bytes(const ss_ssd_dims* dims, uint32_t flags) {
+    if (!dims || (flags & ~kKnownFlags) || dims->batch < 0 || dims->seqlen < 0 || dims->nheads < 0) return 0;
+    if (dims->headdim != kSsdP || (dims->d_state != 64 && dims->d_state != 128)) return 0;
+    return ssd_layout(dims).total;
+}
+
 int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float* A, const void* B, const void* C,
                const float* D, void* y, float* final_state, uint32_t flags, const ss_ssd_dims* dims,
-               void* stream_v) {
-    if (!dims || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
+               const ss_launch* launch) {
+    if (!dims || !launch || (flags & ~kKnownFlags)) return SS_ERR_INVALID_ARG;
     const int64_t batch = dims->batch, L = dims->seqlen, H = dims->nheads;
     if (batch < 0 || L < 0 || H < 0) return SS_ERR_INVALID_ARG;
     if (dims->headdim != kSsdP || (dims->d_state != 64 && dims->d_state != 128)) return SS_ERR_UNSUPPORTED;
@@ -833,7 +917,10 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
     const void* ptrs[] = {x, dt, dt_bias, A, B, C, D, y, final_state};
     for (const void* q : ptrs)
         if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
-    cudaStream_t stream = static_cast<cudaStream_t>(stream_v);
+    const SsdLayout w = ssd_layout(dims);
+    const bool have_ws = launch->workspace != nullptr;
+    if (have_ws && (launch->workspace_bytes < w.total || !aligned16(launch->workspace))) return SS_ERR_WORKSPACE;
+    cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
     SsdParams p{};
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.dt = static_cast<const __nv_bfloat16*>(dt);
@@ -843,9 +930,16 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
     p.D = D;
     p.y = static_cast<__nv_bfloat16*>(y);
     p.final_state = final_state;
+    if (have_ws) {
+        unsigned char* ws = static_cast<unsigned char*>(launch->workspace);
+        p.rec = reinterpret_cast<float*>(ws + w.rec);
+        p.esum = reinterpret_cast<float*>(ws + w.esum);
+    }
     p.L = L; p.batch = static_cast<int>(batch); p.H = static_cast<int>(H);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
-    const int rc = dims->d_state == 128 ? launch_ssd<128>(p, batch * H, stream) : launch_ssd<64>(p, batch * H, stream);
+    const int64_t items = batch * H;
+    const int rc = dims->d_state == 128 ? launch_ssd<128>(p, items, w, launch->chunk_len, have_ws, stream)
+                                        : launch_ssd<64>(p, items, w, launch->chunk_len, have_ws, stream);
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) {
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;

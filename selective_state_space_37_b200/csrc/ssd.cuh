@@ -18,6 +18,12 @@
 // tiles; warp w owns rows 16w..16w+15 of S and Y (time) and of G (channel).
 // Three CTAs share an SM (62 KB of shared memory and <= 168 registers each),
 // so one CTA's tile copies (cp.async) and barriers overlap the others' products.
+// When batch x heads leaves SMs idle, each sequence is cut into nseg segments
+// of whole chunks and the carry between segments is made exact beforehand
+// (the recurrence is linear with a scalar decay): a state pass (STATE) runs
+// each segment but the last from G = 0 computing only G_out and Σ Δ A, a fold
+// turns those into the state entering every segment, and the main pass runs
+// each segment from its entering state.
 #pragma once
 
 #include "common.cuh"
@@ -40,8 +46,12 @@ struct SsdParams {
     const float* D;            // [H] or null
     __nv_bfloat16* y;          // [batch, L, H, P]
     float* final_state;        // [batch, H, P, N] or null
+    float* rec;                // [batch, H, nseg - 1, P, N]: segment end states from zero, then (folded) the
+                               // state entering the next segment
+    float* esum;               // [batch, H, nseg]: Σ Δ A over each segment
     int64_t L;
     int batch, H;
+    int nseg, cseg;            // time segments of the sequence and chunks per segment
     int softplus;
 };
 
@@ -83,7 +93,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int N>
+// Grid: one CTA per (segment k, batch b, head h), blockIdx.x = (k * batch + b) * H + h;
+// STATE runs segments 0 .. nseg - 2 only.
+template <int N, bool STATE>
 __global__ void __launch_bounds__(kSsdThreads, 3) ss_ssd_kernel(const __grid_constant__ SsdParams p) {
     constexpr int NT = N / 8;          // n8 tiles of the state width
     extern __shared__ __align__(16) unsigned char ssd_smem_raw[];
@@ -91,16 +103,32 @@ __global__ void __launch_bounds__(kSsdThreads, 3) ss_ssd_kernel(const __grid_con
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int g = lane >> 2, c = lane & 3;           // fragment row / column group
     const int h = blockIdx.x % p.H;
-    const int b = blockIdx.x / p.H;
+    const int b = (blockIdx.x / p.H) % p.batch;
+    const int sg = blockIdx.x / (p.H * p.batch);     // segment
+    const int64_t bh = static_cast<int64_t>(b) * p.H + h;
     const float Ah = p.A[h];
     const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
     const float Dh = p.D ? p.D[h] : 0.0f;
+    const int64_t seg_t0 = static_cast<int64_t>(sg) * p.cseg * kSsdQ;
+    const int64_t seg_t1 = min(seg_t0 + static_cast<int64_t>(p.cseg) * kSsdQ, p.L);
 
+    // G entering the segment: zero, or the folded record of the previous segment
+    const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kSsdP * N : nullptr;
     float accG[NT][4];                               // G rows 16w.. (channel p), all n
 #pragma unroll
-    for (int j = 0; j < NT; ++j) accG[j][0] = accG[j][1] = accG[j][2] = accG[j][3] = 0.0f;
-    for (int i = tid; i < kSsdP * (N + kSsdPad) / 2; i += kSsdThreads)
-        reinterpret_cast<uint32_t*>(&S.G[0][0])[i] = 0u;
+    for (int j = 0; j < NT; ++j) {
+        if (gin) {
+            const int nc = 8 * j + 2 * c;
+            const float2 lo = *reinterpret_cast<const float2*>(gin + (16 * w + g) * N + nc);
+            const float2 hi = *reinterpret_cast<const float2*>(gin + (16 * w + g + 8) * N + nc);
+            accG[j][0] = lo.x; accG[j][1] = lo.y; accG[j][2] = hi.x; accG[j][3] = hi.y;
+            *reinterpret_cast<uint32_t*>(&S.G[16 * w + g][nc]) = pack_bf16(lo.x, lo.y);
+            *reinterpret_cast<uint32_t*>(&S.G[16 * w + g + 8][nc]) = pack_bf16(hi.x, hi.y);
+        } else {
+            accG[j][0] = accG[j][1] = accG[j][2] = accG[j][3] = 0.0f;
+        }
+    }
+    float esum = 0.0f;                               // Σ Δ A over the segment (STATE)
 
     // Copies of one chunk's x, B, C tiles (rows past the sequence read as zero).
     auto issue_tiles = [&](int64_t t0, SsdTiles<N>& T) {
@@ -115,7 +143,7 @@ __global__ void __launch_bounds__(kSsdThreads, 3) ss_ssd_kernel(const __grid_con
             const int rr = r < q ? r : 0;
             const int64_t off = (static_cast<int64_t>(b) * p.L + t0 + rr) * N + k;
             cp_async16(&T.Bt[r][k], p.B + off, r < q);
-            cp_async16(&T.Ct[r][k], p.C + off, r < q);
+            if (!STATE) cp_async16(&T.Ct[r][k], p.C + off, r < q);
         }
     };
     // Warp 0 holds Δraw of the next chunk's steps 2·lane and 2·lane + 1.
@@ -127,9 +155,9 @@ __global__ void __launch_bounds__(kSsdThreads, 3) ss_ssd_kernel(const __grid_con
             dtn[e] = t < p.L ? __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t) * p.H + h]) : 0.0f;
         }
     };
-    if (w == 0) load_dt(0);
+    if (w == 0) load_dt(seg_t0);
 
-    for (int64_t t0 = 0; t0 < p.L; t0 += kSsdQ) {
+    for (int64_t t0 = seg_t0; t0 < seg_t1; t0 += kSsdQ) {
         const int q = static_cast<int>(p.L - t0 < kSsdQ ? p.L - t0 : kSsdQ);
         __syncthreads();   // the previous chunk is done with every tile and with cum / dlt
         issue_tiles(t0, S.tile[0]);
@@ -154,16 +182,47 @@ __global__ void __launch_bounds__(kSsdThreads, 3) ss_ssd_kernel(const __grid_con
             S.cum[2 * lane] = sc - a1;
             S.dlt[2 * lane] = dl[0];
             S.dlt[2 * lane + 1] = dl[1];
-            if (t0 + kSsdQ < p.L) load_dt(t0 + kSsdQ);
+            if (t0 + kSsdQ < seg_t1) load_dt(t0 + kSsdQ);
         }
         cp_async_wait_all();   // this thread's copies of the chunk have landed
         __syncthreads();
         auto& T = S.tile[0];
         const float cum_end = S.cum[kSsdQ - 1];
+        if (STATE) {
+            esum += cum_end;
+            // G_out = e^{cum_end} G_in + Xᵀ (scaled B): scale B, then the state product
+            for (int i = tid; i < kSsdQ * (N / 2); i += kSsdThreads) {
+                const int r = i / (N / 2), kk = (i % (N / 2)) * 2;
+                const float sc = __expf(cum_end - S.cum[r]) * S.dlt[r];
+                __nv_bfloat162* v = reinterpret_cast<__nv_bfloat162*>(&T.Bt[r][kk]);
+                const float2 f = __bfloat1622float2(*v);
+                *v = __floats2bfloat162_rn(f.x * sc, f.y * sc);
+            }
+            __syncthreads();
+            const float e_end = __expf(cum_end);
+#pragma unroll
+            for (int j = 0; j < NT; ++j) {
+                accG[j][0] *= e_end; accG[j][1] *= e_end;
+                accG[j][2] *= e_end; accG[j][3] *= e_end;
+            }
+#pragma unroll
+            for (int ks = 0; ks < kSsdQ; ks += 16) {
+                uint32_t af[4];
+                ldsm_x4_t(af, &T.X[ks + (lane & 7) + (lane >> 4) * 8][16 * w + ((lane >> 3) & 1) * 8]);
+#pragma unroll
+                for (int j = 0; j < NT; j += 2) {
+                    uint32_t bf[4];
+                    ldsm_x4_t(bf, &T.Bt[ks + (lane & 7) + ((lane >> 3) & 1) * 8][8 * j + (lane >> 4) * 8]);
+                    mma_bf16(accG[j], af, bf[0], bf[1]);
+                    mma_bf16(accG[j + 1], af, bf[2], bf[3]);
+                }
+            }
+            continue;
+        }
 
         // ----------- S = C Bᵀ (causal tiles only) and C G_inᵀ, sharing C's fragments
         const int nS = 2 * (w + 1);                 // s-tiles 0 .. 16w+15
-        const bool carry = t0 > 0;                  // G_in is zero before the first chunk
+        const bool carry = t0 > seg_t0 || sg > 0;   // G_in is zero before the sequence's first chunk
         float accS[8][4], accY[8][4];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -289,13 +348,43 @@ __global__ void __launch_bounds__(kSsdThreads, 3) ss_ssd_kernel(const __grid_con
             *reinterpret_cast<uint32_t*>(&S.G[16 * w + g + 8][nc]) = pack_bf16(accG[j][2], accG[j][3]);
         }
     }
-    if (p.final_state) {
-        float* fs = p.final_state + (static_cast<int64_t>(b) * p.H + h) * kSsdP * N;
+    if (STATE) {
+        float* gout = p.rec + (bh * (p.nseg - 1) + sg) * kSsdP * N;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+            const int nc = 8 * j + 2 * c;
+            *reinterpret_cast<float2*>(gout + (16 * w + g) * N + nc) = make_float2(accG[j][0], accG[j][1]);
+            *reinterpret_cast<float2*>(gout + (16 * w + g + 8) * N + nc) = make_float2(accG[j][2], accG[j][3]);
+        }
+        if (tid == 0) p.esum[bh * p.nseg + sg] = esum;
+        return;
+    }
+    if (p.final_state && sg == p.nseg - 1) {
+        float* fs = p.final_state + bh * kSsdP * N;
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
             const int nc = 8 * j + 2 * c;
             *reinterpret_cast<float2*>(fs + (16 * w + g) * N + nc) = make_float2(accG[j][0], accG[j][1]);
             *reinterpret_cast<float2*>(fs + (16 * w + g + 8) * N + nc) = make_float2(accG[j][2], accG[j][3]);
+        }
+    }
+}
+
+// Between the passes: one thread per (batch, head, p, n) folds the segment
+// records in order, G_in(k + 1) = e^{Σ_k Δ A} G_in(k) + G_loc(k) from
+// G_in(0) = 0, writing G_in(k + 1) over G_loc(k).
+template <int N>
+__global__ void __launch_bounds__(256) ss_ssd_fold_kernel(const __grid_constant__ SsdParams p) {
+    const int64_t per = static_cast<int64_t>(kSsdP) * N;
+    const int64_t total = static_cast<int64_t>(p.batch) * p.H * per;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t bh = i / per, e = i % per;
+        float gv = 0.0f;
+        for (int k = 0; k + 1 < p.nseg; ++k) {
+            float* r = p.rec + (bh * (p.nseg - 1) + k) * per + e;
+            gv = fmaf(expf(p.esum[bh * p.nseg + k]), gv, *r);
+            *r = gv;
         }
     }
 }

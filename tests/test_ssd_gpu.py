@@ -3,6 +3,8 @@ against oracle.ssd (fp64 recurrence, pinned in test_oracle_ssd_pins.py).
 Bound: max|y - y_ref| <= 2e-2 · max|y_ref| and the same for the final state
 -- the kernel rounds the decay-weighted C Bᵀ, the scaled B and the carried
 state's copy to bf16 (2^-9 relative each) before the tensor-core products."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -17,9 +19,9 @@ DEV = torch.device("cuda:0")
 TOL = 2e-2
 
 
-def run_and_ref(inp, softplus=True):
+def run_and_ref(inp, softplus=True, chunk_len=0, split=True):
     y, st = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
-                          softplus=softplus, sync_check=True)
+                          softplus=softplus, chunk_len=chunk_len, split=split, sync_check=True)
     yr, sr = oracle.ssd(to_f64(inp["x"]), to_f64(inp["dt"]), to_f64(inp["A"]), to_f64(inp["B"]),
                         to_f64(inp["C"]), D=to_f64(inp["D"]), dt_bias=to_f64(inp["dt_bias"]), softplus=softplus)
     return y, st, yr, sr
@@ -52,7 +54,9 @@ def test_ssd_zero_length_and_bad_sizes():
     y, st = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], sync_check=True)
     assert torch.count_nonzero(st).item() == 0
     dims = ss.ss_ssd_dims(1, 8, 2, 32, 64)        # headdim 32: unsupported
-    rc = ss.lib().ss_ssd_fwd(None, None, None, inp["A"].data_ptr(), None, None, None, None, None, 0, dims, None)
+    launch = ss.ss_launch(torch.cuda.current_stream().cuda_stream, None, 0, 0, 0)
+    rc = ss.lib().ss_ssd_fwd(None, None, None, inp["A"].data_ptr(), None, None, None, None, None, 0, dims,
+                             ctypes.byref(launch))
     assert rc == ss.SS_ERR_UNSUPPORTED
 
 
@@ -75,3 +79,39 @@ def test_ssd_full_size_sampled_heads():
         assert rel_max_err(to_f64(st[bi:bi + 1, h:h + 1]), sr) <= TOL, (bi, h)
     del inp, y, st
     torch.cuda.empty_cache()
+
+
+# Forced time segments (the segment length rounds up to whole 64-step
+# chunks): 2 .. 8 segments, ragged last chunk and segment, both state widths;
+# the state pass, the fold and the main pass must carry the state exactly.
+SEGS = [((2, 1000, 3, 128), 128), ((1, 333, 2, 64), 64), ((3, 700, 2, 128), 200), ((1, 4096, 1, 64), 512)]
+
+
+@pytest.mark.parametrize("shape,seg", SEGS, ids=[f"b{b}_L{l}_H{h}_N{n}_s{s}" for (b, l, h, n), s in SEGS])
+def test_ssd_time_segments(shape, seg):
+    b, L, H, N = shape
+    inp = ssd_inputs(b, L, H, N, seed=700 + L + seg, device=DEV)
+    y, st, yr, sr = run_and_ref(inp, chunk_len=seg)
+    assert rel_max_err(to_f64(y), yr) <= TOL
+    assert rel_max_err(to_f64(st), sr) <= TOL
+
+
+def test_ssd_split_matches_whole():
+    """Segments re-associate an exact linear recurrence: split and whole
+    results agree far inside the bf16 bound."""
+    inp = ssd_inputs(2, 2048, 4, 128, seed=17, device=DEV)
+    y1, s1 = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
+                           split=False, sync_check=True)
+    y2, s2 = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
+                           chunk_len=256, sync_check=True)
+    assert rel_max_err(to_f64(y2), to_f64(y1)) <= 1e-2
+    assert rel_max_err(to_f64(s2), to_f64(s1)) <= 1e-2
+
+
+def test_ssd_mamba2_130m_full():
+    """The Mamba-2-130M-shaped layer (batch 8, L 2048, 24 heads, d_state 128)
+    with the library's own segment choice, every output against the oracle."""
+    inp = ssd_inputs(8, 2048, 24, 128, seed=3, device=DEV)
+    y, st, yr, sr = run_and_ref(inp)
+    assert rel_max_err(to_f64(y), yr) <= TOL
+    assert rel_max_err(to_f64(st), sr) <= TOL
