@@ -695,6 +695,13 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
     sl.workspace_bytes = h.ws;
     const uint32_t fflags = flags & ~static_cast<uint32_t>(SS_SYNC_CHECK);
     auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+    // On an error after copies were queued, let them finish before returning:
+    // they read and write the caller's host buffers.
+    auto fail = [&](int code) {
+        cudaStreamSynchronize(hp->up);
+        cudaStreamSynchronize(hp->down);
+        return code;
+    };
     // the copy streams start after the work already queued on the caller's stream
     if (!ok(cudaEventRecord(hp->start, cs)) || !ok(cudaStreamWaitEvent(hp->up, hp->start, 0)) ||
         !ok(cudaStreamWaitEvent(hp->down, hp->start, 0)))
@@ -714,7 +721,7 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
         const size_t act_bytes = static_cast<size_t>(nr * L * d) * es, act_off = static_cast<size_t>(r0 * L * d) * es;
         const size_t bc_bytes = static_cast<size_t>(nr * L * kN) * es, bc_off = static_cast<size_t>(r0 * L * kN) * es;
         // upload (after the forward of slice s - 2 has read this slot)
-        if (s >= 2 && !ok(cudaStreamWaitEvent(hp->up, hp->done[slot], 0))) return SS_ERR_CUDA;
+        if (s >= 2 && !ok(cudaStreamWaitEvent(hp->up, hp->done[slot], 0))) return fail(SS_ERR_CUDA);
         if (!ok(cudaMemcpyAsync(su, static_cast<const unsigned char*>(u) + act_off, act_bytes, cudaMemcpyHostToDevice,
                                 hp->up)) ||
             !ok(cudaMemcpyAsync(sd, static_cast<const unsigned char*>(delta) + act_off, act_bytes,
@@ -726,17 +733,17 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
             !ok(cudaMemcpyAsync(sC, static_cast<const unsigned char*>(C) + bc_off, bc_bytes, cudaMemcpyHostToDevice,
                                 hp->up)) ||
             !ok(cudaEventRecord(hp->in_ready[slot], hp->up)))
-            return SS_ERR_CUDA;
+            return fail(SS_ERR_CUDA);
         // forward of the slice (after its upload, and after slice s - 2's y left this slot)
         if (!ok(cudaStreamWaitEvent(cs, hp->in_ready[slot], 0)) ||
             (s >= 2 && !ok(cudaStreamWaitEvent(cs, hp->out_free[slot], 0))))
-            return SS_ERR_CUDA;
+            return fail(SS_ERR_CUDA);
         ss_dims sdims = *dims;
         sdims.batch = nr;
         rc = fwd_impl(su, sd, delta_bias, A, sB, sC, D, z ? sz : nullptr, sy, last_state ? sst : nullptr, nullptr,
                       nullptr, fflags, &sdims, &sl);
-        if (rc != SS_OK) return rc;
-        if (!ok(cudaEventRecord(hp->done[slot], cs))) return SS_ERR_CUDA;
+        if (rc != SS_OK) return fail(rc);
+        if (!ok(cudaEventRecord(hp->done[slot], cs))) return fail(SS_ERR_CUDA);
         // download
         if (!ok(cudaStreamWaitEvent(hp->down, hp->done[slot], 0)) ||
             !ok(cudaMemcpyAsync(static_cast<unsigned char*>(y) + act_off, sy, act_bytes, cudaMemcpyDeviceToHost,
@@ -745,10 +752,11 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
                                                static_cast<size_t>(nr * d * kN) * sizeof(float),
                                                cudaMemcpyDeviceToHost, hp->down))) ||
             !ok(cudaEventRecord(hp->out_free[slot], hp->down)))
-            return SS_ERR_CUDA;
+            return fail(SS_ERR_CUDA);
     }
     // the caller's stream continues after the last download
-    if (!ok(cudaEventRecord(hp->end, hp->down)) || !ok(cudaStreamWaitEvent(cs, hp->end, 0))) return SS_ERR_CUDA;
+    if (!ok(cudaEventRecord(hp->end, hp->down)) || !ok(cudaStreamWaitEvent(cs, hp->end, 0)))
+        return fail(SS_ERR_CUDA);
     if (flags & SS_SYNC_CHECK) return ss_check(&sl);
     return SS_OK;
 }
