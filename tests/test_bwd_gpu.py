@@ -97,6 +97,15 @@ def test_bwd_time_chunks_fp32_general_A():
     check(got, ref, torch.float32)
 
 
+def test_bwd_time_chunks_fp32_aligned_rows():
+    """fp32 rows a multiple of 16 bytes: the chunk pass stages them with
+    16-byte asynchronous copies (4 channels each)."""
+    inp = fwd_inputs(2, 230, 64, 16, "fp32", 78, DEV, gate=True, D_kind="normal")
+    dy, dl = bwd_upstream(2, 230, 64, 16, "fp32", 78, DEV)
+    got, ref = run_both(inp, dy, dl, chunk_len=64)
+    check(got, ref, torch.float32)
+
+
 def test_bwd_chunked_matches_unchunked():
     """Chunking re-associates exact linear recurrences: the chunked and the
     one-chunk gradients agree to fp32 rounding."""
