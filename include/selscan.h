@@ -23,6 +23,7 @@
  *            (projections on cuBLAS, conv, scan, gate, output projection).
  *   ss_ssd_fwd  the multi-head scan with a scalar decay per head (Mamba-2's
  *            SSD model) on the tensor cores.
+ *   ss_fwd_with_state  ss_fwd from a given entering state (continuation).
  *   ss_fwd_host  ss_fwd on activations in host memory, with uploads, scans
  *            and downloads of batch slices overlapped.
  *   ss_bwd   the gradients of ss_fwd's inputs from the gradient of its outputs
@@ -303,6 +304,21 @@ SS_API int ss_bwd(const void* u, const void* delta, const float* delta_bias, con
                   const void* C, const float* D, const void* z, const void* dy, const float* dlast_state,
                   void* du, void* ddelta, float* dA, float* dB, float* dC, float* dD, void* dz,
                   float* ddelta_bias, uint32_t flags, const ss_dims* dims, const ss_launch* launch);
+
+/* ss_fwd_with_state -- ss_fwd from a given entering state instead of zero:
+ * h_{-1} = h_init ([batch, d_inner, d_state] fp32, device, 16-byte aligned;
+ * NULL is ss_fwd).  Continues a sequence after a previous call's last_state
+ * (a prompt processed in pieces, or the tail of a sequence whose head was
+ * scanned elsewhere): ss_fwd over [0, T) then ss_fwd_with_state over [T, L)
+ * from its last_state gives ss_fwd over [0, L) up to rounding.  Only the
+ * first time chunk reads h_init; the chunks' carry takes it to the rest.
+ * With seqlen 0, last_state = h_init.  Other arguments, workspace and errors:
+ * as ss_fwd.  (An engineering addition: the pages start every sequence from
+ * h = 0.) */
+SS_API int ss_fwd_with_state(const void* u, const void* delta, const float* delta_bias, const float* A,
+                             const void* B, const void* C, const float* D, const void* z, const float* h_init,
+                             void* y, float* last_state, uint32_t flags, const ss_dims* dims,
+                             const ss_launch* launch);
 
 /* ss_fwd_host -- ss_fwd on activations in HOST memory (an engineering
  * addition: the pages have no counterpart).  u, delta, z, B, C (inputs) and

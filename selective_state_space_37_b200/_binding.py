@@ -35,7 +35,7 @@ D_STATE = 16
 EXPORTED = ("ss_fwd", "ss_step", "ss_fwd_workspace_bytes", "ss_fwd_chunk_len", "ss_check",
             "ss_status_string", "ss_version", "ss_fwd_noalloc", "ss_bwd", "ss_bwd_workspace_bytes",
             "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_block_scratch_bytes", "ss_ssd_fwd",
-            "ss_fwd_host", "ss_fwd_host_workspace_bytes", "ss_ssd_fwd_workspace_bytes")
+            "ss_fwd_host", "ss_fwd_host_workspace_bytes", "ss_ssd_fwd_workspace_bytes", "ss_fwd_with_state")
 
 
 class ss_dims(ctypes.Structure):
@@ -103,6 +103,9 @@ def lib():
         L.ss_step.restype = ctypes.c_int
         L.ss_fwd_workspace_bytes.argtypes = [ctypes.POINTER(ss_dims), ctypes.c_uint32, ctypes.c_int32]
         L.ss_fwd_workspace_bytes.restype = ctypes.c_size_t
+        L.ss_fwd_with_state.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, f32p, vp, f32p, ctypes.c_uint32,
+                                        ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch)]
+        L.ss_fwd_with_state.restype = ctypes.c_int
         L.ss_fwd_host.argtypes = [vp, vp, f32p, f32p, vp, vp, f32p, vp, vp, f32p, ctypes.c_uint32,
                                   ctypes.POINTER(ss_dims), ctypes.POINTER(ss_launch), ctypes.c_int32]
         L.ss_fwd_host.restype = ctypes.c_int
@@ -207,8 +210,10 @@ def fwd_chunk_len(batch, seqlen, d_inner, bf16=True, d_state=D_STATE):
 
 def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, y=None, last_state=None,
            return_last_state=True, softplus=True, force_general_A=False, chunk_len=0,
-           timeout_iters=0, workspace=None, stream=None, sync_check=False, extra_flags=0):
-    """Selective-scan forward pass through libselscan's ss_fwd.
+           timeout_iters=0, workspace=None, stream=None, sync_check=False, extra_flags=0,
+           initial_state=None):
+    """Selective-scan forward pass through libselscan's ss_fwd (or
+    ss_fwd_with_state when initial_state [batch, d_inner, 16] fp32 is given).
 
     u, delta, z: [batch, L, d_inner]; B, C: [batch, L, 16] (bf16 or fp32, all the
     same); A: [d_inner, 16] fp32; D, delta_bias: [d_inner] fp32 or None.
@@ -247,9 +252,15 @@ def ss_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, *, y=None, last_s
         workspace = workspace_for(need, dev, sh)
     launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                        int(timeout_iters), int(chunk_len))
-    rc = lib().ss_fwd(_ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
-                      _ptr(z), _ptr(y), _ptr(last_state), flags, ctypes.byref(dims),
-                      ctypes.byref(launch))
+    if initial_state is not None:
+        _check(initial_state, "initial_state", (batch, d, D_STATE), torch.float32, dev)
+        rc = lib().ss_fwd_with_state(_ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                     _ptr(z), _ptr(initial_state), _ptr(y), _ptr(last_state), flags,
+                                     ctypes.byref(dims), ctypes.byref(launch))
+    else:
+        rc = lib().ss_fwd(_ptr(u), _ptr(delta), _ptr(delta_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                          _ptr(z), _ptr(y), _ptr(last_state), flags, ctypes.byref(dims),
+                          ctypes.byref(launch))
     if rc != SS_OK:
         raise SelscanError(rc, "ss_fwd")
     return y, last_state

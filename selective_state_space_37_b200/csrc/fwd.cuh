@@ -87,6 +87,7 @@ struct FwdParams {
     const void* z;
     void* y;
     float* last_state;
+    const float* h_init;   // [batch][d][kN] state entering the sequence, or null (zero)
     const float* conv_w;   // [d, kConvW] (conv prologue only)
     const float* conv_b;   // [d] or null
     int64_t L;
@@ -737,6 +738,11 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
 #pragma unroll
     for (int m = 0; m < 4; ++m) H[m] = pk2(0.f, 0.f);
     bool exact = true;
+    if (it.c == 0 && p.h_init && cp.valid) {   // the sequence starts from a given state
+        const float* r = p.h_init + (static_cast<int64_t>(it.b) * it.d + ch) * kN + hp;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) H[m] = pk2(__ldg(r + 2 * m), __ldg(r + 2 * m + 1));
+    }
     if (it.c > 0) {
         if (tid == 0)
             S.st = ld_acquire_gpu(p.status + (static_cast<int64_t>(it.b) * p.nchunks + (it.c - 1)) * p.nblk + it.g);

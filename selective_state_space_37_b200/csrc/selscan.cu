@@ -533,7 +533,8 @@ int ss_check(const ss_launch* launch) {
 // causal conv1d + SiLU prologue).
 static int fwd_impl(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
                     const void* C, const float* D, const void* z, void* y, float* last_state, const float* conv_w,
-                    const float* conv_b, uint32_t flags, const ss_dims* dims, const ss_launch* launch) {
+                    const float* conv_b, uint32_t flags, const ss_dims* dims, const ss_launch* launch,
+                    const float* h_init = nullptr) {
     const bool conv = conv_w != nullptr;
     int rc = validate_dims(dims, true);
     if (rc != SS_OK) return rc;
@@ -541,16 +542,16 @@ static int fwd_impl(const void* u, const void* delta, const float* delta_bias, c
     const int64_t batch = dims->batch, L = dims->seqlen, d = dims->d_inner;
     if (batch == 0 || d == 0) return SS_OK;
     cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
-    if (L == 0) {
-        if (last_state && !aligned16(last_state)) return SS_ERR_INVALID_ARG;
-        if (last_state &&
-            cudaMemsetAsync(last_state, 0, static_cast<size_t>(batch * d * kN) * sizeof(float), stream) !=
-                cudaSuccess)
+    if (L == 0) {   // last_state = the entering state
+        if ((last_state && !aligned16(last_state)) || (h_init && !aligned16(h_init))) return SS_ERR_INVALID_ARG;
+        const size_t bytes = static_cast<size_t>(batch * d * kN) * sizeof(float);
+        if (last_state && (h_init ? cudaMemcpyAsync(last_state, h_init, bytes, cudaMemcpyDeviceToDevice, stream)
+                                  : cudaMemsetAsync(last_state, 0, bytes, stream)) != cudaSuccess)
             return SS_ERR_CUDA;
         return SS_OK;
     }
     if (!u || !delta || !A || !B || !C || !y) return SS_ERR_INVALID_ARG;
-    const void* ptrs[] = {u, delta, delta_bias, A, B, C, D, z, y, last_state, conv_w, conv_b};
+    const void* ptrs[] = {u, delta, delta_bias, A, B, C, D, z, y, last_state, conv_w, conv_b, h_init};
     for (const void* q : ptrs)
         if (q && !aligned16(q)) return SS_ERR_INVALID_ARG;
 
@@ -566,7 +567,7 @@ static int fwd_impl(const void* u, const void* delta, const float* delta_bias, c
 
     FwdParams p{};
     p.u = u; p.delta = delta; p.bias = delta_bias; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
-    p.y = y; p.last_state = last_state;
+    p.y = y; p.last_state = last_state; p.h_init = h_init;
     p.conv_w = conv_w; p.conv_b = conv_b;
     p.L = L; p.batch = static_cast<int>(batch); p.d = static_cast<int>(d);
     p.chunk_len = static_cast<int>(pl.chunk_len > 0 ? pl.chunk_len : L);
@@ -759,6 +760,12 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
         return fail(SS_ERR_CUDA);
     if (flags & SS_SYNC_CHECK) return ss_check(&sl);
     return SS_OK;
+}
+
+int ss_fwd_with_state(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
+                      const void* C, const float* D, const void* z, const float* h_init, void* y, float* last_state,
+                      uint32_t flags, const ss_dims* dims, const ss_launch* launch) {
+    return fwd_impl(u, delta, delta_bias, A, B, C, D, z, y, last_state, nullptr, nullptr, flags, dims, launch, h_init);
 }
 
 int ss_fwd_conv(const void* x, const float* conv_w, const float* conv_b, const void* delta, const float* delta_bias,

@@ -201,3 +201,38 @@ def test_config_sampled(name, count):
         assert es <= 2e-2, f"{name} state vs {prec}: {es:.3g}"
     del inp, y, st
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------- entering state (continuation)
+CONT = [((2, 400, 256), 150, 0, 0), ((2, 400, 256), 256, 64, 64), ((1, 700, 128), 333, 0, 96),
+        ((3, 130, 70), 64, 32, 32)]
+
+
+@pytest.mark.parametrize("shape,split,c1,c2", CONT,
+                         ids=[f"b{b}_L{l}_d{d}_at{s}_c{c1}_{c2}" for (b, l, d), s, c1, c2 in CONT])
+def test_continuation_from_last_state(shape, split, c1, c2):
+    """ss_fwd over [0, T) then ss_fwd_with_state over [T, L) from its last
+    state reproduces the whole-sequence oracle (every output of both parts
+    and the final state), with and without time chunks in either part."""
+    b, L, d = shape
+    inp = fwd_inputs(b, L, d, 16, "bf16", 55 + L + split, DEV, gate=True, D_kind="normal")
+    part = lambda sl: {k: (v[:, sl].contiguous() if k in ("u", "delta", "z", "B", "C") and v is not None else v)
+                       for k, v in inp.items()}
+    p1, p2 = part(slice(0, split)), part(slice(split, L))
+    y1, s1 = run(p1, chunk_len=c1, sync_check=True)
+    y2, s2 = run(p2, chunk_len=c2, initial_state=s1, sync_check=True)
+    yr, sr = oracle_full(inp, precision="f64")
+    tol = tol_for(torch.bfloat16)
+    assert rel_max_err(to_f64(torch.cat([y1, y2], dim=1)), yr) <= tol
+    assert rel_max_err(to_f64(s2), sr) <= tol
+
+
+def test_with_state_zero_length_and_zero_state():
+    inp = fwd_inputs(2, 0, 64, 16, "bf16", 3, DEV)
+    h0 = torch.randn(2, 64, 16, device=DEV)
+    _, st = run(inp, initial_state=h0, sync_check=True)
+    assert torch.equal(st, h0)
+    inp = fwd_inputs(2, 100, 64, 16, "bf16", 4, DEV, gate=True)
+    ya, sa = run(inp, sync_check=True)
+    yb, sb = run(inp, initial_state=torch.zeros(2, 64, 16, device=DEV), sync_check=True)
+    assert torch.equal(ya, yb) and torch.equal(sa, sb)
