@@ -125,8 +125,6 @@ struct BwdSmem {
 struct BwdChan {
     float A[kBH];      // A[ch, 8p + m]
     float Al[kBH];     // A[ch, 8p + m] · log2 e (exp(Δ A) = 2^(Δ Al))
-    float al;          // structured path (A[ch, n] = a (n + 1)): a · log2 e
-    float alb;         // a (8p + 1) · log2 e: exponent factor of the half's first decay
     float bias, Dv;
     float al_s, bias_s;   // a · log2 e and the bias of the channel this thread stages (threadIdx.x % kBwdCh)
     int c;             // channel within the block
@@ -685,8 +683,6 @@ __device__ __forceinline__ bool init_chan(const BwdParams& p, int blk, BwdChan& 
         cp.Al[m] = cp.A[m] * kLog2e;
         structured = structured && (cp.A[m] == a0 * static_cast<float>(hp + m + 1));
     }
-    cp.al = a0 * kLog2e;
-    cp.alb = cp.al * static_cast<float>(hp + 1);
     cp.bias = (cp.valid && p.bias) ? p.bias[ch] : 0.0f;
     {
         const int cs = blk * kBwdCh + static_cast<int>(threadIdx.x % kBwdCh);   // channel this thread stages
