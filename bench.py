@@ -438,7 +438,8 @@ def time_decode(ss, torch, device, steps_total=1000, reps=3):
     step is timed alone with CUDA events after an L2 flush (a 256 MB write
     followed by a 256 MB read of another buffer);
     returns (ms per step, bytes per step, ms per step back to back in one CUDA
-    graph with no flush, where the state may stay in L2)."""
+    graph with no flush, where the state may stay in L2, and (ms, bytes) of a
+    bare in-place stream over the same state timed the same way)."""
     from ss_inputs import CONFIGS, step_inputs, step_sequence_inputs
     c = CONFIGS["decode"]
     base = step_inputs(c.batch, c.d_inner, c.d_state, c.dtype, c.seed, device, gate=c.gate)
@@ -470,6 +471,24 @@ def time_decode(ss, torch, device, steps_total=1000, reps=3):
     torch.cuda.synchronize(device)
     ms_cold = sum(s.elapsed_time(e) for s, e in zip(starts, ends)) / steps_total
 
+    # Calibration: the bare in-place stream over the same state (multiply by
+    # one, torch's elementwise kernel), timed the same way -- the ceiling of a
+    # read-modify-write stream of this size, below the long-stream copy peak.
+    cal = []
+    for i in range(30):
+        flush_w.zero_()
+        torch.sum(flush_r, dim=None, out=sink)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        state.mul_(1.0)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        if i >= 5:
+            cal.append(e0.elapsed_time(e1))
+    ms_inplace = statistics.median(cal)
+    inplace_bytes = 2 * state.numel() * state.element_size()
+
     def run_all():
         # launches on whatever stream is current (the capture stream in graph mode)
         for t in range(steps_total):
@@ -496,7 +515,7 @@ def time_decode(ss, torch, device, steps_total=1000, reps=3):
     torch.cuda.synchronize(device)
     ms_warm = e0.elapsed_time(e1) / (reps * steps_total)
     del g
-    return ms_cold, c.compulsory_bytes_per_step(), ms_warm
+    return ms_cold, c.compulsory_bytes_per_step(), ms_warm, (ms_inplace, inplace_bytes)
 
 
 def cpu_baseline(cfg, budget_s=10.0):
@@ -587,14 +606,19 @@ def run_ours(args):
                             "chunk_len": ss.fwd_chunk_len(c.batch, c.seqlen, c.d_inner)}
             del i2, y2, s2, w2
             torch.cuda.empty_cache()
-        dms, dbytes, dms_warm = time_decode(ss, torch, device)
+        dms, dbytes, dms_warm, (ims, ibytes) = time_decode(ss, torch, device)
+        igbs = ibytes / (ims * 1e-3) / 1e9
         extras["decode"] = {"ms_per_step": dms, "steps_per_s": 1e3 / dms,
                             "GB_s": dbytes / (dms * 1e-3) / 1e9,
                             "frac_of_hbm": dbytes / (dms * 1e-3) / 1e9 / hbm,
                             "note": "1000 ss_step calls, batch 256, d_inner 5120; each step "
                                     "timed alone after an L2 flush (the 84 MB state fits in L2)",
                             "graph_back_to_back_ms_per_step": dms_warm,
-                            "graph_back_to_back_steps_per_s": 1e3 / dms_warm}
+                            "graph_back_to_back_steps_per_s": 1e3 / dms_warm,
+                            "inplace_stream_same_size": {"ms": ims, "GB_s": igbs,
+                                                         "what": "torch in-place multiply of the same "
+                                                                 "state, timed the same way"},
+                            "frac_of_inplace_stream": dbytes / (dms * 1e-3) / 1e9 / igbs}
         torch.cuda.empty_cache()
         for name in ("mamba2p8b", "mamba130m"):
             c = CONFIGS[name]
@@ -731,11 +755,13 @@ def run_decode_only(args):
     torch.cuda.set_device(device)
     ss.lib()
     hbm, peak_kind = peaks()
-    ms, nbytes, ms_warm = time_decode(ss, torch, device, steps_total=max(args.steps, 4), reps=1)
+    ms, nbytes, ms_warm, (ims, ibytes) = time_decode(ss, torch, device, steps_total=max(args.steps, 4), reps=1)
+    gbs = nbytes / (ms * 1e-3) / 1e9
     print(json.dumps({"metric": "decode steps/s", "value": 1e3 / ms, "unit": "steps/s",
                       "n_gpus": 1, "steps": args.steps, "ms_per_step": ms,
-                      "GB_s": nbytes / (ms * 1e-3) / 1e9, "frac_of_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
-                      "peak_kind": peak_kind, "graph_back_to_back_ms_per_step": ms_warm}), flush=True)
+                      "GB_s": gbs, "frac_of_hbm": gbs / hbm,
+                      "peak_kind": peak_kind, "graph_back_to_back_ms_per_step": ms_warm,
+                      "frac_of_inplace_stream": gbs / (ibytes / (ims * 1e-3) / 1e9)}), flush=True)
 
 
 def run_bwd_only(args):
