@@ -166,4 +166,73 @@ __global__ void __launch_bounds__(kStepThreads) ss_step_kernel(const __grid_cons
     }
 }
 
+// The same step for problems the grid tiles exactly (d_inner a multiple of
+// kStepChanPerBlock, batch = 2 x gridDim.y, batch x d_inner x kN < 2^31) and
+// no conv prologue: every thread has a valid channel and two valid batch
+// rows, and every element offset fits in 32 bits, so the body carries no
+// bounds predicates and no 64-bit index arithmetic (about half the
+// instructions of the general kernel on the decode workload).
+template <typename IO>
+__global__ void __launch_bounds__(kStepThreads) ss_step_full_kernel(const __grid_constant__ StepParams p) {
+    constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
+    const int q = threadIdx.x & 3;   // states 4q .. 4q+3
+    const int ch = blockIdx.x * kStepChanPerBlock + (threadIdx.x >> 2);
+    const int d = p.d;
+    float Av[4];
+    load4<float>(p.A + ch * kN + 4 * q, Av);
+    const float Dv = p.D ? __ldg(p.D + ch) : 0.f;
+    const float bv = p.bias ? __ldg(p.bias + ch) : 0.f;
+    const IO* u = static_cast<const IO*>(p.u);
+    const IO* dl = static_cast<const IO*>(p.delta);
+    const IO* zp = static_cast<const IO*>(p.z);
+    const IO* Bp = static_cast<const IO*>(p.B);
+    const IO* Cp = static_cast<const IO*>(p.C);
+    IO* yp = static_cast<IO*>(p.y);
+    int bb[2], cs[2];
+    bb[0] = blockIdx.y;
+    bb[1] = blockIdx.y + gridDim.y;
+    float4 h4[2];
+    float uu[2], xr[2], zz[2], Bv[2][4], Cv[2][4];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        cs[r] = bb[r] * d + ch;
+        h4[r] = *(reinterpret_cast<const float4*>(p.state + cs[r] * kN) + q);
+        uu[r] = to_f32(u[cs[r]]);
+        xr[r] = to_f32(dl[cs[r]]);
+        zz[r] = zp ? to_f32(zp[cs[r]]) : 0.f;
+        load4<IO>(Bp + bb[r] * kN + 4 * q, Bv[r]);
+        load4<IO>(Cp + bb[r] * kN + 4 * q, Cv[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        float lam, dscale;
+        if (FAST) {
+            const float y2 = fmaf(xr[r], kLog2e, bv * kLog2e);
+            lam = p.softplus ? softplus_log2_fast(y2) : y2;
+            dscale = kLn2;
+        } else {
+            const float x = xr[r] + bv;
+            lam = p.softplus ? softplus_accurate(x) : x;
+            dscale = 1.0f;
+        }
+        const float du = lam * (dscale * uu[r]);
+        float hv[4] = {h4[r].x, h4[r].y, h4[r].z, h4[r].w};
+        float acc = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            const float a = FAST ? ex2_approx(lam * Av[m]) : expf(lam * Av[m]);
+            hv[m] = fmaf(a, hv[m], du * Bv[r][m]);
+            acc = fmaf(Cv[r][m], hv[m], acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        *(reinterpret_cast<float4*>(p.state + cs[r] * kN) + q) = make_float4(hv[0], hv[1], hv[2], hv[3]);
+        if (q == 0) {
+            float yv = fmaf(Dv, uu[r], acc);
+            if (zp) yv *= FAST ? silu_tanh(zz[r]) : silu_accurate(zz[r]);
+            yp[cs[r]] = from_f32<IO>(yv);
+        }
+    }
+}
+
 }  // namespace selscan
