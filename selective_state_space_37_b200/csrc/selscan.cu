@@ -819,11 +819,13 @@ static int step_impl(float* state, const void* u, const void* delta, const float
                     static_cast<unsigned>(std::min<int64_t>(ceil_div(batch, 2), 65535)));
     cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
     // exact tiling, 32-bit offsets: the predicate-free kernel
-    const bool full = !conv && d % kStepChanPerBlock == 0 && batch % 2 == 0 && batch / 2 <= 65535 &&
-                      batch * d * kN < (int64_t(1) << 31);
+    constexpr int kFullRows = 1;   // batch rows per thread of the exact-tiling kernel (1, 2, 4 measured: 1 best)
+    const bool full = !conv && d % kStepChanPerBlock == 0 && batch % kFullRows == 0 &&
+                      batch / kFullRows <= 65535 && batch * d * kN < (int64_t(1) << 31);
     if (full) {
-        if (bf16) ss_step_full_kernel<__nv_bfloat16><<<grid, kStepThreads, 0, stream>>>(p);
-        else      ss_step_full_kernel<float><<<grid, kStepThreads, 0, stream>>>(p);
+        const dim3 fgrid(static_cast<unsigned>(d / kStepChanPerBlock), static_cast<unsigned>(batch / kFullRows));
+        if (bf16) ss_step_full_kernel<__nv_bfloat16, kFullRows><<<fgrid, kStepThreads, 0, stream>>>(p);
+        else      ss_step_full_kernel<float, kFullRows><<<fgrid, kStepThreads, 0, stream>>>(p);
     } else if (bf16) {
         if (conv) ss_step_kernel<__nv_bfloat16, true><<<grid, kStepThreads, 0, stream>>>(p);
         else      ss_step_kernel<__nv_bfloat16, false><<<grid, kStepThreads, 0, stream>>>(p);

@@ -167,12 +167,12 @@ __global__ void __launch_bounds__(kStepThreads) ss_step_kernel(const __grid_cons
 }
 
 // The same step for problems the grid tiles exactly (d_inner a multiple of
-// kStepChanPerBlock, batch = 2 x gridDim.y, batch x d_inner x kN < 2^31) and
-// no conv prologue: every thread has a valid channel and two valid batch
-// rows, and every element offset fits in 32 bits, so the body carries no
+// kStepChanPerBlock, batch = R x gridDim.y, batch x d_inner x kN < 2^31) and
+// no conv prologue: every thread has a valid channel and R valid batch
+// rows (all loads issued before the math), and every element offset fits in 32 bits, so the body carries no
 // bounds predicates and no 64-bit index arithmetic (about half the
 // instructions of the general kernel on the decode workload).
-template <typename IO>
+template <typename IO, int R>
 __global__ void __launch_bounds__(kStepThreads) ss_step_full_kernel(const __grid_constant__ StepParams p) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
     const int q = threadIdx.x & 3;   // states 4q .. 4q+3
@@ -188,13 +188,12 @@ __global__ void __launch_bounds__(kStepThreads) ss_step_full_kernel(const __grid
     const IO* Bp = static_cast<const IO*>(p.B);
     const IO* Cp = static_cast<const IO*>(p.C);
     IO* yp = static_cast<IO*>(p.y);
-    int bb[2], cs[2];
-    bb[0] = blockIdx.y;
-    bb[1] = blockIdx.y + gridDim.y;
-    float4 h4[2];
-    float uu[2], xr[2], zz[2], Bv[2][4], Cv[2][4];
+    int bb[R], cs[R];
+    float4 h4[R];
+    float uu[R], xr[R], zz[R], Bv[R][4], Cv[R][4];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < R; ++r) {
+        bb[r] = blockIdx.y + r * gridDim.y;
         cs[r] = bb[r] * d + ch;
         h4[r] = *(reinterpret_cast<const float4*>(p.state + cs[r] * kN) + q);
         uu[r] = to_f32(u[cs[r]]);
@@ -204,7 +203,7 @@ __global__ void __launch_bounds__(kStepThreads) ss_step_full_kernel(const __grid
         load4<IO>(Cp + bb[r] * kN + 4 * q, Cv[r]);
     }
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
+    for (int r = 0; r < R; ++r) {
         float lam, dscale;
         if (FAST) {
             const float y2 = fmaf(xr[r], kLog2e, bv * kLog2e);
