@@ -147,3 +147,42 @@ def test_python_binding_checks_arguments():
     with pytest.raises(ValueError):
         ss.ss_step(torch.zeros(1, 8, 16), torch.zeros(1, 8), torch.zeros(1, 8), torch.zeros(8, 16),
                    torch.zeros(1, 16), torch.zeros(1, 16))
+
+
+def test_python_binding_checks_new_entry_points():
+    """The host-buffer forward wants its parameters on a CUDA device; the
+    backward, SSD and entering-state forward refuse CPU tensors before any
+    library call (no GPU needed to check)."""
+    import torch
+    u = torch.zeros(1, 4, 8)
+    A = torch.zeros(8, 16)
+    B = torch.zeros(1, 4, 16)
+    with pytest.raises(ValueError):
+        ss.ss_fwd_host(u, u, A, B, B)                  # A on the CPU
+    with pytest.raises(ValueError):
+        ss.ss_bwd(u, u, A, B, B, u)                    # CPU tensors
+    with pytest.raises(ValueError):
+        ss.ss_fwd(u, u, A, B, B, initial_state=torch.zeros(1, 8, 16))
+    with pytest.raises(ValueError):
+        ss.ss_fwd_host(torch.zeros(1, 4), u, A, B, B)  # u not [batch, L, d_inner]
+
+
+def test_host_and_ssd_workspace_sizes(L):
+    """ss_fwd_host's staging is two slots of one slice's activations and
+    states plus one slice's forward workspace; ss_ssd_fwd's workspace holds
+    segment records for min(8, chunks) segments."""
+    al = lambda x: (x + 255) // 256 * 256
+    dims = ss.ss_dims(3, 100, 64, 16)
+    for rows in (1, 2, 3, 5):
+        r = min(rows, 3)
+        slot = 4 * al(r * 100 * 64 * 2) + 2 * al(r * 100 * 16 * 2) + al(r * 64 * 16 * 4)
+        fwd = al(L.ss_fwd_workspace_bytes(ctypes.byref(ss.ss_dims(r, 100, 64, 16)), ss.SS_BF16, 0))
+        assert L.ss_fwd_host_workspace_bytes(ctypes.byref(dims), ss.SS_BF16, rows) == 2 * slot + fwd
+    assert L.ss_fwd_host_workspace_bytes(ctypes.byref(ss.ss_dims(0, 100, 64, 16)), ss.SS_BF16, 1) == 0
+    for b, Lq, H, N in ((2, 1000, 3, 128), (1, 64, 2, 64), (4, 8192, 80, 128)):
+        chunks = max(1, -(-Lq // 64))
+        k = min(8, chunks)
+        want = al(b * H * (k - 1) * 64 * N * 4) + al(b * H * k * 4)
+        got = L.ss_ssd_fwd_workspace_bytes(ctypes.byref(ss.ss_ssd_dims(b, Lq, H, 64, N)), 0)
+        assert got == want, (b, Lq, H, N)
+    assert L.ss_ssd_fwd_workspace_bytes(ctypes.byref(ss.ss_ssd_dims(1, 64, 2, 32, 64)), 0) == 0
