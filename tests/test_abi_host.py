@@ -186,3 +186,21 @@ def test_host_and_ssd_workspace_sizes(L):
         got = L.ss_ssd_fwd_workspace_bytes(ctypes.byref(ss.ss_ssd_dims(b, Lq, H, 64, N)), 0)
         assert got == want, (b, Lq, H, N)
     assert L.ss_ssd_fwd_workspace_bytes(ctypes.byref(ss.ss_ssd_dims(1, 64, 2, 32, 64)), 0) == 0
+
+
+def test_missing_library_fails_loudly():
+    """With the native library absent, the binding raises instead of falling
+    back to any other implementation (checked in a fresh interpreter)."""
+    import subprocess
+    import sys
+    code = ("import selective_state_space_37_b200 as ss\n"
+            "try:\n"
+            "    ss.lib()\n"
+            "except RuntimeError as e:\n"
+            "    print('raised', 'not found' in str(e))\n"
+            "else:\n"
+            "    print('loaded')\n")
+    env = dict(os.environ, SELSCAN_LIB="/nonexistent/libselscan.so")
+    out = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, env=env,
+                         cwd=os.path.dirname(os.path.dirname(os.path.abspath(__file__))), timeout=300)
+    assert out.stdout.strip() == "raised True", out.stdout + out.stderr
