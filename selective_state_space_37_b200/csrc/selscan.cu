@@ -6,6 +6,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -29,15 +30,32 @@ constexpr int kMaxDevices = 64;
 constexpr uint32_t kKnownFlags = SS_BF16 | SS_DELTA_SOFTPLUS | SS_SYNC_CHECK | SS_FORCE_GENERAL_A |
                                  SS_TEST_DROP_CARRY;
 
+// Per-device caches below are atomics: host threads may make their first
+// calls concurrently (they store the same values).
 int sm_count_of_current_device() {
-    static int cache[kMaxDevices] = {0};
+    static std::atomic<int> cache[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
-    if (dev < kMaxDevices && cache[dev] > 0) return cache[dev];
+    if (dev < kMaxDevices) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     int n = 0;
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-    if (dev < kMaxDevices) cache[dev] = n;
+    if (dev < kMaxDevices) cache[dev].store(n, std::memory_order_relaxed);
     return n;
+}
+
+// Raises a kernel's dynamic shared-memory limit to `smem` once per device.
+template <typename Kern>
+int set_smem_limit(Kern kern, size_t smem, std::atomic<bool> (&done)[kMaxDevices], int dev) {
+    const bool cached = dev >= 0 && dev < kMaxDevices;
+    if (cached && done[dev].load(std::memory_order_acquire)) return SS_OK;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+        cudaSuccess)
+        return SS_ERR_CUDA;
+    if (cached) done[dev].store(true, std::memory_order_release);
+    return SS_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -166,15 +184,9 @@ template <typename IO, bool TMA, int STAGES, int MINB, int G, bool UNROLL, bool 
 int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
     auto kern = ss_fwd_kernel<IO, TMA, STAGES, MINB, G, UNROLL, CONV>;
     const size_t smem = sizeof(FwdSmem<IO, STAGES>);
-    static bool attr_set[kMaxDevices] = {false};
+    static std::atomic<bool> attr_set[kMaxDevices];
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-            cudaSuccess)
-            return SS_ERR_CUDA;
-        if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
-    }
+    if (cudaGetDevice(&dev) != cudaSuccess || set_smem_limit(kern, smem, attr_set, dev) != SS_OK) return SS_ERR_CUDA;
     kern<<<static_cast<unsigned>(items), kNT, smem, stream>>>(p, maps[0], maps[1], maps[2], maps[3], maps[4],
                                                               maps[5]);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
@@ -246,17 +258,6 @@ void ssd_segments(int64_t items, int64_t nchunks, int64_t kmax, int64_t slots, i
     }
 }
 
-template <typename Kern>
-int ssd_smem_attr(Kern kern, size_t smem, bool (&attr_set)[kMaxDevices], int dev) {
-    if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-            cudaSuccess)
-            return SS_ERR_CUDA;
-        if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
-    }
-    return SS_OK;
-}
-
 // Plans the segments (split only with a workspace) and launches the state
 // pass, the fold and the main pass.
 template <int N>
@@ -265,11 +266,11 @@ int launch_ssd(SsdParams& p, int64_t items, const SsdLayout& w, int32_t chunk_le
     auto kmain = ss_ssd_kernel<N, false>;
     auto kstate = ss_ssd_kernel<N, true>;
     const size_t smem = sizeof(SsdSmem<N>);
-    static bool attr_main[kMaxDevices] = {false};
-    static bool attr_state[kMaxDevices] = {false};
+    static std::atomic<bool> attr_main[kMaxDevices];
+    static std::atomic<bool> attr_state[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
-    if (ssd_smem_attr(kmain, smem, attr_main, dev) != SS_OK || ssd_smem_attr(kstate, smem, attr_state, dev) != SS_OK)
+    if (set_smem_limit(kmain, smem, attr_main, dev) != SS_OK || set_smem_limit(kstate, smem, attr_state, dev) != SS_OK)
         return SS_ERR_CUDA;
     p.nseg = 1;
     p.cseg = static_cast<int>(w.nchunks);
@@ -363,17 +364,6 @@ void bwd_chunks(int64_t items, int64_t nseg, int64_t kmax, int64_t slots, int32_
     }
 }
 
-template <typename Kern>
-int set_bwd_smem(Kern kern, size_t smem, bool (&attr_set)[kMaxDevices], int dev) {
-    if (dev < 0 || dev >= kMaxDevices || !attr_set[dev]) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-            cudaSuccess)
-            return SS_ERR_CUDA;
-        if (dev >= 0 && dev < kMaxDevices) attr_set[dev] = true;
-    }
-    return SS_OK;
-}
-
 // Plans the chunks (needs the kernels' occupancy) and launches the chunk pass
 // then the gradient pass.
 template <typename IO, bool SP, bool HZ>
@@ -381,13 +371,13 @@ int launch_bwd(BwdParams& p, int64_t items, int64_t kmax, int32_t chunk_len, cud
     auto kchunk = ss_bwd_chunk_kernel<IO, SP, HZ>;
     auto kgrad = ss_bwd_kernel<IO, SP, HZ>;
     const size_t smem = sizeof(BwdSmem<IO>);
-    static bool attr_chunk[kMaxDevices] = {false};
-    static bool attr_grad[kMaxDevices] = {false};
+    static std::atomic<bool> attr_chunk[kMaxDevices];
+    static std::atomic<bool> attr_grad[kMaxDevices];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
     const size_t smem_chunk = sizeof(ChunkSmem<IO>);
-    if (set_bwd_smem(kchunk, smem_chunk, attr_chunk, dev) != SS_OK ||
-        set_bwd_smem(kgrad, smem, attr_grad, dev) != SS_OK)
+    if (set_smem_limit(kchunk, smem_chunk, attr_chunk, dev) != SS_OK ||
+        set_smem_limit(kgrad, smem, attr_grad, dev) != SS_OK)
         return SS_ERR_CUDA;
     int per_sm = 0, sms = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kgrad, kBwdThreads, smem) != cudaSuccess ||
