@@ -28,7 +28,9 @@
 //               checkpoints, with Σ Δ since the chunk's start) and the
 //               chunk's end state h_loc; then (chunks k > 0) the adjoint-only
 //               recurrence g ← exp(Δ A)(g + ds C) from zero backwards over
-//               the chunk, giving g_loc.
+//               the chunk, giving g_loc.  Its segment tiles arrive by
+//               cp.async into a double-buffered raw area while the previous
+//               segment's steps run (ChunkSmem).
 //   ss_bwd_combine_kernel -- folds the records in chunk order into h_in(k)
 //               and G_in(k) for every chunk (one thread per state).
 //   ss_bwd_kernel -- per item: h_in and G_in from the folded records; then
