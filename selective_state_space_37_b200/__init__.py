@@ -23,12 +23,12 @@ from ._binding import (D_STATE, EXPORTED, LIB_PATH, SS_BF16, SS_DELTA_SOFTPLUS,
                        fwd_chunk_len, ss_block_fwd, ss_block_weights, ss_ssd_dims, ss_ssd_fwd,
                        fwd_workspace_bytes, lib, ss_bwd, ss_check, ss_dims, ss_fwd, ss_fwd_conv,
                        ss_launch, ss_step, ss_step_conv, status_string, workspace_for,
-                       ss_fwd_host, fwd_host_workspace_bytes)
+                       ss_fwd_host, fwd_host_workspace_bytes, clear_workspaces)
 
 __all__ = ["ss_fwd", "ss_fwd_host", "fwd_host_workspace_bytes", "ss_step", "ss_bwd", "ss_fwd_conv", "ss_step_conv", "ss_block_fwd", "ss_ssd_fwd",
            "block_scratch_bytes", "ss_block_weights", "ss_ssd_dims", "ss_check", "fwd_workspace_bytes", "fwd_chunk_len",
            "bwd_workspace_bytes",
-           "status_string", "lib", "SelscanError", "ss_dims", "ss_launch", "workspace_for",
+           "status_string", "lib", "SelscanError", "ss_dims", "ss_launch", "workspace_for", "clear_workspaces",
            "D_STATE", "EXPORTED", "LIB_PATH", "SS_OK", "SS_ERR_INVALID_ARG",
            "SS_ERR_UNSUPPORTED", "SS_ERR_CUDA", "SS_ERR_TIMEOUT", "SS_ERR_WORKSPACE",
            "SS_BF16", "SS_DELTA_SOFTPLUS", "SS_SYNC_CHECK", "SS_FORCE_GENERAL_A",

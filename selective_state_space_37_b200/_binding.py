@@ -183,13 +183,24 @@ _ws_cache = {}
 
 
 def workspace_for(nbytes, device, stream_handle):
-    """A cached device workspace of at least nbytes for (device, stream)."""
+    """A cached device workspace of at least nbytes for (device, stream).
+
+    One buffer per (device, stream), grown when a call needs more; calls on
+    one stream run in order, so they can share it.  A replaced buffer is
+    returned to torch's stream-ordered allocator.  clear_workspaces() drops
+    them all."""
     key = (device.index, int(stream_handle))
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < nbytes:
         ws = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
         _ws_cache[key] = ws
     return ws
+
+
+def clear_workspaces():
+    """Releases the cached workspaces (call after synchronizing the streams
+    that used them)."""
+    _ws_cache.clear()
 
 
 def _stream_handle(stream, device):
