@@ -29,6 +29,21 @@ import numpy as np
 
 from . import conv_silu, fwd
 
+# Test-only switch: plants one named mistake in block_fwd so that the tests
+# can check that the pins catch it.  None (the default) runs the block as
+# written above.
+MUTATIONS = ("swap_xz", "gate_from_x", "conv_reversed", "dt_bias_ignored", "swap_BC", "no_D",
+             "out_proj_T", "select_from_x", "no_softplus")
+_mutation = None
+
+
+def set_mutation(name):
+    """Plant mistake `name` (one of MUTATIONS) in block_fwd; None clears it."""
+    global _mutation
+    if name is not None and name not in MUTATIONS:
+        raise ValueError(name)
+    _mutation = name
+
 
 def round_bf16(a):
     """float64 -> nearest bf16 value (ties to even), returned as float64."""
@@ -51,15 +66,28 @@ def block_fwd(hidden, w, store_bf16=True, precision="f64"):
     [d_inner, d_state], D [d_inner], out_proj [d_model, d_inner]).  Returns
     out [b, L, d_model] in float64."""
     r = round_bf16 if store_bf16 else (lambda a: a)
+    mut = _mutation
     h = np.asarray(hidden, dtype=np.float64)
     g = {k: (None if v is None else np.asarray(v, dtype=np.float64)) for k, v in w.items()}
+    if mut == "swap_xz":
+        g["in_proj_x"], g["in_proj_z"] = g["in_proj_z"], g["in_proj_x"]
+    if mut == "conv_reversed":
+        g["conv_w"] = g["conv_w"][:, ::-1]
+    if mut == "swap_BC":
+        g["x_proj_B"], g["x_proj_C"] = g["x_proj_C"], g["x_proj_B"]
+    if mut == "out_proj_T":
+        g["out_proj"] = g["out_proj"].T
     x = r(h @ g["in_proj_x"].T)
     z = r(h @ g["in_proj_z"].T)
     u = r(conv_silu(x, g["conv_w"], g["conv_b"]))
-    dt_low = r(u @ g["x_proj_dt"].T)
-    B = r(u @ g["x_proj_B"].T)
-    C = r(u @ g["x_proj_C"].T)
+    src = x if mut == "select_from_x" else u
+    dt_low = r(src @ g["x_proj_dt"].T)
+    B = r(src @ g["x_proj_B"].T)
+    C = r(src @ g["x_proj_C"].T)
     delta = r(dt_low @ g["dt_proj"].T)
-    y, _ = fwd(u, delta, g["A"], B, C, D=g["D"], z=z, delta_bias=g["dt_bias"], precision=precision)
+    y, _ = fwd(u, delta, g["A"], B, C, D=None if mut == "no_D" else g["D"],
+               z=x if mut == "gate_from_x" else z,
+               delta_bias=None if mut == "dt_bias_ignored" else g["dt_bias"],
+               softplus=mut != "no_softplus", precision=precision)
     y = r(y)
     return r(y @ g["out_proj"].T)

@@ -188,7 +188,7 @@ def test_config_mamba130m_full():
     assert ey <= 2e-2 and es <= 2e-2
 
 
-@pytest.mark.parametrize("name,count", [("mamba2p8b", 64), ("million", 24)])
+@pytest.mark.parametrize("name,count", [("mamba2p8b", 64), ("million", 64)])
 def test_config_sampled(name, count):
     c, inp = cfg_inputs(name)
     y, st = run(inp, sync_check=True)

@@ -92,7 +92,7 @@ def test_config_decode_1000_steps():
     base = step_inputs(c.batch, c.d_inner, c.d_state, c.dtype, c.seed, DEV, gate=c.gate)
     seq = step_sequence_inputs(c.steps, c.batch, c.d_inner, c.d_state, c.dtype, c.seed + 1, DEV,
                                gate=c.gate)
-    samples = sample_channels(c.batch, c.d_inner, 48, c.seed)
+    samples = sample_channels(c.batch, c.d_inner, 64, c.seed)
     bidx = sorted(set(b for b, _ in samples))
     state0 = base["state"].clone()
     y_hist = {}
