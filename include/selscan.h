@@ -296,8 +296,13 @@ SS_API size_t ss_ssd_fwd_workspace_bytes(const ss_ssd_dims* dims, uint32_t flags
  * bytes (forward-state checkpoints every 32 steps), 16-byte aligned, else
  * SS_ERR_WORKSPACE.  The sums over channels, batch and time use float
  * atomic adds, so the last bits of dA, dB, dC, dD and ddelta_bias depend on
- * the order the hardware applies them in.  One CTA scans a (batch, 64
- * channel) block over the whole sequence; there is no time chunking.
+ * the order the hardware applies them in.  The sequence is cut into time
+ * chunks (launch->chunk_len > 0 fixes their length; 0 lets the library
+ * choose), scanned in three launches: a chunk pass (each chunk's forward
+ * from zero, with state checkpoints every 32 steps, and for every chunk but
+ * the last the adjoint-only recurrence from zero), a fold of the chunk
+ * records into each chunk's exact entering forward state and adjoint, and
+ * the gradient pass over (batch, 64-channel block, chunk) items.
  * Errors: as ss_fwd (SS_ERR_INVALID_ARG for a NULL required pointer, a
  * misaligned pointer or dz/z mismatch). */
 SS_API int ss_bwd(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
@@ -337,7 +342,11 @@ SS_API int ss_fwd_with_state(const void* u, const void* delta, const float* delt
  * created on the first call of each host thread on each device and kept.
  * The call is asynchronous on launch->stream: y and last_state are complete
  * once launch->stream has been synchronized (SS_SYNC_CHECK does it and
- * returns the device status).  Errors: as ss_fwd. */
+ * returns the device status).  The workspace starts with one status word
+ * shared by all slices: a device-side failure in any slice stays recorded
+ * there, so ss_check(launch) after the call (or SS_SYNC_CHECK) reports it.
+ * SS_TEST_DROP_CARRY applies to the caller's batch entry 0 (the first
+ * slice) only.  Errors: as ss_fwd. */
 SS_API int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
                        const void* C, const float* D, const void* z, void* y, float* last_state, uint32_t flags,
                        const ss_dims* dims, const ss_launch* launch, int32_t rows_per_slice);
@@ -399,7 +408,10 @@ SS_API int ss_version(void);
  *   streams, other host threads) race on it and give wrong results: order
  *   them on one stream.
  * - Pass SS_SYNC_CHECK in flags to synchronize and get the device status;
- *   ss_check cannot be used (the array is not exposed).
+ *   ss_check cannot be used (the array is not exposed).  Without
+ *   SS_SYNC_CHECK a device-side failure (a bounded cross-chunk wait that ran
+ *   out: SS_ERR_TIMEOUT, its outputs invalid) is not reported to the caller
+ *   at all, so callers that cannot afford the synchronization accept that.
  * Returns the same codes as ss_fwd. */
 SS_API int ss_fwd_noalloc(const void* u, const void* delta, const float* delta_bias, const float* A,
                           const void* B, const void* C, const float* D, const void* z, void* y,

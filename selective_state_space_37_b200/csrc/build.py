@@ -41,8 +41,9 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()) -> str:
-    """Compile the library to `out`; `defines` are extra -D tuning macros
-    (SELSCAN_CTAS_PER_SM, SELSCAN_GROUP, SELSCAN_UNROLL_TILE)."""
+    """Compile the library to `out`; `defines` are extra -D preprocessor
+    definitions passed to nvcc (e.g. for a differently configured copy built
+    next to the in-tree one and loaded through SELSCAN_LIB)."""
     if not force and out == LIB and not defines and up_to_date():
         return out
     cmd = [NVCC, *NVCC_FLAGS] + [f"-D{d}" for d in defines]

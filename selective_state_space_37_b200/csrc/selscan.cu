@@ -521,10 +521,12 @@ int ss_check(const ss_launch* launch) {
 
 // ss_fwd and ss_fwd_conv (conv_w non-null: u is computed from x = `u` by the
 // causal conv1d + SiLU prologue).
+// keep_status: leave the status word (header word 0) as it is, so that one
+// word collects the failures of several calls (ss_fwd_host's slices).
 static int fwd_impl(const void* u, const void* delta, const float* delta_bias, const float* A, const void* B,
                     const void* C, const float* D, const void* z, void* y, float* last_state, const float* conv_w,
                     const float* conv_b, uint32_t flags, const ss_dims* dims, const ss_launch* launch,
-                    const float* h_init = nullptr) {
+                    const float* h_init = nullptr, bool keep_status = false) {
     const bool conv = conv_w != nullptr;
     int rc = validate_dims(dims, true);
     if (rc != SS_OK) return rc;
@@ -553,7 +555,9 @@ static int fwd_impl(const void* u, const void* delta, const float* delta_bias, c
     if (items >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
 
     unsigned char* ws = static_cast<unsigned char*>(launch->workspace);
-    if (cudaMemsetAsync(ws, 0, pl.status_off + pl.status_bytes, stream) != cudaSuccess) return SS_ERR_CUDA;
+    const size_t keep = keep_status ? sizeof(uint32_t) : 0;
+    if (cudaMemsetAsync(ws + keep, 0, pl.status_off + pl.status_bytes - keep, stream) != cudaSuccess)
+        return SS_ERR_CUDA;
 
     FwdParams p{};
     p.u = u; p.delta = delta; p.bias = delta_bias; p.A = A; p.B = B; p.C = C; p.D = D; p.z = z;
@@ -599,9 +603,10 @@ int ss_fwd(const void* u, const void* delta, const float* delta_bias, const floa
 }
 
 // ------------------------------------------------------------- host-buffer forward
-// Staging of ss_fwd_host: two slots, each holding one batch slice's u, Δraw,
-// z, y [rows, L, d], B, C [rows, L, 16] and last_state [rows, d, 16], then
-// the forward workspace for one slice; every region 256-byte aligned.
+// Staging of ss_fwd_host: the forward workspace of one slice first (its
+// header word 0 is the call's status word), then two slots, each holding one
+// batch slice's u, Δraw, z, y [rows, L, d], B, C [rows, L, 16] and
+// last_state [rows, d, 16]; every region 256-byte aligned.
 struct HostPlan {
     size_t act, bc, st, slot, ws_off, ws, total;
     int64_t rows;
@@ -618,9 +623,9 @@ static HostPlan host_plan(const ss_dims* dims, uint32_t flags, int32_t rows_per_
     h.slot = 4 * h.act + 2 * h.bc + h.st;
     ss_dims sd = *dims;
     sd.batch = h.rows;
-    h.ws_off = 2 * h.slot;
     h.ws = al(ss_fwd_workspace_bytes(&sd, flags, 0));
-    h.total = h.ws_off + h.ws;
+    h.ws_off = h.ws;   // the slots follow the forward workspace
+    h.total = h.ws + 2 * h.slot;
     return h;
 }
 
@@ -681,10 +686,12 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
     if (!hp) return SS_ERR_CUDA;
     const size_t es = (flags & SS_BF16) ? 2 : 4;
     unsigned char* base = static_cast<unsigned char*>(launch->workspace);
-    ss_launch sl = *launch;   // the slices' forward: workspace after the two slots
-    sl.workspace = base + h.ws_off;
+    ss_launch sl = *launch;   // the slices' forward: workspace at the start, before the two slots
+    sl.workspace = base;
     sl.workspace_bytes = h.ws;
     const uint32_t fflags = flags & ~static_cast<uint32_t>(SS_SYNC_CHECK);
+    // one status word for the whole call: cleared once here, kept by every slice
+    if (cudaMemsetAsync(base, 0, sizeof(uint32_t), cs) != cudaSuccess) return SS_ERR_CUDA;
     auto ok = [](cudaError_t e) { return e == cudaSuccess; };
     // On an error after copies were queued, let them finish before returning:
     // they read and write the caller's host buffers.
@@ -701,7 +708,7 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
     for (int64_t s = 0; s < nslices; ++s) {
         const int slot = static_cast<int>(s & 1);
         const int64_t r0 = s * h.rows, nr = std::min(h.rows, batch - r0);
-        unsigned char* sp = base + slot * h.slot;
+        unsigned char* sp = base + h.ws_off + slot * h.slot;
         void* su = sp;
         void* sd = sp + h.act;
         void* sz = sp + 2 * h.act;
@@ -731,8 +738,10 @@ int ss_fwd_host(const void* u, const void* delta, const float* delta_bias, const
             return fail(SS_ERR_CUDA);
         ss_dims sdims = *dims;
         sdims.batch = nr;
+        // the test-only dropped carry belongs to the caller's batch entry 0: the first slice
+        const uint32_t sflags = s == 0 ? fflags : (fflags & ~static_cast<uint32_t>(SS_TEST_DROP_CARRY));
         rc = fwd_impl(su, sd, delta_bias, A, sB, sC, D, z ? sz : nullptr, sy, last_state ? sst : nullptr, nullptr,
-                      nullptr, fflags, &sdims, &sl);
+                      nullptr, sflags, &sdims, &sl, nullptr, /*keep_status=*/true);
         if (rc != SS_OK) return fail(rc);
         if (!ok(cudaEventRecord(hp->done[slot], cs))) return fail(SS_ERR_CUDA);
         // download

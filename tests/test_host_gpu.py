@@ -88,3 +88,33 @@ def test_host_zero_length_and_bad_workspace():
                               p(inp["D"]), p(h["z"]), p(y), None, ss.SS_BF16 | ss.SS_DELTA_SOFTPLUS,
                               ctypes.byref(dims), ctypes.byref(launch), 1)
     assert rc == ss.SS_ERR_WORKSPACE
+
+
+def test_host_failure_in_first_slice_stays_reported():
+    """A device-side failure in one slice stays in the call's status word: the
+    first slice's dropped carry (test-only flag, batch entry 0) makes its
+    bounded wait run out, the later slices scan normally without clearing the
+    word, and both SS_SYNC_CHECK and ss_check on the same launch report
+    SS_ERR_TIMEOUT; the next call on the same context is correct."""
+    b, L, d = 3, 512, 128
+    inp = fwd_inputs(b, L, d, 16, "bf16", 12, DEV, gate=True)
+    h = host_copy(inp)
+    dims = ss.ss_dims(b, L, d, 16)
+    flags = ss.SS_BF16 | ss.SS_DELTA_SOFTPLUS | ss.SS_SYNC_CHECK
+    assert int(ss.lib().ss_fwd_chunk_len(ctypes.byref(ss.ss_dims(1, L, d, 16)), ss.SS_BF16)) > 0  # slices are chunked
+    need = int(ss.lib().ss_fwd_host_workspace_bytes(ctypes.byref(dims), flags, 1))
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    y = torch.empty_like(h["u"]).pin_memory()
+    stream = torch.cuda.current_stream().cuda_stream
+    launch = ss.ss_launch(stream, ws.data_ptr(), need, 2000, 0)
+    p = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    rc = ss.lib().ss_fwd_host(p(h["u"]), p(h["delta"]), p(inp["delta_bias"]), p(inp["A"]), p(h["B"]), p(h["C"]),
+                              p(inp["D"]), p(h["z"]), p(y), None, flags | ss.SS_TEST_DROP_CARRY,
+                              ctypes.byref(dims), ctypes.byref(launch), 1)
+    assert rc == ss.SS_ERR_TIMEOUT
+    assert ss.lib().ss_check(ctypes.byref(launch)) == ss.SS_ERR_TIMEOUT
+    rc = ss.lib().ss_fwd_host(p(h["u"]), p(h["delta"]), p(inp["delta_bias"]), p(inp["A"]), p(h["B"]), p(h["C"]),
+                              p(inp["D"]), p(h["z"]), p(y), None, flags, ctypes.byref(dims), ctypes.byref(launch), 1)
+    assert rc == ss.SS_OK
+    y_ref, _ = device_slices(inp, 1)
+    assert torch.equal(y, y_ref)

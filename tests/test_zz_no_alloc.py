@@ -7,7 +7,7 @@ Checked through the C ABI against ss_fwd (the entry point with a caller
 workspace) on the same inputs, within the bf16 parity bound the other tests
 use, on two calls in a row (the shared array keeps the previous call's
 contents, so the second call also checks that what must start at zero is
-reset).  This file is collected last; it passes alone in a fresh process and
+reset), and against the CPU oracle as well.  This file is collected last; it passes alone in a fresh process and
 after the other tests.
 """
 import ctypes
@@ -16,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import selective_state_space_37_b200 as ss
 from selective_state_space_37_b200 import _binding as bd
 from ss_inputs import fwd_inputs, to_f64
@@ -47,6 +48,9 @@ def test_noalloc_matches_workspace_entry_point_twice():
     dims = bd.ss_dims(batch, L, d, 16)
     flags = bd.SS_BF16 | bd.SS_DELTA_SOFTPLUS | bd.SS_SYNC_CHECK
     stream = torch.cuda.current_stream(DEV).cuda_stream
+    yo, so = oracle.fwd(to_f64(inp["u"]), to_f64(inp["delta"]), to_f64(inp["A"]), to_f64(inp["B"]),
+                        to_f64(inp["C"]), D=to_f64(inp["D"]), z=to_f64(inp["z"]),
+                        delta_bias=to_f64(inp["delta_bias"]), precision="f32")
     for _ in range(2):
         y = torch.full_like(y_ref, float("nan"))
         st = torch.full_like(st_ref, float("nan"))
@@ -54,6 +58,8 @@ def test_noalloc_matches_workspace_entry_point_twice():
         assert rc == ss.SS_OK, ss.status_string(rc)
         assert _rel(y, y_ref) <= TOL
         assert _rel(st, st_ref) <= TOL
+        assert float(np.max(np.abs(to_f64(y) - yo)) / np.max(np.abs(yo))) <= TOL
+        assert float(np.max(np.abs(to_f64(st) - so)) / np.max(np.abs(so))) <= TOL
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
