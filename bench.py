@@ -757,8 +757,10 @@ def run_ours(args):
             extras[name] = {"ms_per_step": sms, "TFLOP_s": tf, "frac_of_bf16_peak": tf / bf16_peak,
                             "GB_s": gbs, "frac_of_hbm": gbs / hbm,
                             "shape": {"batch": b, "seq_len": L, "nheads": H, "headdim": 64, "d_state": N},
-                            "note": "ss_ssd_fwd: chunked matrix form on mma.sync bf16 tensor-core "
-                                    "instructions; TFLOP_s counts the causal-half products"}
+                            "note": "ss_ssd_fwd: chunked matrix form, d_state 128 on tcgen05.mma (TMEM "
+                                    "accumulators, TMA SWIZZLE_128B tiles, 128-step chunks); TFLOP_s "
+                                    "counts the causal-half products of 64-step chunks, a fixed "
+                                    "definition independent of the kernel's chunk"}
         for name in BLOCK_SHAPES:
             kms, toks, flops = time_block(ss, torch, name, device, 10, 3)
             extras[name] = {"ms_per_step": kms, "tokens_per_s": toks / (kms * 1e-3),

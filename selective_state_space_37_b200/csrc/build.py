@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(os.path.dirname(HERE))
 LIB = os.path.join(HERE, "libselscan.so")
 SOURCES = ["selscan.cu"]
-HEADERS = ["common.cuh", "cp_async.cuh", "fwd.cuh", "bwd.cuh", "step.cuh", "block.cuh", "ssd.cuh"]
+HEADERS = ["common.cuh", "cp_async.cuh", "fwd.cuh", "ssd_tc.cuh", "bwd.cuh", "step.cuh", "block.cuh", "ssd.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 NVCC_FLAGS = [

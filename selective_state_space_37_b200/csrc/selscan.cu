@@ -16,6 +16,7 @@
 #include "bwd.cuh"
 #include "fwd.cuh"
 #include "ssd.cuh"
+#include "ssd_tc.cuh"
 #include "step.cuh"
 
 using namespace selscan;
@@ -208,9 +209,11 @@ int launch_variant(bool bf16, bool tma, Variant v, const FwdParams& p, int64_t i
                : launch_fwd<float, false, 1, 1, 8, false, CONV>(p, items, maps, stream);
 }
 
-// SSD time segments: workspace for up to kSsdMaxSeg segments per sequence --
-// the segment end-state records [batch, H, kmax - 1, P, N] fp32, then Σ Δ A
-// per segment [batch, H, kmax]; each region 256-byte aligned.
+// SSD workspace: a 256-byte header (word 0: the device status word), then,
+// for up to kSsdMaxSeg time segments per sequence, the segment end-state
+// records [batch, H, kmax - 1, P, N] fp32 and Σ Δ A per segment
+// [batch, H, kmax]; each region 256-byte aligned.  kmax counts 64-step
+// chunks, so it also covers the tensor-core kernel's 128-step chunks.
 constexpr int64_t kSsdMaxSeg = 8;
 struct SsdLayout {
     size_t rec, esum, total;
@@ -222,10 +225,101 @@ SsdLayout ssd_layout(const ss_ssd_dims* d) {
     w.nchunks = ceil_div(std::max<int64_t>(d->seqlen, 1), kSsdQ);
     w.kmax = std::min(kSsdMaxSeg, w.nchunks);
     const int64_t bh = d->batch * d->nheads;
-    w.rec = 0;
-    w.esum = al(static_cast<size_t>(bh * (w.kmax - 1) * kSsdP * d->d_state) * sizeof(float));
+    w.rec = kHeaderBytes;
+    w.esum = w.rec + al(static_cast<size_t>(bh * (w.kmax - 1) * kSsdP * d->d_state) * sizeof(float));
     w.total = w.esum + al(static_cast<size_t>(bh * w.kmax) * sizeof(float));
     return w;
+}
+
+// SELSCAN_SSD_MMA_SYNC=1 builds the d_state 128 scan on the warp-level
+// mma.sync kernel of ssd.cuh instead of the tcgen05 one (comparisons).
+#ifndef SELSCAN_SSD_MMA_SYNC
+#define SELSCAN_SSD_MMA_SYNC 0
+#endif
+
+// Tensor map of a row-major tensor of `rank` dimensions (innermost first,
+// byte strides of dimensions 1..rank-1), bf16, 128-byte swizzle, box `box`.
+bool make_map_sw128(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
+                    const cuuint32_t* box) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank), const_cast<void*>(base),
+                           dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// The tcgen05 scan (d_state 128): segments of whole 128-step chunks chosen
+// like launch_ssd's (one resident CTA per SM; state pass charged half a
+// chunk, splitting 10 %), then the state pass, the fold and the main pass.
+int launch_ssd_tc(const tc::Params& base_p, const SsdParams& fold_p, const void* x, const void* B, const void* C,
+                  int64_t items, const SsdLayout& w, int32_t chunk_len, bool have_ws, cudaStream_t stream) {
+    tc::Params p = base_p;
+    const int64_t L = p.L;
+    const int64_t nchunks = ceil_div(std::max<int64_t>(L, 1), tc::kQ);
+    const int64_t kmax = std::min<int64_t>(w.kmax, nchunks);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return SS_ERR_CUDA;
+    auto kmain = tc::ss_ssd_tc_kernel<false>;
+    auto kstate = tc::ss_ssd_tc_kernel<true>;
+    static std::atomic<bool> attr_main[kMaxDevices];
+    static std::atomic<bool> attr_state[kMaxDevices];
+    if (set_smem_limit(kmain, tc::kSmemBytes, attr_main, dev) != SS_OK ||
+        set_smem_limit(kstate, tc::kSmemBytes, attr_state, dev) != SS_OK)
+        return SS_ERR_CUDA;
+    int nseg = 1, cseg = static_cast<int>(nchunks);
+    if (have_ws) {
+        const int64_t slots = sm_count_of_current_device();
+        if (chunk_len > 0) {
+            int64_t cs = std::max<int64_t>(1, ceil_div(chunk_len, tc::kQ));
+            if (ceil_div(nchunks, cs) > kmax) cs = ceil_div(nchunks, kmax);
+            cseg = static_cast<int>(cs);
+            nseg = static_cast<int>(ceil_div(nchunks, cs));
+        } else {
+            double best = 0.0;
+            for (int64_t k = 1; k <= kmax; ++k) {
+                const int64_t cs = ceil_div(nchunks, k);
+                if (ceil_div(nchunks, cs) != k) continue;
+                double cost = static_cast<double>(ceil_div(items * k, slots) * cs);
+                if (k > 1) cost = 1.1 * (cost + 0.5 * static_cast<double>(ceil_div(items * (k - 1), slots) * cs));
+                if (k == 1 || cost < best - 1e-9) {
+                    best = cost;
+                    nseg = static_cast<int>(k);
+                    cseg = static_cast<int>(cs);
+                }
+            }
+        }
+    }
+    p.nseg = nseg;
+    p.cseg = cseg;
+    if (items * nseg >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    const int64_t H = p.H, batch = p.batch;
+    CUtensorMap mx, mb, mc;
+    {
+        const cuuint64_t dx[4] = {static_cast<cuuint64_t>(tc::kP), static_cast<cuuint64_t>(H),
+                                  static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(batch)};
+        const cuuint64_t sx[3] = {static_cast<cuuint64_t>(tc::kP * 2), static_cast<cuuint64_t>(H * tc::kP * 2),
+                                  static_cast<cuuint64_t>(L * H * tc::kP * 2)};
+        const cuuint32_t bx[4] = {64, 1, static_cast<cuuint32_t>(tc::kQ), 1};
+        const cuuint64_t db[3] = {static_cast<cuuint64_t>(tc::kN), static_cast<cuuint64_t>(L),
+                                  static_cast<cuuint64_t>(batch)};
+        const cuuint64_t sb[2] = {static_cast<cuuint64_t>(tc::kN * 2), static_cast<cuuint64_t>(L * tc::kN * 2)};
+        const cuuint32_t bb[3] = {64, static_cast<cuuint32_t>(tc::kQ), 1};
+        if (!make_map_sw128(&mx, x, 4, dx, sx, bx) || !make_map_sw128(&mb, B, 3, db, sb, bb) ||
+            !make_map_sw128(&mc, C, 3, db, sb, bb))
+            return SS_ERR_CUDA;
+    }
+    if (nseg > 1) {
+        kstate<<<static_cast<unsigned>(items * (nseg - 1)), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc);
+        SsdParams f = fold_p;
+        f.nseg = nseg;
+        const int64_t total = items * kSsdP * tc::kN;
+        const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), 4096);
+        ss_ssd_fold_kernel<tc::kN><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(f);
+    }
+    kmain<<<static_cast<unsigned>(items * nseg), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc);
+    return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
 // Segments for `items` (batch x heads) sequences of nchunks chunks on `slots`
@@ -943,6 +1037,8 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
     const bool have_ws = launch->workspace != nullptr;
     if (have_ws && (launch->workspace_bytes < w.total || !aligned16(launch->workspace))) return SS_ERR_WORKSPACE;
     cudaStream_t stream = static_cast<cudaStream_t>(launch->stream);
+    if (have_ws && cudaMemsetAsync(launch->workspace, 0, sizeof(uint32_t), stream) != cudaSuccess)
+        return SS_ERR_CUDA;
     SsdParams p{};
     p.x = static_cast<const __nv_bfloat16*>(x);
     p.dt = static_cast<const __nv_bfloat16*>(dt);
@@ -960,10 +1056,30 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
     p.L = L; p.batch = static_cast<int>(batch); p.H = static_cast<int>(H);
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
     const int64_t items = batch * H;
-    const int rc = dims->d_state == 128 ? launch_ssd<128>(p, items, w, launch->chunk_len, have_ws, stream)
-                                        : launch_ssd<64>(p, items, w, launch->chunk_len, have_ws, stream);
+    int rc;
+    if (dims->d_state == 128 && !SELSCAN_SSD_MMA_SYNC) {
+        if (L == 0) {   // no steps: the final state is zero
+            if (final_state &&
+                cudaMemsetAsync(final_state, 0, static_cast<size_t>(items * kSsdP * 128) * sizeof(float), stream) !=
+                    cudaSuccess)
+                return SS_ERR_CUDA;
+            rc = SS_OK;
+        } else {
+            tc::Params q{};
+            q.dt = p.dt; q.dt_bias = p.dt_bias; q.A = p.A; q.D = p.D; q.y = p.y; q.final_state = p.final_state;
+            q.rec = p.rec; q.esum = p.esum;
+            q.status = have_ws ? static_cast<uint32_t*>(launch->workspace) : nullptr;
+            q.L = L; q.batch = p.batch; q.H = p.H; q.softplus = p.softplus;
+            q.wait_ns = kTmaWaitNs;
+            rc = launch_ssd_tc(q, p, x, B, C, items, w, launch->chunk_len, have_ws, stream);
+        }
+    } else {
+        rc = dims->d_state == 128 ? launch_ssd<128>(p, items, w, launch->chunk_len, have_ws, stream)
+                                  : launch_ssd<64>(p, items, w, launch->chunk_len, have_ws, stream);
+    }
     if (rc != SS_OK) return rc;
     if (flags & SS_SYNC_CHECK) {
+        if (have_ws) return ss_check(launch);
         if (cudaStreamSynchronize(stream) != cudaSuccess) return SS_ERR_CUDA;
     }
     return SS_OK;

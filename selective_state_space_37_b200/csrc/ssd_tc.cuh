@@ -1,0 +1,545 @@
+// ssd_tc.cuh -- the multi-head scalar-decay scan (Mamba-2's SSD model) on the
+// fifth-generation tensor cores of sm_100a: tcgen05.mma with its accumulators
+// in tensor memory (TMEM), operand tiles staged by TMA in the 128-byte
+// swizzled shared-memory layout the MMA descriptors read.
+//
+// Per (batch b, head h), with the head's P = 64 channels sharing Δ, B, C (the
+// mamba README's Mamba-2 section; the model-architecture page's "Mamba-2
+// (multi-head, larger state)", headdim 64, ngroups 1):
+//   Δ_t = softplus(dt_t + dt_bias),  H_t = exp(Δ_t A) H_{t-1} + Δ_t x_t B_tᵀ,
+//   y_t = H_t C_t + D x_t           (H_t is P x N, x_t ∈ R^P, B_t, C_t ∈ R^N).
+// Over a chunk of Q = 128 steps with cum_t = Σ_{r<=t} Δ_r A (the recurrence
+// has one scalar decay per step, so a chunk is a set of dense products):
+//   Y = (C Bᵀ ∘ M) X + diag(e^{cum}) (C Gᵀ),   M[t,s] = e^{cum_t - cum_s} Δ_s (s <= t)
+//   G ← e^{cum_end} G + (Bᵀ X̃)ᵀ,                X̃[s,:] = e^{cum_end - cum_s} Δ_s x_s
+// with G the P x N state entering the chunk.
+//
+// One CTA (8 warps) walks the chunks of one (b, h) in order.  Thread 0 issues
+// the MMAs (bf16 operands, fp32 accumulation, M = 128):
+//   S   = C Bᵀ          128 x 128, K = N     -> TMEM columns [0, 128)
+//   CG  = C (G_hi + G_lo)ᵀ 128 x 64, K = N   -> TMEM columns [192, 256)
+//   Y   = Mm X          128 x 64,  K = Q     -> TMEM columns [128, 192)
+//   ΔGᵀ = Bᵀ X̃          128 x 64,  K = Q     -> TMEM columns [256, 320)
+// and the eight warps do the elementwise work between them, two threads per
+// TMEM lane (one time step t, or one state index n), each on half of the
+// lane's columns: the causal decay mask Mm from S, X̃ from x, the outputs
+// y = Y + e^{cum_t} CG + D x, and the state update.  The carried state G
+// stays fp32 in registers (the two threads of row n hold G[:, n]); the
+// product with C reads it as two bf16 terms G_hi + G_lo, so it is not
+// rounded to bf16 before the readout.  x, B, C tiles arrive by TMA
+// (x double-buffered and fetched a chunk ahead, C reloaded as soon as its
+// last MMA is done, B likewise), each tensor on its own mbarrier; the MMAs
+// of C Bᵀ and of C Gᵀ complete on separate mbarriers so the mask can start
+// while C Gᵀ still runs.  Every wait (TMA and MMA completions) is bounded.
+//
+// Time segments: when batch x heads leaves SMs idle, each sequence is cut into
+// segments of whole chunks with an exact carry (state pass from G = 0 keeping
+// only G_out and Σ Δ A, the fold of ssd.cuh, then the main pass from each
+// segment's entering state).
+#pragma once
+
+#include "common.cuh"
+#include "ssd.cuh"
+
+namespace selscan {
+namespace tc {
+
+constexpr int kQ = 128;            // chunk length (MMA M for the time rows)
+constexpr int kP = 64;             // head dimension
+constexpr int kN = 128;            // state width handled here
+constexpr int kRows = 128;         // TMEM lanes / tile rows
+constexpr int kThreads = 256;      // two threads per row: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
+constexpr uint32_t kTmemCols = 512;   // allocation (power of two >= the 320 columns used)
+constexpr uint32_t kColS = 0, kColY = 128, kColCG = 192, kColG = 256;
+
+// Instruction descriptors (kind::f16, bf16 x bf16 -> fp32, M = 128): bit 4 D
+// format f32, bits 7/10 A/B format bf16, bit 15/16 A/B major (1: MN-major),
+// bits 17.. N >> 3, bits 24.. M >> 4.
+constexpr uint32_t kIdesc_128x128_KK = (1u << 4) | (1u << 7) | (1u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdesc_128x64_KMN = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((64u >> 3) << 17) |
+                                       ((128u >> 4) << 24);
+constexpr uint32_t kIdesc_128x64_MNMN = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                        ((64u >> 3) << 17) | ((128u >> 4) << 24);
+
+// Shared memory, byte offsets from a 1024-aligned base.  Every operand tile
+// is a set of [rows][64 bf16] blocks of 128-byte rows in the 128-byte
+// swizzle (16-byte chunk c of row r stored at chunk c ^ (r & 7)).
+constexpr uint32_t kOffX0 = 0;            // x [t][p], two buffers
+constexpr uint32_t kOffX1 = 16384;
+constexpr uint32_t kOffXt = 32768;        // X̃ [s][p]
+constexpr uint32_t kOffB = 49152;         // B [s][n]: blocks n 0..63, 64..127
+constexpr uint32_t kOffC = 81920;         // C [t][n]: blocks n 0..63, 64..127
+constexpr uint32_t kOffM = 114688;        // Mm [t][s]: blocks s 0..63, 64..127
+constexpr uint32_t kOffGh = 147456;       // G_hi [n][p]
+constexpr uint32_t kOffGl = 163840;       // G_lo [n][p]
+constexpr uint32_t kOffCum = 180224;      // cum[128] f32
+constexpr uint32_t kOffCs = kOffCum + 512;    // cum · log2 e
+constexpr uint32_t kOffDlt = kOffCs + 512;    // Δ
+constexpr uint32_t kOffBar = kOffDlt + 512;   // 7 mbarriers (8 B each), then the TMEM base address
+constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;  // + alignment slack
+
+struct Params {
+    const __nv_bfloat16* dt;   // [batch, L, H]
+    const float* dt_bias;      // [H] or null
+    const float* A;            // [H]
+    const float* D;            // [H] or null
+    __nv_bfloat16* y;          // [batch, L, H, P]
+    float* final_state;        // [batch, H, P, N] or null
+    float* rec;                // [batch, H, nseg - 1, P, N]
+    float* esum;               // [batch, H, nseg]
+    uint32_t* status;          // error word or null
+    int64_t L;
+    int batch, H, nseg, cseg;  // cseg: chunks of kQ steps per segment
+    int softplus;
+    uint64_t wait_ns;
+};
+
+// ------------------------------------------------------------ tcgen05 / TMA
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)),
+                 "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem desc] · B[smem desc]; issued by one thread.
+__device__ __forceinline__ void umma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    const uint32_t z = 0;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}"
+        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc), "r"(z), "r"(z), "r"(z), "r"(z)
+        : "memory");
+}
+// Arrive (once) on `bar` when every MMA this thread issued so far is done.
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes 32w..32w+31).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Shared-memory matrix descriptor: 128-byte swizzle, start / leading / stride
+// byte offsets in 16-byte units, descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm, int x, int y, int z, int w,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_u(uint32_t dst, const CUtensorMap* tm, int x, int y, int z,
+                                              uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// bf16 pair from two floats (round to nearest even), and back.
+__device__ __forceinline__ uint32_t pk(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+__device__ __forceinline__ float lo_f(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float hi_f(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Address of logical 16-byte chunk c (0..7) of row r of a swizzled block.
+__device__ __forceinline__ uint32_t chunk_addr(uint32_t block, int r, int c) {
+    return block + static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>(c ^ (r & 7)) << 4);
+}
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+// Grid: one CTA per (segment k, batch b, head h), blockIdx.x = (k * batch + b) * H + h;
+// STATE runs segments 0 .. nseg - 2 only (G_out from zero, no outputs).
+template <bool STATE>
+__global__ void __launch_bounds__(kThreads, 1)
+ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
+                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;   // 1024-aligned: the swizzle pattern is address based
+    unsigned char* gbase = smem_raw + (base - raw);
+    float* cum = reinterpret_cast<float*>(gbase + kOffCum);
+    float* cs = reinterpret_cast<float*>(gbase + kOffCs);
+    float* dlt = reinterpret_cast<float*>(gbase + kOffDlt);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kOffBar);
+    uint64_t* x_bar = bars;        // [2]: x tile of buffer 0 / 1 landed
+    uint64_t* b_bar = bars + 2;    // B tile landed
+    uint64_t* c_bar = bars + 3;    // C tile landed
+    uint64_t* s_bar = bars + 4;    // C Bᵀ done
+    uint64_t* yg_bar = bars + 6;   // Mm X, Bᵀ X̃ and every earlier MMA done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 64);
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int row = tid & (kRows - 1);   // TMEM lane / tile row of this thread
+    const int hf = tid >> 7;             // which half of the row's columns
+    const int h = blockIdx.x % p.H;
+    const int b = (blockIdx.x / p.H) % p.batch;
+    const int sg = blockIdx.x / (p.H * p.batch);
+    const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+    const float Ah = p.A[h];
+    const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
+    const float Dh = p.D ? p.D[h] : 0.0f;
+    const int64_t seg_t0 = static_cast<int64_t>(sg) * p.cseg * kQ;
+    const int64_t seg_t1 = min(seg_t0 + static_cast<int64_t>(p.cseg) * kQ, p.L);
+    const int nchunk = static_cast<int>((seg_t1 - seg_t0 + kQ - 1) / kQ);
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;   // this warp's TMEM lanes
+
+    if (tid == 0) {
+        for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_x);
+        tma_prefetch_desc(&tm_B);
+        if (!STATE) tma_prefetch_desc(&tm_C);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    // TMA of chunk ci's tiles (thread 0): x into buffer ci & 1, B, C.
+    auto chunk_t0 = [&](int ci) { return static_cast<int>(seg_t0 + static_cast<int64_t>(ci) * kQ); };
+    auto issue_x = [&](int ci) {
+        uint64_t* bar = x_bar + (ci & 1);
+        mbar_arrive_expect_tx(bar, kQ * kP * 2);
+        tma_load_4d(base + ((ci & 1) ? kOffX1 : kOffX0), &tm_x, 0, h, chunk_t0(ci), b, bar);
+    };
+    auto issue_b = [&](int ci) {
+        mbar_arrive_expect_tx(b_bar, 2 * kQ * 64 * 2);
+        tma_load_3d_u(base + kOffB, &tm_B, 0, chunk_t0(ci), b, b_bar);
+        tma_load_3d_u(base + kOffB + 16384, &tm_B, 64, chunk_t0(ci), b, b_bar);
+    };
+    auto issue_c = [&](int ci) {
+        mbar_arrive_expect_tx(c_bar, 2 * kQ * 64 * 2);
+        tma_load_3d_u(base + kOffC, &tm_C, 0, chunk_t0(ci), b, c_bar);
+        tma_load_3d_u(base + kOffC + 16384, &tm_C, 64, chunk_t0(ci), b, c_bar);
+    };
+    if (tid == 0 && nchunk > 0) {
+        issue_x(0);
+        issue_b(0);
+        if (!STATE) issue_c(0);
+    }
+
+    // Carried state: thread (n, hf) holds G[32 hf .. 32 hf + 31, n] (fp32).
+    // Entering a segment > 0 of the main pass it is the folded record, else zero.
+    float G[kP / 2];
+    const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kP * kN : nullptr;
+#pragma unroll
+    for (int q = 0; q < kP / 2; ++q) G[q] = gin ? gin[(32 * hf + q) * kN + row] : 0.0f;
+    auto store_g = [&]() {   // bf16 hi / lo copies of G: row n, chunks 4 hf .. 4 hf + 3 of the [n][p] tiles
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float g0 = G[8 * c + 2 * e], g1 = G[8 * c + 2 * e + 1];
+                hw[e] = pk(g0, g1);
+                lw[e] = pk(g0 - lo_f(hw[e]), g1 - hi_f(hw[e]));
+            }
+            sts128(chunk_addr(base + kOffGh, row, 4 * hf + c), make_uint4(hw[0], hw[1], hw[2], hw[3]));
+            sts128(chunk_addr(base + kOffGl, row, 4 * hf + c), make_uint4(lw[0], lw[1], lw[2], lw[3]));
+        }
+    };
+    if (!STATE && gin) {
+        store_g();
+        fence_proxy_async_smem();   // before the first MMA reads them (ordered by the first wait's barrier)
+    }
+    float esum = 0.0f;
+
+    // Δraw of the chunk's steps 4·lane .. 4·lane + 3 (warp 0)
+    float dtn[4] = {0.f, 0.f, 0.f, 0.f};
+    auto load_dt = [&](int ci) {
+        const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int64_t t = t0 + 4 * lane + e;
+            dtn[e] = t < p.L ? __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t) * p.H + h]) : 0.0f;
+        }
+    };
+    if (warp == 0 && nchunk > 0) load_dt(0);
+
+    bool ok = true;
+    // Tile copies issued and waited for, per tensor (the same counts on every
+    // thread): copies still in flight are drained before the shared memory is
+    // released after a failure.
+    const int first = nchunk > 0 ? 1 : 0;
+    int x_issued = first, x_waited = 0, b_issued = first, b_waited = 0, c_issued = STATE ? 0 : first, c_waited = 0;
+    auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
+        const bool got = mbar_wait_bounded(bar, parity, p.wait_ns);
+        const int bad = __syncthreads_or(got ? 0 : 1);
+        if (bad) {
+            ok = false;
+            if (tid == 0 && p.status) atomicCAS(p.status, 0u, static_cast<uint32_t>(-4));
+        }
+        return !bad;
+    };
+
+    for (int ci = 0; ci < nchunk && ok; ++ci) {
+        const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
+        const int q = static_cast<int>(p.L - t0 < kQ ? p.L - t0 : kQ);
+        const int xb = ci & 1;
+        const uint32_t xbase = base + (xb ? kOffX1 : kOffX0);
+        const bool carry = !STATE && (ci > 0 || sg > 0);
+        // the next chunk's x (its buffer was last read by chunk ci - 1, now done)
+        if (ci + 1 < nchunk) {
+            if (tid == 0) issue_x(ci + 1);
+            ++x_issued;
+        }
+        // Δ and the inclusive prefix of Δ A (warp 0: four steps per lane, one warp scan)
+        if (warp == 0) {
+            float dl[4], a[4], run = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                // softplus through the hardware ex2 / lg2: log1p(e^x) = ln 2 · log2(1 + 2^(x log2 e)),
+                // identity above x = 20 (well inside the bf16 outputs' precision)
+                const float xr = dtn[e] + bias;
+                const float spv = (xr > 20.0f) ? xr : kLn2 * lg2_approx(1.0f + ex2_approx(xr * kLog2e));
+                dl[e] = (4 * lane + e < q) ? (p.softplus ? spv : xr) : 0.0f;
+                run = fmaf(dl[e], Ah, run);
+                a[e] = run;
+            }
+            float sc = run;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, sc, o);
+                if (lane >= o) sc += v;
+            }
+            const float excl = sc - run;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                cum[4 * lane + e] = excl + a[e];
+                cs[4 * lane + e] = (excl + a[e]) * kLog2e;
+                dlt[4 * lane + e] = dl[e];
+            }
+            if (ci + 1 < nchunk) load_dt(ci + 1);
+        }
+        if (!wait_bar(x_bar + (ci & 1), static_cast<uint32_t>((ci >> 1) & 1))) break;   // also orders cum / dlt
+        ++x_waited;
+        if (!wait_bar(b_bar, static_cast<uint32_t>(ci & 1))) break;
+        ++b_waited;
+        if (!STATE) {
+            if (!wait_bar(c_bar, static_cast<uint32_t>(ci & 1))) break;
+            ++c_waited;
+        }
+        const float cum_end = cum[kQ - 1];
+        if (STATE) esum += cum_end;
+
+        // -------- S = C Bᵀ and CG = C (G_hi + G_lo)ᵀ (thread 0), X̃ (all threads)
+        if (!STATE && tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int k = 0; k < kN / 16; ++k) {
+                const uint32_t off = (k >> 2) * 16384u + (k & 3) * 32u;
+                umma(tmem + kColS, sdesc(base + kOffC + off, 16, 1024), sdesc(base + kOffB + off, 16, 1024),
+                     kIdesc_128x128_KK, k > 0);
+            }
+            umma_commit(s_bar);
+            if (carry) {
+#pragma unroll
+                for (int k = 0; k < kN / 16; ++k) {
+                    const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
+                    const uint64_t ad = sdesc(base + kOffC + aoff, 16, 1024);
+                    umma(tmem + kColCG, ad, sdesc(base + kOffGh + k * 2048u, 0, 1024), kIdesc_128x64_KMN, k > 0);
+                    umma(tmem + kColCG, ad, sdesc(base + kOffGl + k * 2048u, 0, 1024), kIdesc_128x64_KMN, 1);
+                }
+            }
+        }
+        {   // X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s; a per-row scale, so chunks keep their places)
+            const int s = row;
+            const float w = __expf(cum_end - cum[s]) * dlt[s];
+#pragma unroll
+            for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
+                const uint32_t a = xbase + static_cast<uint32_t>(s) * 128u + (c << 4);
+                const uint4 v = lds128(a);
+                const uint4 o = make_uint4(pk(lo_f(v.x) * w, hi_f(v.x) * w), pk(lo_f(v.y) * w, hi_f(v.y) * w),
+                                           pk(lo_f(v.z) * w, hi_f(v.z) * w), pk(lo_f(v.w) * w, hi_f(v.w) * w));
+                sts128(base + kOffXt + static_cast<uint32_t>(s) * 128u + (c << 4), o);
+            }
+        }
+        if (!STATE) {
+            // -------- Mm = S ∘ decay mask (row t, s-block hf), once S is in TMEM
+            if (!wait_bar(s_bar, static_cast<uint32_t>(ci & 1))) break;
+            tc_fence_after();
+            const int t = row;
+            const float ct = cs[t];
+#pragma unroll 1
+            for (int g = 2 * hf; g < 2 * hf + 2; ++g) {
+                const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
+                const int c0 = (g & 1) * 4;
+                if (32 * g > t) {   // above the diagonal: zeros
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) sts128(chunk_addr(blk, t, c0 + c), make_uint4(0, 0, 0, 0));
+                    continue;
+                }
+                float sv[32];
+                tmem_ld32(tmem + lane_base + kColS + 32 * g, sv);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t wv[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        float m2[2];
+#pragma unroll
+                        for (int f = 0; f < 2; ++f) {
+                            const int j = 8 * c + 2 * e + f;
+                            const int s = 32 * g + j;
+                            m2[f] = (s <= t) ? sv[j] * ex2_approx(ct - cs[s]) * dlt[s] : 0.0f;
+                        }
+                        wv[e] = pk(m2[0], m2[1]);
+                    }
+                    sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                }
+            }
+        }
+        fence_proxy_async_smem();   // Mm and X̃ (generic writes) before the MMAs read them
+        tc_fence_before();
+        __syncthreads();
+
+        // -------- Y = Mm X (main pass) and ΔGᵀ = Bᵀ X̃ (thread 0)
+        if (tid == 0) {
+            tc_fence_after();
+            if (!STATE) {
+#pragma unroll
+                for (int k = 0; k < kQ / 16; ++k) {
+                    const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
+                    umma(tmem + kColY, sdesc(base + kOffM + aoff, 16, 1024), sdesc(xbase + k * 2048u, 0, 1024),
+                         kIdesc_128x64_KMN, k > 0);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kQ / 16; ++k)
+                umma(tmem + kColG, sdesc(base + kOffB + k * 2048u, 16384, 1024),
+                     sdesc(base + kOffXt + k * 2048u, 0, 1024), kIdesc_128x64_MNMN, k > 0);
+            umma_commit(yg_bar);   // also covers C Gᵀ and C Bᵀ, issued before
+        }
+        if (!wait_bar(yg_bar, static_cast<uint32_t>(ci & 1))) break;
+        tc_fence_after();
+        // B and C are free: the next chunk's B and C
+        if (ci + 1 < nchunk) {
+            if (tid == 0) {
+                issue_b(ci + 1);
+                if (!STATE) issue_c(ci + 1);
+            }
+            ++b_issued;
+            if (!STATE) ++c_issued;
+        }
+
+        if (!STATE) {
+            // -------- y = Y + e^{cum_t} CG + D x (row t, columns 32 hf .. 32 hf + 31)
+            const int t = row;
+            const float et = __expf(cum[t]);
+            {
+                const int half = hf;
+                float yv[32], cg[32];
+                tmem_ld32(tmem + lane_base + kColY + 32 * half, yv);
+                if (carry) tmem_ld32(tmem + lane_base + kColCG + 32 * half, cg);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint4 xv = lds128(chunk_addr(xbase, t, 4 * half + c));
+                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    uint32_t ow[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 8 * c + 2 * e;
+                        float o0 = fmaf(Dh, lo_f(xw[e]), yv[j]);
+                        float o1 = fmaf(Dh, hi_f(xw[e]), yv[j + 1]);
+                        if (carry) {
+                            o0 = fmaf(et, cg[j], o0);
+                            o1 = fmaf(et, cg[j + 1], o1);
+                        }
+                        ow[e] = pk(o0, o1);
+                    }
+                    if (t < q) {
+                        __nv_bfloat16* yp = p.y + ((static_cast<int64_t>(b) * p.L + t0 + t) * p.H + h) * kP +
+                                            32 * half + 8 * c;
+                        *reinterpret_cast<uint4*>(yp) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+                    }
+                }
+            }
+        }
+        {   // -------- G = e^{cum_end} G + ΔGᵀ[n, :] (row n, columns 32 hf .. 32 hf + 31)
+            const float e_end = __expf(cum_end);
+            float dg[32];
+            tmem_ld32(tmem + lane_base + kColG + 32 * hf, dg);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) G[j] = fmaf(e_end, G[j], dg[j]);
+            if (!STATE) store_g();
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+    }
+
+    // outputs of the state: the segment's G_out (state pass) or the final state
+    if (ok) {
+        float* out = nullptr;
+        if (STATE) out = p.rec + (bh * (p.nseg - 1) + sg) * kP * kN;
+        else if (p.final_state && sg == p.nseg - 1) out = p.final_state + bh * kP * kN;
+        if (out) {
+#pragma unroll
+            for (int q2 = 0; q2 < kP / 2; ++q2) out[(32 * hf + q2) * kN + row] = G[q2];
+        }
+        if (STATE && tid == 0) p.esum[bh * p.nseg + sg] = esum;
+    }
+    // After a wait that ran out: let copies still in flight land before the
+    // shared memory is released (bounded as well; their phases are the next
+    // ones of each barrier, so a completed phase is recognised too).
+    if (!ok) {
+        for (int cj = x_waited; cj < x_issued; ++cj)   // chunk cj's x: buffer cj & 1, phase cj >> 1
+            mbar_wait_bounded(x_bar + (cj & 1), static_cast<uint32_t>((cj >> 1) & 1), p.wait_ns);
+        if (b_waited < b_issued) mbar_wait_bounded(b_bar, static_cast<uint32_t>(b_waited & 1), p.wait_ns);
+        if (c_waited < c_issued) mbar_wait_bounded(c_bar, static_cast<uint32_t>(c_waited & 1), p.wait_ns);
+    }
+    // every TMEM read and MMA is complete (waited above); release the columns
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+}  // namespace tc
+}  // namespace selscan

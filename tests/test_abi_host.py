@@ -169,8 +169,8 @@ def test_python_binding_checks_new_entry_points():
 
 def test_host_and_ssd_workspace_sizes(L):
     """ss_fwd_host's staging is two slots of one slice's activations and
-    states plus one slice's forward workspace; ss_ssd_fwd's workspace holds
-    segment records for min(8, chunks) segments."""
+    states plus one slice's forward workspace; ss_ssd_fwd's workspace is a
+    256-byte status header then segment records for min(8, chunks) segments."""
     al = lambda x: (x + 255) // 256 * 256
     dims = ss.ss_dims(3, 100, 64, 16)
     for rows in (1, 2, 3, 5):
@@ -182,7 +182,7 @@ def test_host_and_ssd_workspace_sizes(L):
     for b, Lq, H, N in ((2, 1000, 3, 128), (1, 64, 2, 64), (4, 8192, 80, 128)):
         chunks = max(1, -(-Lq // 64))
         k = min(8, chunks)
-        want = al(b * H * (k - 1) * 64 * N * 4) + al(b * H * k * 4)
+        want = 256 + al(b * H * (k - 1) * 64 * N * 4) + al(b * H * k * 4)
         got = L.ss_ssd_fwd_workspace_bytes(ctypes.byref(ss.ss_ssd_dims(b, Lq, H, 64, N)), 0)
         assert got == want, (b, Lq, H, N)
     assert L.ss_ssd_fwd_workspace_bytes(ctypes.byref(ss.ss_ssd_dims(1, 64, 2, 32, 64)), 0) == 0
