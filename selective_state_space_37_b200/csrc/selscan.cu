@@ -295,7 +295,7 @@ int launch_ssd_tc(const tc::Params& base_p, const SsdParams& fold_p, const void*
     p.cseg = cseg;
     if (items * nseg >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
     const int64_t H = p.H, batch = p.batch;
-    CUtensorMap mx, mb, mc;
+    CUtensorMap mx, mb, mc, my;
     {
         const cuuint64_t dx[4] = {static_cast<cuuint64_t>(tc::kP), static_cast<cuuint64_t>(H),
                                   static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(batch)};
@@ -307,18 +307,18 @@ int launch_ssd_tc(const tc::Params& base_p, const SsdParams& fold_p, const void*
         const cuuint64_t sb[2] = {static_cast<cuuint64_t>(tc::kN * 2), static_cast<cuuint64_t>(L * tc::kN * 2)};
         const cuuint32_t bb[3] = {64, static_cast<cuuint32_t>(tc::kQ), 1};
         if (!make_map_sw128(&mx, x, 4, dx, sx, bx) || !make_map_sw128(&mb, B, 3, db, sb, bb) ||
-            !make_map_sw128(&mc, C, 3, db, sb, bb))
+            !make_map_sw128(&mc, C, 3, db, sb, bb) || !make_map_sw128(&my, p.y, 4, dx, sx, bx))
             return SS_ERR_CUDA;
     }
     if (nseg > 1) {
-        kstate<<<static_cast<unsigned>(items * (nseg - 1)), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc);
+        kstate<<<static_cast<unsigned>(items * (nseg - 1)), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
         SsdParams f = fold_p;
         f.nseg = nseg;
         const int64_t total = items * kSsdP * tc::kN;
         const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), 4096);
         ss_ssd_fold_kernel<tc::kN><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(f);
     }
-    kmain<<<static_cast<unsigned>(items * nseg), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc);
+    kmain<<<static_cast<unsigned>(items * nseg), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 

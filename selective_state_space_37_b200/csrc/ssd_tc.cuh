@@ -17,9 +17,9 @@
 // One CTA (8 warps) walks the chunks of one (b, h) in order.  Thread 0 issues
 // the MMAs (bf16 operands, fp32 accumulation, M = 128):
 //   S   = C Bᵀ          128 x 128, K = N     -> TMEM columns [0, 128)
-//   CG  = C (G_hi + G_lo)ᵀ 128 x 64, K = N   -> TMEM columns [192, 256)
+//   CG  = C [G_hi; G_lo]ᵀ 128 x 128, K = N  -> TMEM columns [192, 320)
 //   Y   = Mm X          128 x 64,  K = Q     -> TMEM columns [128, 192)
-//   ΔGᵀ = Bᵀ X̃          128 x 64,  K = Q     -> TMEM columns [256, 320)
+//   ΔGᵀ = Bᵀ X̃          128 x 64,  K = Q     -> TMEM columns [320, 384)
 // and the eight warps do the elementwise work between them, two threads per
 // TMEM lane (one time step t, or one state index n), each on half of the
 // lane's columns: the causal decay mask Mm from S, X̃ from x, the outputs
@@ -49,8 +49,9 @@ constexpr int kP = 64;             // head dimension
 constexpr int kN = 128;            // state width handled here
 constexpr int kRows = 128;         // TMEM lanes / tile rows
 constexpr int kThreads = 256;      // two threads per row: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
-constexpr uint32_t kTmemCols = 512;   // allocation (power of two >= the 320 columns used)
-constexpr uint32_t kColS = 0, kColY = 128, kColCG = 192, kColG = 256;
+constexpr int kPrefixWarp = 1;   // not warp 0, whose thread 0 issues the MMAs
+constexpr uint32_t kTmemCols = 512;   // allocation (power of two >= the 384 columns used)
+constexpr uint32_t kColS = 0, kColY = 128, kColCG = 192, kColG = 320;   // CG: C G_hiᵀ | C G_loᵀ
 
 // Instruction descriptors (kind::f16, bf16 x bf16 -> fp32, M = 128): bit 4 D
 // format f32, bits 7/10 A/B format bf16, bit 15/16 A/B major (1: MN-major),
@@ -60,6 +61,8 @@ constexpr uint32_t kIdesc_128x64_KMN = (1u << 4) | (1u << 7) | (1u << 10) | (1u 
                                        ((128u >> 4) << 24);
 constexpr uint32_t kIdesc_128x64_MNMN = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
                                         ((64u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kIdesc_128x128_KMN = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((128u >> 3) << 17) |
+                                        ((128u >> 4) << 24);
 
 // Shared memory, byte offsets from a 1024-aligned base.  Every operand tile
 // is a set of [rows][64 bf16] blocks of 128-byte rows in the 128-byte
@@ -70,12 +73,14 @@ constexpr uint32_t kOffXt = 32768;        // X̃ [s][p]
 constexpr uint32_t kOffB = 49152;         // B [s][n]: blocks n 0..63, 64..127
 constexpr uint32_t kOffC = 81920;         // C [t][n]: blocks n 0..63, 64..127
 constexpr uint32_t kOffM = 114688;        // Mm [t][s]: blocks s 0..63, 64..127
-constexpr uint32_t kOffGh = 147456;       // G_hi [n][p]
-constexpr uint32_t kOffGl = 163840;       // G_lo [n][p]
-constexpr uint32_t kOffCum = 180224;      // cum[128] f32
-constexpr uint32_t kOffCs = kOffCum + 512;    // cum · log2 e
-constexpr uint32_t kOffDlt = kOffCs + 512;    // Δ
-constexpr uint32_t kOffBar = kOffDlt + 512;   // 7 mbarriers (8 B each), then the TMEM base address
+constexpr uint32_t kOffGh = 147456;       // G_hi [n][p]  } one MN-major operand of
+constexpr uint32_t kOffGl = 163840;       // G_lo [n][p]  } width 128: blocks 16 KB apart
+constexpr uint32_t kOffY = 180224;        // y [t][p] staged for the bulk tensor store
+constexpr uint32_t kOffCum = 196608;      // cum[2][128] f32 (by chunk parity)
+constexpr uint32_t kOffCs = kOffCum + 1024;   // cum · log2 e, [2][128]
+constexpr uint32_t kOffDlt = kOffCs + 1024;   // Δ, [2][128]
+constexpr uint32_t kOffCf = kOffDlt + 1024;   // Δ_s e^{cum_r - cum_s}, r the last step of s's 32-block, [2][128]
+constexpr uint32_t kOffBar = kOffCf + 1024;   // 7 mbarriers (8 B each), then the TMEM base address
 constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;  // + alignment slack
 
 struct Params {
@@ -156,6 +161,18 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* tm,
         "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
         : "memory");
 }
+// Tile of this CTA's shared memory -> global through the 4-D map (rows past the
+// tensor's extent are not written); completion tracked by the bulk group.
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* tm, uint32_t src, int x, int y, int z, int w) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(tm)),
+                 "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// every committed bulk store has finished reading shared memory / is complete
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tma_load_3d_u(uint32_t dst, const CUtensorMap* tm, int x, int y, int z,
                                               uint64_t* bar) {
     asm volatile(
@@ -192,14 +209,16 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 template <bool STATE>
 __global__ void __launch_bounds__(kThreads, 1)
 ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
-                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C) {
+                 const __grid_constant__ CUtensorMap tm_B, const __grid_constant__ CUtensorMap tm_C,
+                 const __grid_constant__ CUtensorMap tm_y) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;   // 1024-aligned: the swizzle pattern is address based
     unsigned char* gbase = smem_raw + (base - raw);
-    float* cum = reinterpret_cast<float*>(gbase + kOffCum);
-    float* cs = reinterpret_cast<float*>(gbase + kOffCs);
-    float* dlt = reinterpret_cast<float*>(gbase + kOffDlt);
+    float* const cum2 = reinterpret_cast<float*>(gbase + kOffCum);
+    float* const cs2 = reinterpret_cast<float*>(gbase + kOffCs);
+    float* const dlt2 = reinterpret_cast<float*>(gbase + kOffDlt);
+    float* const cf2 = reinterpret_cast<float*>(gbase + kOffCf);
     uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kOffBar);
     uint64_t* x_bar = bars;        // [2]: x tile of buffer 0 / 1 landed
     uint64_t* b_bar = bars + 2;    // B tile landed
@@ -228,7 +247,10 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
         fence_mbar_init();
         tma_prefetch_desc(&tm_x);
         tma_prefetch_desc(&tm_B);
-        if (!STATE) tma_prefetch_desc(&tm_C);
+        if (!STATE) {
+            tma_prefetch_desc(&tm_C);
+            tma_prefetch_desc(&tm_y);
+        }
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -288,17 +310,58 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     }
     float esum = 0.0f;
 
-    // Δraw of the chunk's steps 4·lane .. 4·lane + 3 (warp 0)
-    float dtn[4] = {0.f, 0.f, 0.f, 0.f};
+    // Δraw of the chunk's steps 4·lane .. 4·lane + 3 (the prefix warp)
+    // (raw bf16 bits: widened where they are used, so the load's latency stays off this chunk)
+    uint32_t dtn[4] = {0u, 0u, 0u, 0u};
     auto load_dt = [&](int ci) {
         const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int64_t t = t0 + 4 * lane + e;
-            dtn[e] = t < p.L ? __bfloat162float(p.dt[(static_cast<int64_t>(b) * p.L + t) * p.H + h]) : 0.0f;
+            dtn[e] = t < p.L ? reinterpret_cast<const unsigned short*>(p.dt)[(static_cast<int64_t>(b) * p.L + t) * p.H + h]
+                             : 0u;
         }
     };
-    if (warp == 0 && nchunk > 0) load_dt(0);
+    // Δ and the inclusive prefix of Δ A of chunk ci into buffer ci & 1 (the prefix warp: four
+    // steps per lane, one warp scan); then Δraw of chunk ci + 1 into dtn.
+    auto prefix = [&](int ci) {
+        const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
+        const int q = static_cast<int>(p.L - t0 < kQ ? p.L - t0 : kQ);
+        float dl[4], a[4], run = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            // softplus through the hardware ex2 / lg2: log1p(e^x) = ln 2 · log2(1 + 2^(x log2 e)),
+            // identity above x = 20 (well inside the bf16 outputs' precision)
+            const float xr = __uint_as_float(dtn[e] << 16) + bias;
+            const float spv = (xr > 20.0f) ? xr : kLn2 * lg2_approx(1.0f + ex2_approx(xr * kLog2e));
+            dl[e] = (4 * lane + e < q) ? (p.softplus ? spv : xr) : 0.0f;
+            run = fmaf(dl[e], Ah, run);
+            a[e] = run;
+        }
+        float sc = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float v = __shfl_up_sync(0xffffffffu, sc, o);
+            if (lane >= o) sc += v;
+        }
+        const float excl = sc - run;
+        const int o = (ci & 1) * kQ + 4 * lane;
+        float c2[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c2[e] = (excl + a[e]) * kLog2e;
+        const float c2_end = __shfl_sync(0xffffffffu, c2[3], lane | 7);   // step 32·(lane / 8) + 31
+        *reinterpret_cast<float4*>(cum2 + o) = make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
+        *reinterpret_cast<float4*>(cs2 + o) = make_float4(c2[0], c2[1], c2[2], c2[3]);
+        *reinterpret_cast<float4*>(dlt2 + o) = make_float4(dl[0], dl[1], dl[2], dl[3]);
+        *reinterpret_cast<float4*>(cf2 + o) =
+            make_float4(ex2_approx(c2_end - c2[0]) * dl[0], ex2_approx(c2_end - c2[1]) * dl[1],
+                        ex2_approx(c2_end - c2[2]) * dl[2], ex2_approx(c2_end - c2[3]) * dl[3]);
+        if (ci + 1 < nchunk) load_dt(ci + 1);
+    };
+    if (warp == kPrefixWarp && nchunk > 0) {   // made visible by the first tile wait's barrier
+        load_dt(0);
+        prefix(0);
+    }
 
     bool ok = true;
     // Tile copies issued and waited for, per tensor (the same counts on every
@@ -318,7 +381,6 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
 
     for (int ci = 0; ci < nchunk && ok; ++ci) {
         const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
-        const int q = static_cast<int>(p.L - t0 < kQ ? p.L - t0 : kQ);
         const int xb = ci & 1;
         const uint32_t xbase = base + (xb ? kOffX1 : kOffX0);
         const bool carry = !STATE && (ci > 0 || sg > 0);
@@ -327,35 +389,11 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
             if (tid == 0) issue_x(ci + 1);
             ++x_issued;
         }
-        // Δ and the inclusive prefix of Δ A (warp 0: four steps per lane, one warp scan)
-        if (warp == 0) {
-            float dl[4], a[4], run = 0.0f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                // softplus through the hardware ex2 / lg2: log1p(e^x) = ln 2 · log2(1 + 2^(x log2 e)),
-                // identity above x = 20 (well inside the bf16 outputs' precision)
-                const float xr = dtn[e] + bias;
-                const float spv = (xr > 20.0f) ? xr : kLn2 * lg2_approx(1.0f + ex2_approx(xr * kLog2e));
-                dl[e] = (4 * lane + e < q) ? (p.softplus ? spv : xr) : 0.0f;
-                run = fmaf(dl[e], Ah, run);
-                a[e] = run;
-            }
-            float sc = run;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float v = __shfl_up_sync(0xffffffffu, sc, o);
-                if (lane >= o) sc += v;
-            }
-            const float excl = sc - run;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                cum[4 * lane + e] = excl + a[e];
-                cs[4 * lane + e] = (excl + a[e]) * kLog2e;
-                dlt[4 * lane + e] = dl[e];
-            }
-            if (ci + 1 < nchunk) load_dt(ci + 1);
-        }
-        if (!wait_bar(x_bar + (ci & 1), static_cast<uint32_t>((ci >> 1) & 1))) break;   // also orders cum / dlt
+        const float* cum = cum2 + xb * kQ;   // this chunk's prefix, written during the previous one
+        const float* cs = cs2 + xb * kQ;
+        const float* dlt = dlt2 + xb * kQ;
+        const float* cf = cf2 + xb * kQ;
+        if (!wait_bar(x_bar + (ci & 1), static_cast<uint32_t>((ci >> 1) & 1))) break;
         ++x_waited;
         if (!wait_bar(b_bar, static_cast<uint32_t>(ci & 1))) break;
         ++b_waited;
@@ -376,60 +414,84 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                      kIdesc_128x128_KK, k > 0);
             }
             umma_commit(s_bar);
-            if (carry) {
+            if (carry) {   // B operand [G_hi | G_lo]: N = 128 over two MN blocks 16 KB apart
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k) {
                     const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
-                    const uint64_t ad = sdesc(base + kOffC + aoff, 16, 1024);
-                    umma(tmem + kColCG, ad, sdesc(base + kOffGh + k * 2048u, 0, 1024), kIdesc_128x64_KMN, k > 0);
-                    umma(tmem + kColCG, ad, sdesc(base + kOffGl + k * 2048u, 0, 1024), kIdesc_128x64_KMN, 1);
+                    umma(tmem + kColCG, sdesc(base + kOffC + aoff, 16, 1024), sdesc(base + kOffGh + k * 2048u, 16384, 1024),
+                         kIdesc_128x128_KMN, k > 0);
                 }
             }
         }
-        {   // X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s; a per-row scale, so chunks keep their places)
+        {   // X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s; a per-row scale, so every 16-byte chunk keeps
+            // its place; addressed through the swizzle so that eight consecutive rows hit eight bank groups)
             const int s = row;
             const float w = __expf(cum_end - cum[s]) * dlt[s];
 #pragma unroll
             for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
-                const uint32_t a = xbase + static_cast<uint32_t>(s) * 128u + (c << 4);
-                const uint4 v = lds128(a);
+                const uint4 v = lds128(chunk_addr(xbase, s, c));
                 const uint4 o = make_uint4(pk(lo_f(v.x) * w, hi_f(v.x) * w), pk(lo_f(v.y) * w, hi_f(v.y) * w),
                                            pk(lo_f(v.z) * w, hi_f(v.z) * w), pk(lo_f(v.w) * w, hi_f(v.w) * w));
-                sts128(base + kOffXt + static_cast<uint32_t>(s) * 128u + (c << 4), o);
+                sts128(chunk_addr(base + kOffXt, s, c), o);
             }
         }
         if (!STATE) {
-            // -------- Mm = S ∘ decay mask (row t, s-block hf), once S is in TMEM
+            // -------- Mm = S ∘ decay mask (row t, 32-column blocks 2 hf, 2 hf + 1), once S is in TMEM.
+            // Blocks right of the diagonal are zero.  Strictly below it every s <= t, and the decay
+            // factors through the block's last step r: e^{cum_t - cum_s} = e^{cum_t - cum_r} e^{cum_r - cum_s},
+            // both factors between the exact value and 1, so neither overflows nor loses the product.
+            // The diagonal block takes e^{cum_t - cum_s} per element.
             if (!wait_bar(s_bar, static_cast<uint32_t>(ci & 1))) break;
             tc_fence_after();
             const int t = row;
+            const int rb = warp & 3;   // this warp's 32-row block
             const float ct = cs[t];
 #pragma unroll 1
             for (int g = 2 * hf; g < 2 * hf + 2; ++g) {
                 const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
                 const int c0 = (g & 1) * 4;
-                if (32 * g > t) {   // above the diagonal: zeros
+                if (g > rb) {
 #pragma unroll
                     for (int c = 0; c < 4; ++c) sts128(chunk_addr(blk, t, c0 + c), make_uint4(0, 0, 0, 0));
                     continue;
                 }
                 float sv[32];
                 tmem_ld32(tmem + lane_base + kColS + 32 * g, sv);
+                if (g < rb) {
+                    const float rf = ex2_approx(ct - cs[32 * g + 31]);
+                    const float2 rf2 = make_float2(rf, rf);
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t wv[4];
+                    for (int c = 0; c < 4; ++c) {
+                        const float4 fa = *reinterpret_cast<const float4*>(cf + 32 * g + 8 * c);
+                        const float4 fb = *reinterpret_cast<const float4*>(cf + 32 * g + 8 * c + 4);
+                        const float2 f2[4] = {make_float2(fa.x, fa.y), make_float2(fa.z, fa.w), make_float2(fb.x, fb.y),
+                                              make_float2(fb.z, fb.w)};
+                        uint32_t wv[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        float m2[2];
-#pragma unroll
-                        for (int f = 0; f < 2; ++f) {
-                            const int j = 8 * c + 2 * e + f;
-                            const int s = 32 * g + j;
-                            m2[f] = (s <= t) ? sv[j] * ex2_approx(ct - cs[s]) * dlt[s] : 0.0f;
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 m2 =
+                                __fmul2_rn(__fmul2_rn(make_float2(sv[8 * c + 2 * e], sv[8 * c + 2 * e + 1]), f2[e]), rf2);
+                            wv[e] = pk(m2.x, m2.y);
                         }
-                        wv[e] = pk(m2[0], m2[1]);
+                        sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
                     }
-                    sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t wv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            float m2[2];
+#pragma unroll
+                            for (int f = 0; f < 2; ++f) {
+                                const int j = 8 * c + 2 * e + f;
+                                const int s = 32 * g + j;
+                                m2[f] = (s <= t) ? sv[j] * ex2_approx(ct - cs[s]) * dlt[s] : 0.0f;
+                            }
+                            wv[e] = pk(m2[0], m2[1]);
+                        }
+                        sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                    }
                 }
             }
         }
@@ -454,6 +516,9 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                      sdesc(base + kOffXt + k * 2048u, 0, 1024), kIdesc_128x64_MNMN, k > 0);
             umma_commit(yg_bar);   // also covers C Gᵀ and C Bᵀ, issued before
         }
+        // the next chunk's prefix while the tensor core works (its buffer was last read by chunk ci - 1)
+        if (warp == kPrefixWarp && ci + 1 < nchunk) prefix(ci + 1);
+        if (!STATE && tid == 0) bulk_wait_read0();   // the previous chunk's y tile has left shared memory
         if (!wait_bar(yg_bar, static_cast<uint32_t>(ci & 1))) break;
         tc_fence_after();
         // B and C are free: the next chunk's B and C
@@ -472,9 +537,14 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
             const float et = __expf(cum[t]);
             {
                 const int half = hf;
-                float yv[32], cg[32];
+                float yv[32], cg[32], cl[32];
                 tmem_ld32(tmem + lane_base + kColY + 32 * half, yv);
-                if (carry) tmem_ld32(tmem + lane_base + kColCG + 32 * half, cg);
+                if (carry) {
+                    tmem_ld32(tmem + lane_base + kColCG + 32 * half, cg);
+                    tmem_ld32(tmem + lane_base + kColCG + 64 + 32 * half, cl);
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) cg[j] += cl[j];
+                }
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint4 xv = lds128(chunk_addr(xbase, t, 4 * half + c));
@@ -491,11 +561,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                         }
                         ow[e] = pk(o0, o1);
                     }
-                    if (t < q) {
-                        __nv_bfloat16* yp = p.y + ((static_cast<int64_t>(b) * p.L + t0 + t) * p.H + h) * kP +
-                                            32 * half + 8 * c;
-                        *reinterpret_cast<uint4*>(yp) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
-                    }
+                    sts128(chunk_addr(base + kOffY, t, 4 * half + c), make_uint4(ow[0], ow[1], ow[2], ow[3]));
                 }
             }
         }
@@ -507,10 +573,15 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
             for (int j = 0; j < 32; ++j) G[j] = fmaf(e_end, G[j], dg[j]);
             if (!STATE) store_g();
         }
-        fence_proxy_async_smem();
+        fence_proxy_async_smem();   // G copies and the y tile (generic writes) before the async proxy reads them
         tc_fence_before();
         __syncthreads();
+        if (!STATE && tid == 0) {   // this chunk's y rows (rows past the sequence's end are clipped)
+            tma_store_4d(&tm_y, base + kOffY, 0, h, static_cast<int>(t0), b);
+            bulk_commit();
+        }
     }
+    if (!STATE && tid == 0) bulk_wait0();
 
     // outputs of the state: the segment's G_out (state pass) or the final state
     if (ok) {
