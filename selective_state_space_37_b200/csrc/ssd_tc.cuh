@@ -14,23 +14,28 @@
 //   G ← e^{cum_end} G + (Bᵀ X̃)ᵀ,                X̃[s,:] = e^{cum_end - cum_s} Δ_s x_s
 // with G the P x N state entering the chunk.
 //
-// One CTA (8 warps) walks the chunks of one (b, h) in order.  Thread 0 issues
-// the MMAs (bf16 operands, fp32 accumulation, M = 128):
-//   S   = C Bᵀ          128 x 128, K = N     -> TMEM columns [0, 128)
-//   CG  = C [G_hi; G_lo]ᵀ 128 x 128, K = N  -> TMEM columns [192, 320)
-//   Y   = Mm X          128 x 64,  K = Q     -> TMEM columns [128, 192)
-//   ΔGᵀ = Bᵀ X̃          128 x 64,  K = Q     -> TMEM columns [320, 384)
-// and the eight warps do the elementwise work between them, two threads per
-// TMEM lane (one time step t, or one state index n), each on half of the
-// lane's columns: the causal decay mask Mm from S, X̃ from x, the outputs
-// y = Y + e^{cum_t} CG + D x, and the state update.  The carried state G
-// stays fp32 in registers (the two threads of row n hold G[:, n]); the
-// product with C reads it as two bf16 terms G_hi + G_lo, so it is not
-// rounded to bf16 before the readout.  x, B, C tiles arrive by TMA
-// (x double-buffered and fetched a chunk ahead, C reloaded as soon as its
-// last MMA is done, B likewise), each tensor on its own mbarrier; the MMAs
-// of C Bᵀ and of C Gᵀ complete on separate mbarriers so the mask can start
-// while C Gᵀ still runs.  Every wait (TMA and MMA completions) is bounded.
+// One CTA walks the chunks of one (b, h) in order, its warps specialised:
+//   warp 8 (producer, one thread): TMA loads of the x, B, C tiles and every
+//     MMA (bf16 operands, fp32 accumulation, M = 128):
+//       S   = C Bᵀ              128 x 128, K = N  -> TMEM columns [0, 128)
+//       CG  = C [G_hi | G_lo]ᵀ  128 x 128, K = N  -> TMEM columns [128, 256)
+//       ΔGᵀ = Bᵀ X̃              128 x 64,  K = Q  -> TMEM columns [320, 384)
+//       Y   = Mm X              128 x 64,  K = Q  -> TMEM columns [256, 320)
+//   warp 9: Δ, the prefix of Δ A and the decay factors, a chunk ahead into
+//     a double buffer;
+//   warps 0..7 (compute): two threads per TMEM lane (one time step t, or one
+//     state index n), each on half of the lane's columns: X̃ from x, the
+//     causal decay mask Mm from S, the state update, and the outputs
+//     y = Y + e^{cum_t} CG + D x, staged in shared memory and written by a
+//     bulk tensor store.
+// The warps hand work over through mbarriers, so the tensor core runs the
+// next chunk's C Bᵀ under this chunk's epilogue and Mm X under the state
+// update, and B and C of the next chunk load as soon as their last MMA is
+// done.  The carried state G stays fp32 in registers (the two threads of row
+// n hold G[:, n]); the product with C reads it as two bf16 terms G_hi + G_lo,
+// so it is not rounded to bf16 before the readout.  Every wait is bounded: a
+// wait that runs out records SS error -4 in the status word and the CTA
+// winds down (copies in flight drained, MMAs completed, TMEM released).
 //
 // Time segments: when batch x heads leaves SMs idle, each sequence is cut into
 // segments of whole chunks with an exact carry (state pass from G = 0 keeping
@@ -48,10 +53,12 @@ constexpr int kQ = 128;            // chunk length (MMA M for the time rows)
 constexpr int kP = 64;             // head dimension
 constexpr int kN = 128;            // state width handled here
 constexpr int kRows = 128;         // TMEM lanes / tile rows
-constexpr int kThreads = 256;      // two threads per row: warps w and w + 4 share TMEM lanes 32 (w % 4) ..
-constexpr int kPrefixWarp = 1;   // not warp 0, whose thread 0 issues the MMAs
+constexpr int kComputeThreads = 256;   // warps 0..7; warps w and w + 4 share TMEM lanes 32 (w % 4) ..
+constexpr int kProducerWarp = 8;      // one thread: TMA loads and MMAs
+constexpr int kPrefixWarp = 9;        // the Δ prefix, a chunk ahead
+constexpr int kThreads = kComputeThreads + 64;
 constexpr uint32_t kTmemCols = 512;   // allocation (power of two >= the 384 columns used)
-constexpr uint32_t kColS = 0, kColY = 128, kColCG = 192, kColG = 320;   // CG: C G_hiᵀ | C G_loᵀ
+constexpr uint32_t kColS = 0, kColCG = 128, kColY = 256, kColG = 320;
 
 // Instruction descriptors (kind::f16, bf16 x bf16 -> fp32, M = 128): bit 4 D
 // format f32, bits 7/10 A/B format bf16, bit 15/16 A/B major (1: MN-major),
@@ -80,8 +87,8 @@ constexpr uint32_t kOffCum = 196608;      // cum[2][128] f32 (by chunk parity)
 constexpr uint32_t kOffCs = kOffCum + 1024;   // cum · log2 e, [2][128]
 constexpr uint32_t kOffDlt = kOffCs + 1024;   // Δ, [2][128]
 constexpr uint32_t kOffCf = kOffDlt + 1024;   // Δ_s e^{cum_r - cum_s}, r the last step of s's 32-block, [2][128]
-constexpr uint32_t kOffBar = kOffCf + 1024;   // 7 mbarriers (8 B each), then the TMEM base address
-constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;  // + alignment slack
+constexpr uint32_t kOffBar = kOffCf + 1024;   // 16 mbarriers; TMEM base address at +128, x tiles waited at +132
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 
 struct Params {
     const __nv_bfloat16* dt;   // [batch, L, H]
@@ -129,19 +136,20 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                  : "memory");
 }
-// 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes 32w..32w+31).
+// 32 consecutive fp32 columns of this thread's TMEM lane (warp w reads lanes 32 (w % 4) ..).  The
+// load and its wait are one asm statement: the registers are defined only once the data is in them.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     uint32_t r[32];
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
           "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
           "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
         : "r"(taddr)
         : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
@@ -204,6 +212,25 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
                  : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Barrier 1 over the 256 compute threads: true on every thread when `pred`
+// holds on any of them.
+__device__ __forceinline__ bool cw_any(bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, 256, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void cw_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
 // Grid: one CTA per (segment k, batch b, head h), blockIdx.x = (k * batch + b) * H + h;
 // STATE runs segments 0 .. nseg - 2 only (G_out from zero, no outputs).
 template <bool STATE>
@@ -220,37 +247,36 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     float* const dlt2 = reinterpret_cast<float*>(gbase + kOffDlt);
     float* const cf2 = reinterpret_cast<float*>(gbase + kOffCf);
     uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kOffBar);
-    uint64_t* x_bar = bars;        // [2]: x tile of buffer 0 / 1 landed
-    uint64_t* b_bar = bars + 2;    // B tile landed
-    uint64_t* c_bar = bars + 3;    // C tile landed
-    uint64_t* s_bar = bars + 4;    // C Bᵀ done
-    uint64_t* yg_bar = bars + 6;   // Mm X, Bᵀ X̃ and every earlier MMA done
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 64);
+    uint64_t* x_full = bars;          // [2]: x tile of buffer 0 / 1 landed
+    uint64_t* b_full = bars + 2;      // B tile landed
+    uint64_t* c_full = bars + 3;      // C tile landed
+    uint64_t* s_full = bars + 4;      // C Bᵀ in TMEM
+    uint64_t* cg_done = bars + 5;     // C Bᵀ and C Gᵀ done: C free, G copies read
+    uint64_t* dg_done = bars + 6;     // Bᵀ X̃ done: B and X̃ free
+    uint64_t* y_done = bars + 7;      // Mm X done (and every MMA before it)
+    uint64_t* xt_ready = bars + 8;    // X̃ written (one arrival per compute warp)
+    uint64_t* mm_ready = bars + 9;    // Mm written and S read (one arrival per compute warp)
+    uint64_t* ep_done = bars + 10;    // a chunk's epilogue done: G copies stored, TMEM columns and
+                                      // its x buffer free
+    uint64_t* pf_full = bars + 11;    // [2]: the Δ prefix of buffer 0 / 1 written
+    uint64_t* pf_empty = bars + 13;   // [2]: the chunk reading prefix buffer 0 / 1 is done
+    uint64_t* fin_bar = bars + 15;    // every MMA issued is done (wind-down)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kOffBar + 128);
+    int* xw_slot = reinterpret_cast<int*>(gbase + kOffBar + 132);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int row = tid & (kRows - 1);   // TMEM lane / tile row of this thread
-    const int hf = tid >> 7;             // which half of the row's columns
     const int h = blockIdx.x % p.H;
     const int b = (blockIdx.x / p.H) % p.batch;
     const int sg = blockIdx.x / (p.H * p.batch);
     const int64_t bh = static_cast<int64_t>(b) * p.H + h;
-    const float Ah = p.A[h];
-    const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
-    const float Dh = p.D ? p.D[h] : 0.0f;
     const int64_t seg_t0 = static_cast<int64_t>(sg) * p.cseg * kQ;
     const int64_t seg_t1 = min(seg_t0 + static_cast<int64_t>(p.cseg) * kQ, p.L);
     const int nchunk = static_cast<int>((seg_t1 - seg_t0 + kQ - 1) / kQ);
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;   // this warp's TMEM lanes
+    const uint64_t lim = p.wait_ns;
 
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(bars + i, 1);
+        for (int i = 0; i < 16; ++i) mbar_init(bars + i, (i == 8 || i == 9) ? 8u : 1u);
         fence_mbar_init();
-        tma_prefetch_desc(&tm_x);
-        tma_prefetch_desc(&tm_B);
-        if (!STATE) {
-            tma_prefetch_desc(&tm_C);
-            tma_prefetch_desc(&tm_y);
-        }
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, kTmemCols);
@@ -261,349 +287,413 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // TMA of chunk ci's tiles (thread 0): x into buffer ci & 1, B, C.
-    auto chunk_t0 = [&](int ci) { return static_cast<int>(seg_t0 + static_cast<int64_t>(ci) * kQ); };
-    auto issue_x = [&](int ci) {
-        uint64_t* bar = x_bar + (ci & 1);
-        mbar_arrive_expect_tx(bar, kQ * kP * 2);
-        tma_load_4d(base + ((ci & 1) ? kOffX1 : kOffX0), &tm_x, 0, h, chunk_t0(ci), b, bar);
+    bool ok = true;
+    auto record = [&]() {
+        ok = false;
+        if (p.status) atomicCAS(p.status, 0u, static_cast<uint32_t>(-4));
     };
-    auto issue_b = [&](int ci) {
-        mbar_arrive_expect_tx(b_bar, 2 * kQ * 64 * 2);
-        tma_load_3d_u(base + kOffB, &tm_B, 0, chunk_t0(ci), b, b_bar);
-        tma_load_3d_u(base + kOffB + 16384, &tm_B, 64, chunk_t0(ci), b, b_bar);
-    };
-    auto issue_c = [&](int ci) {
-        mbar_arrive_expect_tx(c_bar, 2 * kQ * 64 * 2);
-        tma_load_3d_u(base + kOffC, &tm_C, 0, chunk_t0(ci), b, c_bar);
-        tma_load_3d_u(base + kOffC + 16384, &tm_C, 64, chunk_t0(ci), b, c_bar);
-    };
-    if (tid == 0 && nchunk > 0) {
-        issue_x(0);
-        issue_b(0);
-        if (!STATE) issue_c(0);
-    }
+    // tile copies issued / waited for, per tensor (producer's counts; x waits are the compute warps')
+    int x_issued = 0, b_issued = 0, c_issued = 0, b_waited = 0, c_waited = 0;
 
-    // Carried state: thread (n, hf) holds G[32 hf .. 32 hf + 31, n] (fp32).
-    // Entering a segment > 0 of the main pass it is the folded record, else zero.
-    float G[kP / 2];
-    const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kP * kN : nullptr;
+    if (warp == kProducerWarp) {
+        // =============================================================== producer (one thread)
+        if (lane == 0) {
+            auto chunk_t0 = [&](int ci) { return static_cast<int>(seg_t0 + static_cast<int64_t>(ci) * kQ); };
+            auto issue_x = [&](int ci) {
+                uint64_t* bar = x_full + (ci & 1);
+                mbar_arrive_expect_tx(bar, kQ * kP * 2);
+                tma_load_4d(base + ((ci & 1) ? kOffX1 : kOffX0), &tm_x, 0, h, chunk_t0(ci), b, bar);
+            };
+            auto issue_b = [&](int ci) {
+                mbar_arrive_expect_tx(b_full, 2 * kQ * 64 * 2);
+                tma_load_3d_u(base + kOffB, &tm_B, 0, chunk_t0(ci), b, b_full);
+                tma_load_3d_u(base + kOffB + 16384, &tm_B, 64, chunk_t0(ci), b, b_full);
+            };
+            auto issue_c = [&](int ci) {
+                mbar_arrive_expect_tx(c_full, 2 * kQ * 64 * 2);
+                tma_load_3d_u(base + kOffC, &tm_C, 0, chunk_t0(ci), b, c_full);
+                tma_load_3d_u(base + kOffC + 16384, &tm_C, 64, chunk_t0(ci), b, c_full);
+            };
+            auto pw_wait = [&](uint64_t* bar, uint32_t parity) {
+                if (mbar_wait_bounded(bar, parity, lim)) return true;
+                record();
+                return false;
+            };
+            if (nchunk > 0) {
+                tma_prefetch_desc(&tm_x);
+                tma_prefetch_desc(&tm_B);
+                if (!STATE) tma_prefetch_desc(&tm_C);
+                issue_x(0);
+                if (nchunk > 1) issue_x(1);
+                issue_b(0);
+                if (!STATE) issue_c(0);
+                x_issued = nchunk > 1 ? 2 : 1;
+                b_issued = 1;
+                c_issued = STATE ? 0 : 1;
+            }
+            for (int ci = 0; ci < nchunk; ++ci) {
+                const bool carry = !STATE && (ci > 0 || sg > 0);
+                const bool more = ci + 1 < nchunk;
+                const uint32_t par = static_cast<uint32_t>(ci & 1);
+                if (!pw_wait(b_full, par)) break;
+                ++b_waited;
+                if (!STATE) {
+                    if (!pw_wait(c_full, par)) break;
+                    ++c_waited;
+                    // S = C Bᵀ (its columns were last read by the previous chunk's mask)
+                    tc_fence_after();
 #pragma unroll
-    for (int q = 0; q < kP / 2; ++q) G[q] = gin ? gin[(32 * hf + q) * kN + row] : 0.0f;
-    auto store_g = [&]() {   // bf16 hi / lo copies of G: row n, chunks 4 hf .. 4 hf + 3 of the [n][p] tiles
+                    for (int k = 0; k < kN / 16; ++k) {
+                        const uint32_t off = (k >> 2) * 16384u + (k & 3) * 32u;
+                        umma(tmem + kColS, sdesc(base + kOffC + off, 16, 1024), sdesc(base + kOffB + off, 16, 1024),
+                             kIdesc_128x128_KK, k > 0);
+                    }
+                    umma_commit(s_full);
+                }
+                // the previous chunk's epilogue (for ci = 0, the compute warps' set-up)
+                if (!pw_wait(ep_done, par)) break;
+                if (ci >= 1 && more) {   // x buffer (ci + 1) & 1 was chunk ci - 1's
+                    issue_x(ci + 1);
+                    ++x_issued;
+                }
+                if (!STATE) {   // CG = C [G_hi | G_lo]ᵀ: N = 128 over two MN blocks 16 KB apart
+                    tc_fence_after();
+                    if (carry) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            uint32_t hw[4], lw[4];
+                        for (int k = 0; k < kN / 16; ++k) {
+                            const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
+                            umma(tmem + kColCG, sdesc(base + kOffC + aoff, 16, 1024),
+                                 sdesc(base + kOffGh + k * 2048u, 16384, 1024), kIdesc_128x128_KMN, k > 0);
+                        }
+                    }
+                    umma_commit(cg_done);
+                }
+                if (!pw_wait(xt_ready, par)) break;
+                tc_fence_after();   // ΔGᵀ = Bᵀ X̃
+#pragma unroll
+                for (int k = 0; k < kQ / 16; ++k)
+                    umma(tmem + kColG, sdesc(base + kOffB + k * 2048u, 16384, 1024),
+                         sdesc(base + kOffXt + k * 2048u, 0, 1024), kIdesc_128x64_MNMN, k > 0);
+                umma_commit(dg_done);
+                if (!STATE && more) {
+                    if (!pw_wait(cg_done, par)) break;
+                    issue_c(ci + 1);
+                    ++c_issued;
+                }
+                if (more) {
+                    if (!pw_wait(dg_done, par)) break;
+                    issue_b(ci + 1);
+                    ++b_issued;
+                }
+                if (!STATE) {
+                    if (!pw_wait(mm_ready, par)) break;
+                    tc_fence_after();   // Y = Mm X
+                    const uint32_t xbase = base + ((ci & 1) ? kOffX1 : kOffX0);
+#pragma unroll
+                    for (int k = 0; k < kQ / 16; ++k) {
+                        const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
+                        umma(tmem + kColY, sdesc(base + kOffM + aoff, 16, 1024), sdesc(xbase + k * 2048u, 0, 1024),
+                             kIdesc_128x64_KMN, k > 0);
+                    }
+                    umma_commit(y_done);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == kPrefixWarp) {
+        // =============================================================== Δ prefix warp
+        const float Ah = p.A[h];
+        const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
+        // Δraw of the chunk's steps 4·lane .. 4·lane + 3, kept as raw bf16 bits
+        // (widened where used, so the load's latency stays off the chunk it is fetched in)
+        uint32_t dtn[4] = {0u, 0u, 0u, 0u};
+        auto load_dt = [&](int ci) {
+            const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float g0 = G[8 * c + 2 * e], g1 = G[8 * c + 2 * e + 1];
-                hw[e] = pk(g0, g1);
-                lw[e] = pk(g0 - lo_f(hw[e]), g1 - hi_f(hw[e]));
+                const int64_t t = t0 + 4 * lane + e;
+                dtn[e] = t < p.L ? reinterpret_cast<const unsigned short*>(p.dt)[(static_cast<int64_t>(b) * p.L + t) *
+                                                                                     p.H + h]
+                                 : 0u;
             }
-            sts128(chunk_addr(base + kOffGh, row, 4 * hf + c), make_uint4(hw[0], hw[1], hw[2], hw[3]));
-            sts128(chunk_addr(base + kOffGl, row, 4 * hf + c), make_uint4(lw[0], lw[1], lw[2], lw[3]));
-        }
-    };
-    if (!STATE && gin) {
-        store_g();
-        fence_proxy_async_smem();   // before the first MMA reads them (ordered by the first wait's barrier)
-    }
-    float esum = 0.0f;
-
-    // Δraw of the chunk's steps 4·lane .. 4·lane + 3 (the prefix warp)
-    // (raw bf16 bits: widened where they are used, so the load's latency stays off this chunk)
-    uint32_t dtn[4] = {0u, 0u, 0u, 0u};
-    auto load_dt = [&](int ci) {
-        const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
+        };
+        // Δ, the inclusive prefix of Δ A and the block factors of chunk ci into buffer ci & 1
+        // (four steps per lane, one warp scan); then Δraw of chunk ci + 1.
+        auto prefix = [&](int ci) {
+            const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
+            const int q = static_cast<int>(p.L - t0 < kQ ? p.L - t0 : kQ);
+            float dl[4], a[4], run = 0.0f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int64_t t = t0 + 4 * lane + e;
-            dtn[e] = t < p.L ? reinterpret_cast<const unsigned short*>(p.dt)[(static_cast<int64_t>(b) * p.L + t) * p.H + h]
-                             : 0u;
-        }
-    };
-    // Δ and the inclusive prefix of Δ A of chunk ci into buffer ci & 1 (the prefix warp: four
-    // steps per lane, one warp scan); then Δraw of chunk ci + 1 into dtn.
-    auto prefix = [&](int ci) {
-        const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
-        const int q = static_cast<int>(p.L - t0 < kQ ? p.L - t0 : kQ);
-        float dl[4], a[4], run = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            // softplus through the hardware ex2 / lg2: log1p(e^x) = ln 2 · log2(1 + 2^(x log2 e)),
-            // identity above x = 20 (well inside the bf16 outputs' precision)
-            const float xr = __uint_as_float(dtn[e] << 16) + bias;
-            const float spv = (xr > 20.0f) ? xr : kLn2 * lg2_approx(1.0f + ex2_approx(xr * kLog2e));
-            dl[e] = (4 * lane + e < q) ? (p.softplus ? spv : xr) : 0.0f;
-            run = fmaf(dl[e], Ah, run);
-            a[e] = run;
-        }
-        float sc = run;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float v = __shfl_up_sync(0xffffffffu, sc, o);
-            if (lane >= o) sc += v;
-        }
-        const float excl = sc - run;
-        const int o = (ci & 1) * kQ + 4 * lane;
-        float c2[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) c2[e] = (excl + a[e]) * kLog2e;
-        const float c2_end = __shfl_sync(0xffffffffu, c2[3], lane | 7);   // step 32·(lane / 8) + 31
-        *reinterpret_cast<float4*>(cum2 + o) = make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
-        *reinterpret_cast<float4*>(cs2 + o) = make_float4(c2[0], c2[1], c2[2], c2[3]);
-        *reinterpret_cast<float4*>(dlt2 + o) = make_float4(dl[0], dl[1], dl[2], dl[3]);
-        *reinterpret_cast<float4*>(cf2 + o) =
-            make_float4(ex2_approx(c2_end - c2[0]) * dl[0], ex2_approx(c2_end - c2[1]) * dl[1],
-                        ex2_approx(c2_end - c2[2]) * dl[2], ex2_approx(c2_end - c2[3]) * dl[3]);
-        if (ci + 1 < nchunk) load_dt(ci + 1);
-    };
-    if (warp == kPrefixWarp && nchunk > 0) {   // made visible by the first tile wait's barrier
-        load_dt(0);
-        prefix(0);
-    }
-
-    bool ok = true;
-    // Tile copies issued and waited for, per tensor (the same counts on every
-    // thread): copies still in flight are drained before the shared memory is
-    // released after a failure.
-    const int first = nchunk > 0 ? 1 : 0;
-    int x_issued = first, x_waited = 0, b_issued = first, b_waited = 0, c_issued = STATE ? 0 : first, c_waited = 0;
-    auto wait_bar = [&](uint64_t* bar, uint32_t parity) {
-        const bool got = mbar_wait_bounded(bar, parity, p.wait_ns);
-        const int bad = __syncthreads_or(got ? 0 : 1);
-        if (bad) {
-            ok = false;
-            if (tid == 0 && p.status) atomicCAS(p.status, 0u, static_cast<uint32_t>(-4));
-        }
-        return !bad;
-    };
-
-    for (int ci = 0; ci < nchunk && ok; ++ci) {
-        const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
-        const int xb = ci & 1;
-        const uint32_t xbase = base + (xb ? kOffX1 : kOffX0);
-        const bool carry = !STATE && (ci > 0 || sg > 0);
-        // the next chunk's x (its buffer was last read by chunk ci - 1, now done)
-        if (ci + 1 < nchunk) {
-            if (tid == 0) issue_x(ci + 1);
-            ++x_issued;
-        }
-        const float* cum = cum2 + xb * kQ;   // this chunk's prefix, written during the previous one
-        const float* cs = cs2 + xb * kQ;
-        const float* dlt = dlt2 + xb * kQ;
-        const float* cf = cf2 + xb * kQ;
-        if (!wait_bar(x_bar + (ci & 1), static_cast<uint32_t>((ci >> 1) & 1))) break;
-        ++x_waited;
-        if (!wait_bar(b_bar, static_cast<uint32_t>(ci & 1))) break;
-        ++b_waited;
-        if (!STATE) {
-            if (!wait_bar(c_bar, static_cast<uint32_t>(ci & 1))) break;
-            ++c_waited;
-        }
-        const float cum_end = cum[kQ - 1];
-        if (STATE) esum += cum_end;
-
-        // -------- S = C Bᵀ and CG = C (G_hi + G_lo)ᵀ (thread 0), X̃ (all threads)
-        if (!STATE && tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int k = 0; k < kN / 16; ++k) {
-                const uint32_t off = (k >> 2) * 16384u + (k & 3) * 32u;
-                umma(tmem + kColS, sdesc(base + kOffC + off, 16, 1024), sdesc(base + kOffB + off, 16, 1024),
-                     kIdesc_128x128_KK, k > 0);
+            for (int e = 0; e < 4; ++e) {
+                // softplus through the hardware ex2 / lg2: log1p(e^x) = ln 2 · log2(1 + 2^(x log2 e)),
+                // identity above x = 20 (well inside the bf16 outputs' precision)
+                const float xr = __uint_as_float(dtn[e] << 16) + bias;
+                const float spv = (xr > 20.0f) ? xr : kLn2 * lg2_approx(1.0f + ex2_approx(xr * kLog2e));
+                dl[e] = (4 * lane + e < q) ? (p.softplus ? spv : xr) : 0.0f;
+                run = fmaf(dl[e], Ah, run);
+                a[e] = run;
             }
-            umma_commit(s_bar);
-            if (carry) {   // B operand [G_hi | G_lo]: N = 128 over two MN blocks 16 KB apart
+            float sc = run;
 #pragma unroll
-                for (int k = 0; k < kN / 16; ++k) {
-                    const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
-                    umma(tmem + kColCG, sdesc(base + kOffC + aoff, 16, 1024), sdesc(base + kOffGh + k * 2048u, 16384, 1024),
-                         kIdesc_128x128_KMN, k > 0);
+            for (int o = 1; o < 32; o <<= 1) {
+                const float v = __shfl_up_sync(0xffffffffu, sc, o);
+                if (lane >= o) sc += v;
+            }
+            const float excl = sc - run;
+            const int o = (ci & 1) * kQ + 4 * lane;
+            float c2[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) c2[e] = (excl + a[e]) * kLog2e;
+            const float c2_end = __shfl_sync(0xffffffffu, c2[3], lane | 7);   // step 32·(lane / 8) + 31
+            *reinterpret_cast<float4*>(cum2 + o) = make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
+            *reinterpret_cast<float4*>(cs2 + o) = make_float4(c2[0], c2[1], c2[2], c2[3]);
+            *reinterpret_cast<float4*>(dlt2 + o) = make_float4(dl[0], dl[1], dl[2], dl[3]);
+            *reinterpret_cast<float4*>(cf2 + o) =
+                make_float4(ex2_approx(c2_end - c2[0]) * dl[0], ex2_approx(c2_end - c2[1]) * dl[1],
+                            ex2_approx(c2_end - c2[2]) * dl[2], ex2_approx(c2_end - c2[3]) * dl[3]);
+            if (ci + 1 < nchunk) load_dt(ci + 1);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pf_full + (ci & 1));   // release: the writes above precede it
+        };
+        if (nchunk > 0) load_dt(0);
+        for (int ci = 0; ci < nchunk; ++ci) {
+            if (ci >= 2) {   // buffer ci & 1 was chunk ci - 2's
+                bool got = true;
+                if (lane == 0) got = mbar_wait_bounded(pf_empty + (ci & 1), static_cast<uint32_t>(((ci >> 1) - 1) & 1), lim);
+                got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+                if (!got) {
+                    if (lane == 0) record();
+                    break;
                 }
             }
+            prefix(ci);
         }
-        {   // X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s; a per-row scale, so every 16-byte chunk keeps
-            // its place; addressed through the swizzle so that eight consecutive rows hit eight bank groups)
-            const int s = row;
-            const float w = __expf(cum_end - cum[s]) * dlt[s];
+    } else {
+        // =============================================================== compute warps
+        const int row = tid & (kRows - 1);   // TMEM lane / tile row of this thread
+        const int hf = tid >> 7;             // which half of the row's columns
+        const int rb = warp & 3;             // this warp's 32-row block
+        const uint32_t lane_base = static_cast<uint32_t>(rb * 32) << 16;   // this warp's TMEM lanes
+        const float Dh = p.D ? p.D[h] : 0.0f;
+        // Carried state: thread (n, hf) holds G[32 hf .. 32 hf + 31, n] (fp32).
+        // Entering a segment > 0 of the main pass it is the folded record, else zero.
+        float G[kP / 2];
+        const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kP * kN : nullptr;
 #pragma unroll
-            for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
-                const uint4 v = lds128(chunk_addr(xbase, s, c));
-                const uint4 o = make_uint4(pk(lo_f(v.x) * w, hi_f(v.x) * w), pk(lo_f(v.y) * w, hi_f(v.y) * w),
-                                           pk(lo_f(v.z) * w, hi_f(v.z) * w), pk(lo_f(v.w) * w, hi_f(v.w) * w));
-                sts128(chunk_addr(base + kOffXt, s, c), o);
-            }
-        }
-        if (!STATE) {
-            // -------- Mm = S ∘ decay mask (row t, 32-column blocks 2 hf, 2 hf + 1), once S is in TMEM.
-            // Blocks right of the diagonal are zero.  Strictly below it every s <= t, and the decay
-            // factors through the block's last step r: e^{cum_t - cum_s} = e^{cum_t - cum_r} e^{cum_r - cum_s},
-            // both factors between the exact value and 1, so neither overflows nor loses the product.
-            // The diagonal block takes e^{cum_t - cum_s} per element.
-            if (!wait_bar(s_bar, static_cast<uint32_t>(ci & 1))) break;
-            tc_fence_after();
-            const int t = row;
-            const int rb = warp & 3;   // this warp's 32-row block
-            const float ct = cs[t];
-#pragma unroll 1
-            for (int g = 2 * hf; g < 2 * hf + 2; ++g) {
-                const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
-                const int c0 = (g & 1) * 4;
-                if (g > rb) {
+        for (int q = 0; q < kP / 2; ++q) G[q] = gin ? gin[(32 * hf + q) * kN + row] : 0.0f;
+        auto store_g = [&]() {   // bf16 hi / lo copies of G: row n, chunks 4 hf .. 4 hf + 3 of the [n][p] tiles
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) sts128(chunk_addr(blk, t, c0 + c), make_uint4(0, 0, 0, 0));
-                    continue;
+            for (int c = 0; c < 4; ++c) {
+                uint32_t hw[4], lw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float g0 = G[8 * c + 2 * e], g1 = G[8 * c + 2 * e + 1];
+                    hw[e] = pk(g0, g1);
+                    lw[e] = pk(g0 - lo_f(hw[e]), g1 - hi_f(hw[e]));
                 }
-                float sv[32];
-                tmem_ld32(tmem + lane_base + kColS + 32 * g, sv);
-                if (g < rb) {
-                    const float rf = ex2_approx(ct - cs[32 * g + 31]);
-                    const float2 rf2 = make_float2(rf, rf);
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float4 fa = *reinterpret_cast<const float4*>(cf + 32 * g + 8 * c);
-                        const float4 fb = *reinterpret_cast<const float4*>(cf + 32 * g + 8 * c + 4);
-                        const float2 f2[4] = {make_float2(fa.x, fa.y), make_float2(fa.z, fa.w), make_float2(fb.x, fb.y),
-                                              make_float2(fb.z, fb.w)};
-                        uint32_t wv[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 m2 =
-                                __fmul2_rn(__fmul2_rn(make_float2(sv[8 * c + 2 * e], sv[8 * c + 2 * e + 1]), f2[e]), rf2);
-                            wv[e] = pk(m2.x, m2.y);
-                        }
-                        sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t wv[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            float m2[2];
-#pragma unroll
-                            for (int f = 0; f < 2; ++f) {
-                                const int j = 8 * c + 2 * e + f;
-                                const int s = 32 * g + j;
-                                m2[f] = (s <= t) ? sv[j] * ex2_approx(ct - cs[s]) * dlt[s] : 0.0f;
-                            }
-                            wv[e] = pk(m2[0], m2[1]);
-                        }
-                        sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
-                    }
-                }
+                sts128(chunk_addr(base + kOffGh, row, 4 * hf + c), make_uint4(hw[0], hw[1], hw[2], hw[3]));
+                sts128(chunk_addr(base + kOffGl, row, 4 * hf + c), make_uint4(lw[0], lw[1], lw[2], lw[3]));
             }
-        }
-        fence_proxy_async_smem();   // Mm and X̃ (generic writes) before the MMAs read them
-        tc_fence_before();
-        __syncthreads();
+        };
+        if (gin) store_g();
+        fence_proxy_async_smem();   // G copies (generic writes) before the first C Gᵀ reads them
+        cw_sync();
+        if (tid == 0) mbar_arrive(ep_done);
 
-        // -------- Y = Mm X (main pass) and ΔGᵀ = Bᵀ X̃ (thread 0)
-        if (tid == 0) {
-            tc_fence_after();
+        // every thread waits; one barrier over the compute warps makes the outcome uniform
+        auto cw_wait2 = [&](uint64_t* bar0, uint32_t par0, uint64_t* bar1, uint32_t par1) {
+            bool got = bar0 ? mbar_wait_bounded(bar0, par0, lim) : true;
+            if (got && bar1) got = mbar_wait_bounded(bar1, par1, lim);
+            const bool bad = cw_any(!got);
+            if (bad) {
+                ok = false;
+                if (tid == 0) record();
+            }
+            return !bad;
+        };
+        float esum = 0.0f;
+        int x_waited = 0;
+        for (int ci = 0; ci < nchunk; ++ci) {
+            const int64_t t0 = seg_t0 + static_cast<int64_t>(ci) * kQ;
+            const int xb = ci & 1;
+            const uint32_t par = static_cast<uint32_t>(xb);
+            const uint32_t xbase = base + (xb ? kOffX1 : kOffX0);
+            const bool carry = !STATE && (ci > 0 || sg > 0);
+            const float* cum = cum2 + xb * kQ;
+            const float* cs = cs2 + xb * kQ;
+            const float* dlt = dlt2 + xb * kQ;
+            const float* cf = cf2 + xb * kQ;
+            if (!cw_wait2(x_full + xb, static_cast<uint32_t>((ci >> 1) & 1), pf_full + xb, static_cast<uint32_t>((ci >> 1) & 1)))
+                break;
+            ++x_waited;
+            const float cum_end = cum[kQ - 1];
+            if (STATE) esum += cum_end;
+
+            {   // -------- X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s; a per-row scale, so every 16-byte
+                // chunk keeps its place; addressed through the swizzle so that eight consecutive rows hit
+                // eight bank groups).  X̃ was last read by the previous chunk's Bᵀ X̃, waited for below.
+                const int s = row;
+                const float w = __expf(cum_end - cum[s]) * dlt[s];
+#pragma unroll
+                for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
+                    const uint4 v = lds128(chunk_addr(xbase, s, c));
+                    const uint4 o = make_uint4(pk(lo_f(v.x) * w, hi_f(v.x) * w), pk(lo_f(v.y) * w, hi_f(v.y) * w),
+                                               pk(lo_f(v.z) * w, hi_f(v.z) * w), pk(lo_f(v.w) * w, hi_f(v.w) * w));
+                    sts128(chunk_addr(base + kOffXt, s, c), o);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(xt_ready);
+            }
             if (!STATE) {
+                // -------- Mm = S ∘ decay mask (row t, 32-column blocks 2 hf, 2 hf + 1).  Blocks right of the
+                // diagonal are zero.  Strictly below it every s <= t, and the decay factors through the
+                // block's last step r: e^{cum_t - cum_s} = e^{cum_t - cum_r} e^{cum_r - cum_s}, both factors
+                // between the exact value and 1, so neither overflows nor loses the product.  The diagonal
+                // block takes e^{cum_t - cum_s} per element.  Mm was last read by the previous chunk's Mm X.
+                if (!cw_wait2(s_full, par, nullptr, 0)) break;
+                tc_fence_after();
+                const int t = row;
+                const float ct = cs[t];
+#pragma unroll 1
+                for (int gi = 0; gi < 2; ++gi) {
+                    const int g = 2 * hf + gi;
+                    const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
+                    const int c0 = (g & 1) * 4;
+                    if (g > rb) {
 #pragma unroll
-                for (int k = 0; k < kQ / 16; ++k) {
-                    const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
-                    umma(tmem + kColY, sdesc(base + kOffM + aoff, 16, 1024), sdesc(xbase + k * 2048u, 0, 1024),
-                         kIdesc_128x64_KMN, k > 0);
+                        for (int c = 0; c < 4; ++c) sts128(chunk_addr(blk, t, c0 + c), make_uint4(0, 0, 0, 0));
+                        continue;
+                    }
+                    float sv[32];
+                    tmem_ld32(tmem + lane_base + kColS + 32 * g, sv);
+                    if (g < rb) {
+                        const float rf = ex2_approx(ct - cs[32 * g + 31]);
+                        const float2 rf2 = make_float2(rf, rf);
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const float4 fa = *reinterpret_cast<const float4*>(cf + 32 * g + 8 * c);
+                            const float4 fb = *reinterpret_cast<const float4*>(cf + 32 * g + 8 * c + 4);
+                            const float2 f2[4] = {make_float2(fa.x, fa.y), make_float2(fa.z, fa.w),
+                                                  make_float2(fb.x, fb.y), make_float2(fb.z, fb.w)};
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 m2 = __fmul2_rn(
+                                    __fmul2_rn(make_float2(sv[8 * c + 2 * e], sv[8 * c + 2 * e + 1]), f2[e]), rf2);
+                                wv[e] = pk(m2.x, m2.y);
+                            }
+                            sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                        }
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                float m2[2];
+#pragma unroll
+                                for (int f = 0; f < 2; ++f) {
+                                    const int j = 8 * c + 2 * e + f;
+                                    const int s = 32 * g + j;
+                                    m2[f] = (s <= t) ? sv[j] * ex2_approx(ct - cs[s]) * dlt[s] : 0.0f;
+                                }
+                                wv[e] = pk(m2[0], m2[1]);
+                            }
+                            sts128(chunk_addr(blk, t, c0 + c), make_uint4(wv[0], wv[1], wv[2], wv[3]));
+                        }
+                    }
                 }
+                fence_proxy_async_smem();   // Mm before the MMA reads it
+                tc_fence_before();          // S read before its columns are written again
+                __syncwarp();
+                if (lane == 0) mbar_arrive(mm_ready);
             }
-#pragma unroll
-            for (int k = 0; k < kQ / 16; ++k)
-                umma(tmem + kColG, sdesc(base + kOffB + k * 2048u, 16384, 1024),
-                     sdesc(base + kOffXt + k * 2048u, 0, 1024), kIdesc_128x64_MNMN, k > 0);
-            umma_commit(yg_bar);   // also covers C Gᵀ and C Bᵀ, issued before
-        }
-        // the next chunk's prefix while the tensor core works (its buffer was last read by chunk ci - 1)
-        if (warp == kPrefixWarp && ci + 1 < nchunk) prefix(ci + 1);
-        if (!STATE && tid == 0) bulk_wait_read0();   // the previous chunk's y tile has left shared memory
-        if (!wait_bar(yg_bar, static_cast<uint32_t>(ci & 1))) break;
-        tc_fence_after();
-        // B and C are free: the next chunk's B and C
-        if (ci + 1 < nchunk) {
-            if (tid == 0) {
-                issue_b(ci + 1);
-                if (!STATE) issue_c(ci + 1);
-            }
-            ++b_issued;
-            if (!STATE) ++c_issued;
-        }
-
-        if (!STATE) {
-            // -------- y = Y + e^{cum_t} CG + D x (row t, columns 32 hf .. 32 hf + 31)
-            const int t = row;
-            const float et = __expf(cum[t]);
+            // -------- G = e^{cum_end} G + ΔGᵀ[n, :] (row n, columns 32 hf .. 32 hf + 31), once Bᵀ X̃ is
+            // done and C Gᵀ has read the previous copies of G
+            if (!cw_wait2(STATE ? nullptr : cg_done, par, dg_done, par)) break;
+            tc_fence_after();
             {
-                const int half = hf;
-                float yv[32], cg[32], cl[32];
-                tmem_ld32(tmem + lane_base + kColY + 32 * half, yv);
-                if (carry) {
-                    tmem_ld32(tmem + lane_base + kColCG + 32 * half, cg);
-                    tmem_ld32(tmem + lane_base + kColCG + 64 + 32 * half, cl);
+                const float e_end = __expf(cum_end);
+                float dg[32];
+                tmem_ld32(tmem + lane_base + kColG + 32 * hf, dg);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) cg[j] += cl[j];
+                for (int j = 0; j < 32; ++j) G[j] = fmaf(e_end, G[j], dg[j]);
+                if (!STATE) store_g();
+            }
+            if (!STATE) {
+                // -------- y = Y + e^{cum_t} CG + D x (row t, columns 32 hf .. 32 hf + 31) into the staging tile
+                if (tid == 0) bulk_wait_read0();   // the previous chunk's y tile has left shared memory
+                if (!cw_wait2(y_done, par, nullptr, 0)) break;
+                tc_fence_after();
+                const int t = row;
+                const float et = __expf(cum[t]);
+                float acc[32], gv[32];
+                tmem_ld32(tmem + lane_base + kColY + 32 * hf, acc);
+                if (carry) {
+                    tmem_ld32(tmem + lane_base + kColCG + 32 * hf, gv);   // C G_hiᵀ
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
+                    tmem_ld32(tmem + lane_base + kColCG + 64 + 32 * hf, gv);   // C G_loᵀ
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
                 }
+                uint4 xv[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) xv[c] = lds128(chunk_addr(xbase, t, 4 * hf + c));
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const uint4 xv = lds128(chunk_addr(xbase, t, 4 * half + c));
-                    const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+                    const uint32_t xw[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
                     uint32_t ow[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         const int j = 8 * c + 2 * e;
-                        float o0 = fmaf(Dh, lo_f(xw[e]), yv[j]);
-                        float o1 = fmaf(Dh, hi_f(xw[e]), yv[j + 1]);
-                        if (carry) {
-                            o0 = fmaf(et, cg[j], o0);
-                            o1 = fmaf(et, cg[j + 1], o1);
-                        }
-                        ow[e] = pk(o0, o1);
+                        ow[e] = pk(fmaf(Dh, lo_f(xw[e]), acc[j]), fmaf(Dh, hi_f(xw[e]), acc[j + 1]));
                     }
-                    sts128(chunk_addr(base + kOffY, t, 4 * half + c), make_uint4(ow[0], ow[1], ow[2], ow[3]));
+                    sts128(chunk_addr(base + kOffY, t, 4 * hf + c), make_uint4(ow[0], ow[1], ow[2], ow[3]));
                 }
             }
+            fence_proxy_async_smem();   // G copies and the y tile before the async proxy reads them
+            tc_fence_before();          // TMEM reads before the columns are written again
+            cw_sync();
+            if (tid == 0) {
+                if (!STATE) {   // this chunk's y rows (rows past the sequence's end are clipped)
+                    tma_store_4d(&tm_y, base + kOffY, 0, h, static_cast<int>(t0), b);
+                    bulk_commit();
+                }
+                mbar_arrive(ep_done);
+                mbar_arrive(pf_empty + xb);
+            }
         }
-        {   // -------- G = e^{cum_end} G + ΔGᵀ[n, :] (row n, columns 32 hf .. 32 hf + 31)
-            const float e_end = __expf(cum_end);
-            float dg[32];
-            tmem_ld32(tmem + lane_base + kColG + 32 * hf, dg);
+        // outputs of the state: the segment's G_out (state pass) or the final state
+        if (ok) {
+            float* out = nullptr;
+            if (STATE) out = p.rec + (bh * (p.nseg - 1) + sg) * kP * kN;
+            else if (p.final_state && sg == p.nseg - 1) out = p.final_state + bh * kP * kN;
+            if (out) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) G[j] = fmaf(e_end, G[j], dg[j]);
-            if (!STATE) store_g();
+                for (int q2 = 0; q2 < kP / 2; ++q2) out[(32 * hf + q2) * kN + row] = G[q2];
+            }
+            if (STATE && tid == 0) p.esum[bh * p.nseg + sg] = esum;
         }
-        fence_proxy_async_smem();   // G copies and the y tile (generic writes) before the async proxy reads them
-        tc_fence_before();
-        __syncthreads();
-        if (!STATE && tid == 0) {   // this chunk's y rows (rows past the sequence's end are clipped)
-            tma_store_4d(&tm_y, base + kOffY, 0, h, static_cast<int>(t0), b);
-            bulk_commit();
+        if (tid == 0) {
+            if (!STATE) bulk_wait0();
+            *xw_slot = x_waited;
         }
     }
-    if (!STATE && tid == 0) bulk_wait0();
 
-    // outputs of the state: the segment's G_out (state pass) or the final state
-    if (ok) {
-        float* out = nullptr;
-        if (STATE) out = p.rec + (bh * (p.nseg - 1) + sg) * kP * kN;
-        else if (p.final_state && sg == p.nseg - 1) out = p.final_state + bh * kP * kN;
-        if (out) {
-#pragma unroll
-            for (int q2 = 0; q2 < kP / 2; ++q2) out[(32 * hf + q2) * kN + row] = G[q2];
-        }
-        if (STATE && tid == 0) p.esum[bh * p.nseg + sg] = esum;
+    // Wind-down.  Copies still in flight land before the shared memory is
+    // released, and every MMA issued completes before the TMEM columns are
+    // (both bounded; a completed phase is recognised as well).
+    __syncthreads();
+    if (warp == kProducerWarp && lane == 0) {
+        for (int cj = *xw_slot; cj < x_issued; ++cj)   // chunk cj's x: buffer cj & 1, phase cj >> 1
+            mbar_wait_bounded(x_full + (cj & 1), static_cast<uint32_t>((cj >> 1) & 1), lim);
+        if (b_waited < b_issued) mbar_wait_bounded(b_full, static_cast<uint32_t>(b_waited & 1), lim);
+        if (c_waited < c_issued) mbar_wait_bounded(c_full, static_cast<uint32_t>(c_waited & 1), lim);
+        umma_commit(fin_bar);
+        mbar_wait_bounded(fin_bar, 0, lim);
     }
-    // After a wait that ran out: let copies still in flight land before the
-    // shared memory is released (bounded as well; their phases are the next
-    // ones of each barrier, so a completed phase is recognised too).
-    if (!ok) {
-        for (int cj = x_waited; cj < x_issued; ++cj)   // chunk cj's x: buffer cj & 1, phase cj >> 1
-            mbar_wait_bounded(x_bar + (cj & 1), static_cast<uint32_t>((cj >> 1) & 1), p.wait_ns);
-        if (b_waited < b_issued) mbar_wait_bounded(b_bar, static_cast<uint32_t>(b_waited & 1), p.wait_ns);
-        if (c_waited < c_issued) mbar_wait_bounded(c_bar, static_cast<uint32_t>(c_waited & 1), p.wait_ns);
-    }
-    // every TMEM read and MMA is complete (waited above); release the columns
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
