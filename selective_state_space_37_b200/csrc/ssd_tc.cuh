@@ -87,7 +87,8 @@ constexpr uint32_t kOffCum = 196608;      // cum[2][128] f32 (by chunk parity)
 constexpr uint32_t kOffCs = kOffCum + 1024;   // cum · log2 e, [2][128]
 constexpr uint32_t kOffDlt = kOffCs + 1024;   // Δ, [2][128]
 constexpr uint32_t kOffCf = kOffDlt + 1024;   // Δ_s e^{cum_r - cum_s}, r the last step of s's 32-block, [2][128]
-constexpr uint32_t kOffBar = kOffCf + 1024;   // 16 mbarriers; TMEM base address at +128, x tiles waited at +132
+constexpr uint32_t kOffWx = kOffCf + 1024;   // e^{cum_end - cum_s} Δ_s, the scale of X̃'s row s, [2][128]
+constexpr uint32_t kOffBar = kOffWx + 1024;   // 16 mbarriers; TMEM base address at +128, x tiles waited at +132
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;  // + alignment slack
 
 struct Params {
@@ -246,6 +247,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     float* const cs2 = reinterpret_cast<float*>(gbase + kOffCs);
     float* const dlt2 = reinterpret_cast<float*>(gbase + kOffDlt);
     float* const cf2 = reinterpret_cast<float*>(gbase + kOffCf);
+    float* const wx2 = reinterpret_cast<float*>(gbase + kOffWx);
     uint64_t* bars = reinterpret_cast<uint64_t*>(gbase + kOffBar);
     uint64_t* x_full = bars;          // [2]: x tile of buffer 0 / 1 landed
     uint64_t* b_full = bars + 2;      // B tile landed
@@ -445,12 +447,16 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
 #pragma unroll
             for (int e = 0; e < 4; ++e) c2[e] = (excl + a[e]) * kLog2e;
             const float c2_end = __shfl_sync(0xffffffffu, c2[3], lane | 7);   // step 32·(lane / 8) + 31
+            const float c2_tot = __shfl_sync(0xffffffffu, c2[3], 31);         // the chunk's last step
             *reinterpret_cast<float4*>(cum2 + o) = make_float4(excl + a[0], excl + a[1], excl + a[2], excl + a[3]);
             *reinterpret_cast<float4*>(cs2 + o) = make_float4(c2[0], c2[1], c2[2], c2[3]);
             *reinterpret_cast<float4*>(dlt2 + o) = make_float4(dl[0], dl[1], dl[2], dl[3]);
             *reinterpret_cast<float4*>(cf2 + o) =
                 make_float4(ex2_approx(c2_end - c2[0]) * dl[0], ex2_approx(c2_end - c2[1]) * dl[1],
                             ex2_approx(c2_end - c2[2]) * dl[2], ex2_approx(c2_end - c2[3]) * dl[3]);
+            *reinterpret_cast<float4*>(wx2 + o) =
+                make_float4(ex2_approx(c2_tot - c2[0]) * dl[0], ex2_approx(c2_tot - c2[1]) * dl[1],
+                            ex2_approx(c2_tot - c2[2]) * dl[2], ex2_approx(c2_tot - c2[3]) * dl[3]);
             if (ci + 1 < nchunk) load_dt(ci + 1);
             __syncwarp();
             if (lane == 0) mbar_arrive(pf_full + (ci & 1));   // release: the writes above precede it
@@ -496,7 +502,17 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
             }
         };
         if (gin) store_g();
-        fence_proxy_async_smem();   // G copies (generic writes) before the first C Gᵀ reads them
+        if (!STATE) {   // Mm right of the diagonal is zero in every chunk: written once
+            const int rb0 = warp & 3;
+#pragma unroll 1
+            for (int g = 2 * hf; g < 2 * hf + 2; ++g) {
+                if (g <= rb0) continue;
+                const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) sts128(chunk_addr(blk, row, (g & 1) * 4 + c), make_uint4(0, 0, 0, 0));
+            }
+        }
+        fence_proxy_async_smem();   // G copies and the zero blocks (generic writes) before the MMAs read them
         cw_sync();
         if (tid == 0) mbar_arrive(ep_done);
 
@@ -529,17 +545,18 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
             const float cum_end = cum[kQ - 1];
             if (STATE) esum += cum_end;
 
-            {   // -------- X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s; a per-row scale, so every 16-byte
-                // chunk keeps its place; addressed through the swizzle so that eight consecutive rows hit
-                // eight bank groups).  X̃ was last read by the previous chunk's Bᵀ X̃, waited for below.
-                const int s = row;
-                const float w = __expf(cum_end - cum[s]) * dlt[s];
+            {   // -------- X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s, chunks 4 hf .. 4 hf + 3; a per-row
+                // scale, so every 16-byte chunk keeps its place; addressed through the swizzle so that eight
+                // consecutive rows hit eight bank groups).  X̃ was last read by the previous chunk's Bᵀ X̃,
+                // waited for below.
+                const int sr = row;
+                const float w = wx2[xb * kQ + sr];
 #pragma unroll
                 for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
-                    const uint4 v = lds128(chunk_addr(xbase, s, c));
+                    const uint4 v = lds128(chunk_addr(xbase, sr, c));
                     const uint4 o = make_uint4(pk(lo_f(v.x) * w, hi_f(v.x) * w), pk(lo_f(v.y) * w, hi_f(v.y) * w),
                                                pk(lo_f(v.z) * w, hi_f(v.z) * w), pk(lo_f(v.w) * w, hi_f(v.w) * w));
-                    sts128(chunk_addr(base + kOffXt, s, c), o);
+                    sts128(chunk_addr(base + kOffXt, sr, c), o);
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
@@ -560,11 +577,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                     const int g = 2 * hf + gi;
                     const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
                     const int c0 = (g & 1) * 4;
-                    if (g > rb) {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) sts128(chunk_addr(blk, t, c0 + c), make_uint4(0, 0, 0, 0));
-                        continue;
-                    }
+                    if (g > rb) continue;   // zero, written before the first chunk
                     float sv[32];
                     tmem_ld32(tmem + lane_base + kColS + 32 * g, sv);
                     if (g < rb) {
@@ -588,15 +601,21 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                     } else {
 #pragma unroll
                         for (int c = 0; c < 4; ++c) {
+                            const int s0 = 32 * g + 8 * c;
+                            const float4 ca = *reinterpret_cast<const float4*>(cs + s0);
+                            const float4 cb = *reinterpret_cast<const float4*>(cs + s0 + 4);
+                            const float4 da = *reinterpret_cast<const float4*>(dlt + s0);
+                            const float4 db = *reinterpret_cast<const float4*>(dlt + s0 + 4);
+                            const float csv[8] = {ca.x, ca.y, ca.z, ca.w, cb.x, cb.y, cb.z, cb.w};
+                            const float dv[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
                             uint32_t wv[4];
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
                                 float m2[2];
 #pragma unroll
                                 for (int f = 0; f < 2; ++f) {
-                                    const int j = 8 * c + 2 * e + f;
-                                    const int s = 32 * g + j;
-                                    m2[f] = (s <= t) ? sv[j] * ex2_approx(ct - cs[s]) * dlt[s] : 0.0f;
+                                    const int i = 2 * e + f;
+                                    m2[f] = (s0 + i <= t) ? sv[8 * c + i] * ex2_approx(ct - csv[i]) * dv[i] : 0.0f;
                                 }
                                 wv[e] = pk(m2[0], m2[1]);
                             }
