@@ -250,19 +250,26 @@ typedef struct ss_ssd_dims {
  *   final_state  [batch, nheads, headdim, d_state] fp32 or NULL
  *   flags        SS_DELTA_SOFTPLUS, SS_SYNC_CHECK (bf16 only; SS_BF16 ignored)
  *   launch       stream; workspace (optional, see below); chunk_len > 0
- *                fixes the segment length (rounded up to whole 64-step
- *                chunks), 0 lets the library choose; timeout_iters unused
- * Computed chunk by chunk (64 steps) as dense bf16 products with fp32
- * accumulation on the tensor cores; the carried state stays on chip.  With a
- * workspace of at least ss_ssd_fwd_workspace_bytes(dims, flags) bytes
- * (16-byte aligned) the library may also cut each sequence into up to 8
- * segments run in parallel, when batch x heads leaves SMs idle: a first pass
- * computes each segment's end state from zero, a fold makes every
- * segment's entering state exact, and the main pass runs the segments from
- * those (results equal to the unsplit scan up to rounding).  A NULL
- * workspace never splits; a smaller one is SS_ERR_WORKSPACE.
+ *                fixes the segment length (rounded up to whole chunks),
+ *                0 lets the library choose; timeout_iters unused
+ * Computed chunk by chunk as dense bf16 products with fp32 accumulation on
+ * the tensor cores, the carried state fp32 on chip: d_state 128 in 128-step
+ * chunks with tcgen05 MMAs (TMEM accumulators, TMA-staged tiles), d_state 64
+ * in 64-step chunks with warp-level MMAs.  With a workspace of at least
+ * ss_ssd_fwd_workspace_bytes(dims, flags) bytes (16-byte aligned; the call
+ * owns it until its work on the stream is done) the library may also cut
+ * each sequence into up to 8 segments run in parallel, when batch x heads
+ * leaves SMs idle: a first pass computes each segment's end state from
+ * zero, a fold makes every segment's entering state exact, and the main
+ * pass runs the segments from those (results equal to the unsplit scan up
+ * to rounding).  A NULL workspace never splits; a smaller one is
+ * SS_ERR_WORKSPACE.  The workspace's first word is a status word the call
+ * clears: the d_state 128 kernels bound every wait (2 s) and record
+ * SS_ERR_TIMEOUT there if one runs out; with SS_SYNC_CHECK the call
+ * synchronises the stream and returns that word.
  * Errors: SS_ERR_INVALID_ARG for NULL/misaligned pointers or sizes,
- * SS_ERR_UNSUPPORTED for headdim != 64 or d_state not 64 or 128. */
+ * SS_ERR_UNSUPPORTED for headdim != 64 or d_state not 64 or 128,
+ * SS_ERR_CUDA for a failed launch or (with SS_SYNC_CHECK) a stream error. */
 SS_API int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float* A, const void* B,
                       const void* C, const float* D, void* y, float* final_state, uint32_t flags,
                       const ss_ssd_dims* dims, const ss_launch* launch);
