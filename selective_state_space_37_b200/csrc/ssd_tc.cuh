@@ -23,15 +23,15 @@
 //       Y   = Mm X              128 x 64,  K = Q  -> TMEM columns [256, 320)
 //   warp 9: Δ, the prefix of Δ A and the decay factors, a chunk ahead into
 //     a double buffer;
-//   warps 0..7 (compute): two threads per TMEM lane (one time step t, or one
-//     state index n), each on half of the lane's columns: X̃ from x, the
-//     causal decay mask Mm from S, the state update, and the outputs
+//   warps 0..15 (compute): four threads per TMEM lane (one time step t, or
+//     one state index n), each on a quarter of the lane's columns: X̃ from x,
+//     the causal decay mask Mm from S, the state update, and the outputs
 //     y = Y + e^{cum_t} CG + D x, staged in shared memory and written by a
 //     bulk tensor store.
 // The warps hand work over through mbarriers, so the tensor core runs the
 // next chunk's C Bᵀ under this chunk's epilogue and Mm X under the state
 // update, and B and C of the next chunk load as soon as their last MMA is
-// done.  The carried state G stays fp32 in registers (the two threads of row
+// done.  The carried state G stays fp32 in registers (the four threads of row
 // n hold G[:, n]); the product with C reads it as two bf16 terms G_hi + G_lo,
 // so it is not rounded to bf16 before the readout.  Every wait is bounded: a
 // wait that runs out records SS error -4 in the status word and the CTA
@@ -53,10 +53,17 @@ constexpr int kQ = 128;            // chunk length (MMA M for the time rows)
 constexpr int kP = 64;             // head dimension
 constexpr int kN = 128;            // state width handled here
 constexpr int kRows = 128;         // TMEM lanes / tile rows
-constexpr int kComputeThreads = 256;   // warps 0..7; warps w and w + 4 share TMEM lanes 32 (w % 4) ..
-constexpr int kProducerWarp = 8;      // one thread: TMA loads and MMAs
-constexpr int kPrefixWarp = 9;        // the Δ prefix, a chunk ahead
+constexpr int kRT = 4;                // compute threads per tile row (warps w, w + 4, w + 8, w + 12
+                                      // share TMEM lanes 32 (w % 4) ..)
+constexpr int kComputeWarps = 4 * kRT;
+constexpr int kComputeThreads = 32 * kComputeWarps;
+constexpr int kPT = kP / kRT;         // a thread's columns of x, y and the state (16)
+constexpr int kXC = kPT / 8;          // its 16-byte chunks of a 64-column row (2)
+constexpr int kSB = (kQ / 32) / kRT;  // its 32-column blocks of the mask (1)
+constexpr int kProducerWarp = kComputeWarps;       // one thread: TMA loads and MMAs
+constexpr int kPrefixWarp = kComputeWarps + 1;     // the Δ prefix, a chunk ahead
 constexpr int kThreads = kComputeThreads + 64;
+static_assert(kComputeThreads == 512 && kSB == 1 && kXC == 2, "the barriers and splits below assume 4 threads per row");
 constexpr uint32_t kTmemCols = 512;   // allocation (power of two >= the 384 columns used)
 constexpr uint32_t kColS = 0, kColCG = 128, kColY = 256, kColG = 320;
 
@@ -155,6 +162,20 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // Shared-memory matrix descriptor: 128-byte swizzle, start / leading / stride
 // byte offsets in 16-byte units, descriptor version 1.
 __device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -216,21 +237,21 @@ __device__ __forceinline__ void sts128(uint32_t a, uint4 v) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
-// Barrier 1 over the 256 compute threads: true on every thread when `pred`
+// Barrier 1 over the 512 compute threads: true on every thread when `pred`
 // holds on any of them.
 __device__ __forceinline__ bool cw_any(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 1, 256, p;\n\t"
+        "bar.red.or.pred q, 1, 512, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
         : "r"(pred ? 1u : 0u)
         : "memory");
     return r != 0;
 }
-__device__ __forceinline__ void cw_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+__device__ __forceinline__ void cw_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
 // Grid: one CTA per (segment k, batch b, head h), blockIdx.x = (k * batch + b) * H + h;
 // STATE runs segments 0 .. nseg - 2 only (G_out from zero, no outputs).
@@ -277,7 +298,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     const uint64_t lim = p.wait_ns;
 
     if (tid == 0) {
-        for (int i = 0; i < 16; ++i) mbar_init(bars + i, (i == 8 || i == 9) ? 8u : 1u);
+        for (int i = 0; i < 16; ++i) mbar_init(bars + i, (i == 8 || i == 9) ? static_cast<uint32_t>(kComputeWarps) : 1u);
         fence_mbar_init();
     }
     if (warp == 0) {
@@ -477,19 +498,19 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     } else {
         // =============================================================== compute warps
         const int row = tid & (kRows - 1);   // TMEM lane / tile row of this thread
-        const int hf = tid >> 7;             // which half of the row's columns
+        const int qc = tid >> 7;             // which quarter of the row's columns
         const int rb = warp & 3;             // this warp's 32-row block
         const uint32_t lane_base = static_cast<uint32_t>(rb * 32) << 16;   // this warp's TMEM lanes
         const float Dh = p.D ? p.D[h] : 0.0f;
-        // Carried state: thread (n, hf) holds G[32 hf .. 32 hf + 31, n] (fp32).
+        // Carried state: thread (n, qc) holds G[16 qc .. 16 qc + 15, n] (fp32).
         // Entering a segment > 0 of the main pass it is the folded record, else zero.
-        float G[kP / 2];
+        float G[kPT];
         const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kP * kN : nullptr;
 #pragma unroll
-        for (int q = 0; q < kP / 2; ++q) G[q] = gin ? gin[(32 * hf + q) * kN + row] : 0.0f;
-        auto store_g = [&]() {   // bf16 hi / lo copies of G: row n, chunks 4 hf .. 4 hf + 3 of the [n][p] tiles
+        for (int q = 0; q < kPT; ++q) G[q] = gin ? gin[(kPT * qc + q) * kN + row] : 0.0f;
+        auto store_g = [&]() {   // bf16 hi / lo copies of G: row n, chunks 2 qc, 2 qc + 1 of the [n][p] tiles
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+            for (int c = 0; c < kXC; ++c) {
                 uint32_t hw[4], lw[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -497,15 +518,15 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                     hw[e] = pk(g0, g1);
                     lw[e] = pk(g0 - lo_f(hw[e]), g1 - hi_f(hw[e]));
                 }
-                sts128(chunk_addr(base + kOffGh, row, 4 * hf + c), make_uint4(hw[0], hw[1], hw[2], hw[3]));
-                sts128(chunk_addr(base + kOffGl, row, 4 * hf + c), make_uint4(lw[0], lw[1], lw[2], lw[3]));
+                sts128(chunk_addr(base + kOffGh, row, kXC * qc + c), make_uint4(hw[0], hw[1], hw[2], hw[3]));
+                sts128(chunk_addr(base + kOffGl, row, kXC * qc + c), make_uint4(lw[0], lw[1], lw[2], lw[3]));
             }
         };
         if (gin) store_g();
         if (!STATE) {   // Mm right of the diagonal is zero in every chunk: written once
             const int rb0 = warp & 3;
 #pragma unroll 1
-            for (int g = 2 * hf; g < 2 * hf + 2; ++g) {
+            for (int g = kSB * qc; g < kSB * qc + kSB; ++g) {
                 if (g <= rb0) continue;
                 const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
 #pragma unroll
@@ -545,14 +566,14 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
             const float cum_end = cum[kQ - 1];
             if (STATE) esum += cum_end;
 
-            {   // -------- X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s, chunks 4 hf .. 4 hf + 3; a per-row
+            {   // -------- X̃[s, :] = e^{cum_end - cum_s} Δ_s x_s (row s, chunks 2 qc, 2 qc + 1; a per-row
                 // scale, so every 16-byte chunk keeps its place; addressed through the swizzle so that eight
                 // consecutive rows hit eight bank groups).  X̃ was last read by the previous chunk's Bᵀ X̃,
                 // waited for below.
                 const int sr = row;
                 const float w = wx2[xb * kQ + sr];
 #pragma unroll
-                for (int c = 4 * hf; c < 4 * hf + 4; ++c) {
+                for (int c = kXC * qc; c < kXC * qc + kXC; ++c) {
                     const uint4 v = lds128(chunk_addr(xbase, sr, c));
                     const uint4 o = make_uint4(pk(lo_f(v.x) * w, hi_f(v.x) * w), pk(lo_f(v.y) * w, hi_f(v.y) * w),
                                                pk(lo_f(v.z) * w, hi_f(v.z) * w), pk(lo_f(v.w) * w, hi_f(v.w) * w));
@@ -563,7 +584,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                 if (lane == 0) mbar_arrive(xt_ready);
             }
             if (!STATE) {
-                // -------- Mm = S ∘ decay mask (row t, 32-column blocks 2 hf, 2 hf + 1).  Blocks right of the
+                // -------- Mm = S ∘ decay mask (row t, 32-column block qc).  Blocks right of the
                 // diagonal are zero.  Strictly below it every s <= t, and the decay factors through the
                 // block's last step r: e^{cum_t - cum_s} = e^{cum_t - cum_r} e^{cum_r - cum_s}, both factors
                 // between the exact value and 1, so neither overflows nor loses the product.  The diagonal
@@ -573,8 +594,8 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                 const int t = row;
                 const float ct = cs[t];
 #pragma unroll 1
-                for (int gi = 0; gi < 2; ++gi) {
-                    const int g = 2 * hf + gi;
+                for (int gi = 0; gi < kSB; ++gi) {
+                    const int g = kSB * qc + gi;
                     const uint32_t blk = base + kOffM + static_cast<uint32_t>(g >> 1) * 16384u;
                     const int c0 = (g & 1) * 4;
                     if (g > rb) continue;   // zero, written before the first chunk
@@ -628,40 +649,40 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                 __syncwarp();
                 if (lane == 0) mbar_arrive(mm_ready);
             }
-            // -------- G = e^{cum_end} G + ΔGᵀ[n, :] (row n, columns 32 hf .. 32 hf + 31), once Bᵀ X̃ is
+            // -------- G = e^{cum_end} G + ΔGᵀ[n, :] (row n, columns 16 qc .. 16 qc + 15), once Bᵀ X̃ is
             // done and C Gᵀ has read the previous copies of G
             if (!cw_wait2(STATE ? nullptr : cg_done, par, dg_done, par)) break;
             tc_fence_after();
             {
                 const float e_end = __expf(cum_end);
-                float dg[32];
-                tmem_ld32(tmem + lane_base + kColG + 32 * hf, dg);
+                float dg[kPT];
+                tmem_ld16(tmem + lane_base + kColG + kPT * qc, dg);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) G[j] = fmaf(e_end, G[j], dg[j]);
+                for (int j = 0; j < kPT; ++j) G[j] = fmaf(e_end, G[j], dg[j]);
                 if (!STATE) store_g();
             }
             if (!STATE) {
-                // -------- y = Y + e^{cum_t} CG + D x (row t, columns 32 hf .. 32 hf + 31) into the staging tile
+                // -------- y = Y + e^{cum_t} CG + D x (row t, columns 16 qc .. 16 qc + 15) into the staging tile
                 if (tid == 0) bulk_wait_read0();   // the previous chunk's y tile has left shared memory
                 if (!cw_wait2(y_done, par, nullptr, 0)) break;
                 tc_fence_after();
                 const int t = row;
                 const float et = __expf(cum[t]);
-                float acc[32], gv[32];
-                tmem_ld32(tmem + lane_base + kColY + 32 * hf, acc);
+                float acc[kPT], gv[kPT];
+                tmem_ld16(tmem + lane_base + kColY + kPT * qc, acc);
                 if (carry) {
-                    tmem_ld32(tmem + lane_base + kColCG + 32 * hf, gv);   // C G_hiᵀ
+                    tmem_ld16(tmem + lane_base + kColCG + kPT * qc, gv);   // C G_hiᵀ
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
-                    tmem_ld32(tmem + lane_base + kColCG + 64 + 32 * hf, gv);   // C G_loᵀ
+                    for (int j = 0; j < kPT; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
+                    tmem_ld16(tmem + lane_base + kColCG + 64 + kPT * qc, gv);   // C G_loᵀ
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
+                    for (int j = 0; j < kPT; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
                 }
-                uint4 xv[4];
+                uint4 xv[kXC];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) xv[c] = lds128(chunk_addr(xbase, t, 4 * hf + c));
+                for (int c = 0; c < kXC; ++c) xv[c] = lds128(chunk_addr(xbase, t, kXC * qc + c));
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int c = 0; c < kXC; ++c) {
                     const uint32_t xw[4] = {xv[c].x, xv[c].y, xv[c].z, xv[c].w};
                     uint32_t ow[4];
 #pragma unroll
@@ -669,7 +690,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                         const int j = 8 * c + 2 * e;
                         ow[e] = pk(fmaf(Dh, lo_f(xw[e]), acc[j]), fmaf(Dh, hi_f(xw[e]), acc[j + 1]));
                     }
-                    sts128(chunk_addr(base + kOffY, t, 4 * hf + c), make_uint4(ow[0], ow[1], ow[2], ow[3]));
+                    sts128(chunk_addr(base + kOffY, t, kXC * qc + c), make_uint4(ow[0], ow[1], ow[2], ow[3]));
                 }
             }
             fence_proxy_async_smem();   // G copies and the y tile before the async proxy reads them
@@ -691,7 +712,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
             else if (p.final_state && sg == p.nseg - 1) out = p.final_state + bh * kP * kN;
             if (out) {
 #pragma unroll
-                for (int q2 = 0; q2 < kP / 2; ++q2) out[(32 * hf + q2) * kN + row] = G[q2];
+                for (int q2 = 0; q2 < kPT; ++q2) out[(kPT * qc + q2) * kN + row] = G[q2];
             }
             if (STATE && tid == 0) p.esum[bh * p.nseg + sg] = esum;
         }
