@@ -85,8 +85,10 @@ typedef struct ss_dims {
  *                   ss_step does not use it.
  *   workspace_bytes its size.
  *   timeout_iters   bound on the polls of one cross-chunk wait (0: library
- *                   default, about one second).  When it runs out the call
- *                   records SS_ERR_TIMEOUT and finishes without hanging.
+ *                   default, about one second); for ss_ssd_fwd with d_state
+ *                   128, the bound on one wait in microseconds (0: two
+ *                   seconds).  When it runs out the call records
+ *                   SS_ERR_TIMEOUT and finishes without hanging.
  *   chunk_len       timesteps per time chunk; 0 lets the library choose.  Any
  *                   positive value is accepted (it is rounded up to a multiple
  *                   of the 32-step tile); results agree up to rounding. */
@@ -116,7 +118,9 @@ enum {
     SS_FORCE_GENERAL_A = 1u << 3,  /* skip the A[d,n] = a_d (n+1) fast path even when A has that form */
     SS_TEST_DROP_CARRY = 1u << 30  /* TEST ONLY: the first chunk of batch 0, channel block 0 never
                                       publishes its carry, so its successor's bounded wait runs out
-                                      (exercises SS_ERR_TIMEOUT without a hang) */
+                                      (exercises SS_ERR_TIMEOUT without a hang); in ss_ssd_fwd
+                                      (d_state 128) the first CTA never signals its first C Bᵀ
+                                      product, so its compute warps' wait runs out */
 };
 
 /* ss_fwd -- selective-scan forward pass over [batch, seqlen] tokens.
@@ -248,10 +252,12 @@ typedef struct ss_ssd_dims {
  *   A            [nheads] fp32 (negative); dt_bias, D [nheads] fp32 or NULL
  *   B, C         [batch, seqlen, d_state] bf16
  *   final_state  [batch, nheads, headdim, d_state] fp32 or NULL
- *   flags        SS_DELTA_SOFTPLUS, SS_SYNC_CHECK (bf16 only; SS_BF16 ignored)
+ *   flags        SS_DELTA_SOFTPLUS, SS_SYNC_CHECK (bf16 only; SS_BF16 ignored);
+ *                SS_TEST_DROP_CARRY for tests (d_state 128)
  *   launch       stream; workspace (optional, see below); chunk_len > 0
  *                fixes the segment length (rounded up to whole chunks),
- *                0 lets the library choose; timeout_iters unused
+ *                0 lets the library choose; timeout_iters (d_state 128) the
+ *                bound on one wait in microseconds, 0 for two seconds
  * Computed chunk by chunk as dense bf16 products with fp32 accumulation on
  * the tensor cores, the carried state fp32 on chip: d_state 128 in 128-step
  * chunks with tcgen05 MMAs (TMEM accumulators, TMA-staged tiles), d_state 64

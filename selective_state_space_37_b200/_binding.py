@@ -514,13 +514,16 @@ def ss_block_fwd(hidden, weights, *, out=None, scratch=None, stream=None):
 
 
 def ss_ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, *, softplus=True, y=None, final_state=None,
-               return_final_state=True, chunk_len=0, split=True, workspace=None, stream=None, sync_check=False):
+               return_final_state=True, chunk_len=0, split=True, workspace=None, stream=None, sync_check=False,
+               timeout_iters=0, extra_flags=0):
     """Multi-head scan with a scalar decay per head (Mamba-2's SSD model).
     x [batch, L, nheads, 64] bf16; dt [batch, L, nheads] bf16; A [nheads] fp32;
     B, C [batch, L, d_state] bf16 (d_state 64 or 128); D, dt_bias [nheads] fp32
     or None.  Returns (y [batch, L, nheads, 64] bf16, final_state
     [batch, nheads, 64, d_state] fp32 or None).  split=False runs every
-    sequence whole (no workspace); chunk_len > 0 fixes the segment length."""
+    sequence whole (no workspace); chunk_len > 0 fixes the segment length;
+    timeout_iters (d_state 128) bounds one wait in microseconds (0: two
+    seconds); extra_flags adds raw SS_* flags (SS_TEST_DROP_CARRY in tests)."""
     batch, L, H, P = x.shape
     N = B.shape[-1]
     dev = x.device
@@ -538,16 +541,16 @@ def ss_ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, *, softplus=True, y=None, f
     if final_state is None and return_final_state:
         final_state = torch.empty((batch, H, P, N), dtype=torch.float32, device=dev)
     _check(final_state, "final_state", (batch, H, P, N), torch.float32, dev)
-    flags = (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0)
+    flags = (SS_DELTA_SOFTPLUS if softplus else 0) | (SS_SYNC_CHECK if sync_check else 0) | int(extra_flags)
     dims = ss_ssd_dims(batch, L, H, P, N)
     sh = _stream_handle(stream, dev)
     if split:
         if workspace is None:
             workspace = workspace_for(int(lib().ss_ssd_fwd_workspace_bytes(ctypes.byref(dims), flags)), dev, sh)
-        launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(), 0,
-                           int(chunk_len))
+        launch = ss_launch(sh, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                           int(timeout_iters), int(chunk_len))
     else:
-        launch = ss_launch(sh, None, 0, 0, int(chunk_len))
+        launch = ss_launch(sh, None, 0, int(timeout_iters), int(chunk_len))
     rc = lib().ss_ssd_fwd(_ptr(x), _ptr(dt), _ptr(dt_bias), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
                           _ptr(final_state), flags, ctypes.byref(dims), ctypes.byref(launch))
     if rc != SS_OK:

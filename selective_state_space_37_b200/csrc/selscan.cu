@@ -1070,7 +1070,9 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
             q.rec = p.rec; q.esum = p.esum;
             q.status = have_ws ? static_cast<uint32_t*>(launch->workspace) : nullptr;
             q.L = L; q.batch = p.batch; q.H = p.H; q.softplus = p.softplus;
-            q.wait_ns = kTmaWaitNs;
+            q.test_drop = (flags & SS_TEST_DROP_CARRY) ? 1 : 0;
+            q.wait_ns = launch->timeout_iters ? static_cast<uint64_t>(launch->timeout_iters) * 1000ull : kTmaWaitNs;
+            q.drain_ns = kTmaWaitNs;
             rc = launch_ssd_tc(q, p, x, B, C, items, w, launch->chunk_len, have_ws, stream);
         }
     } else {

@@ -111,7 +111,9 @@ struct Params {
     int64_t L;
     int batch, H, nseg, cseg;  // cseg: chunks of kQ steps per segment
     int softplus;
-    uint64_t wait_ns;
+    int test_drop;             // test only: CTA 0 never signals its first C Bᵀ (a wait runs out)
+    uint64_t wait_ns;          // bound on one hand-over wait
+    uint64_t drain_ns;         // bound on the wind-down waits (copies in flight, the last MMAs)
 };
 
 // ------------------------------------------------------------ tcgen05 / TMA
@@ -371,7 +373,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                         umma(tmem + kColS, sdesc(base + kOffC + off, 16, 1024), sdesc(base + kOffB + off, 16, 1024),
                              kIdesc_128x128_KK, k > 0);
                     }
-                    umma_commit(s_full);
+                    if (!(p.test_drop && blockIdx.x == 0 && ci == 0)) umma_commit(s_full);
                 }
                 // the previous chunk's epilogue (for ci = 0, the compute warps' set-up)
                 if (!pw_wait(ep_done, par)) break;
@@ -727,12 +729,13 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     // (both bounded; a completed phase is recognised as well).
     __syncthreads();
     if (warp == kProducerWarp && lane == 0) {
+        const uint64_t dlim = p.drain_ns;
         for (int cj = *xw_slot; cj < x_issued; ++cj)   // chunk cj's x: buffer cj & 1, phase cj >> 1
-            mbar_wait_bounded(x_full + (cj & 1), static_cast<uint32_t>((cj >> 1) & 1), lim);
-        if (b_waited < b_issued) mbar_wait_bounded(b_full, static_cast<uint32_t>(b_waited & 1), lim);
-        if (c_waited < c_issued) mbar_wait_bounded(c_full, static_cast<uint32_t>(c_waited & 1), lim);
+            mbar_wait_bounded(x_full + (cj & 1), static_cast<uint32_t>((cj >> 1) & 1), dlim);
+        if (b_waited < b_issued) mbar_wait_bounded(b_full, static_cast<uint32_t>(b_waited & 1), dlim);
+        if (c_waited < c_issued) mbar_wait_bounded(c_full, static_cast<uint32_t>(c_waited & 1), dlim);
         umma_commit(fin_bar);
-        mbar_wait_bounded(fin_bar, 0, lim);
+        mbar_wait_bounded(fin_bar, 0, dlim);
     }
     tc_fence_before();
     __syncthreads();

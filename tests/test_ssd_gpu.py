@@ -115,3 +115,26 @@ def test_ssd_mamba2_130m_full():
     y, st, yr, sr = run_and_ref(inp)
     assert rel_max_err(to_f64(y), yr) <= TOL
     assert rel_max_err(to_f64(st), sr) <= TOL
+
+
+def test_ssd_bounded_wait_reports_timeout_and_context_survives():
+    """d_state 128: a hand-over that is never signalled (SS_TEST_DROP_CARRY:
+    the first CTA's first C Bᵀ completion) makes the compute warps' bounded
+    wait run out, and with it the producer's wait for their mask.  The call
+    reports SS_ERR_TIMEOUT through the workspace's status word (no hang, no
+    trap: copies in flight are drained, MMAs completed and TMEM released
+    before the CTA ends), and the next call on the same context is correct."""
+    inp = ssd_inputs(2, 300, 3, 128, seed=77, device=DEV)
+    dims = ss.ss_ssd_dims(2, 300, 3, 64, 128)
+    nb = int(ss.lib().ss_ssd_fwd_workspace_bytes(ctypes.byref(dims), 0))
+    ws = torch.zeros(nb, dtype=torch.uint8, device=DEV)
+    args = (inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"])
+    kw = dict(D=inp["D"], dt_bias=inp["dt_bias"], workspace=ws)
+    ss.ss_ssd_fwd(*args, **kw, timeout_iters=200, extra_flags=ss.SS_TEST_DROP_CARRY)
+    assert ss.ss_check(ws) == ss.SS_ERR_TIMEOUT
+    y, st = ss.ss_ssd_fwd(*args, **kw, sync_check=True)
+    assert ss.ss_check(ws) == ss.SS_OK
+    yr, sr = oracle.ssd(to_f64(inp["x"]), to_f64(inp["dt"]), to_f64(inp["A"]), to_f64(inp["B"]),
+                        to_f64(inp["C"]), D=to_f64(inp["D"]), dt_bias=to_f64(inp["dt_bias"]), softplus=True)
+    assert rel_max_err(to_f64(y), yr) <= TOL
+    assert rel_max_err(to_f64(st), sr) <= TOL
