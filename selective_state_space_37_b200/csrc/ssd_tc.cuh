@@ -164,6 +164,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// Two 16-column ranges of this thread's TMEM lane, one wait.
+__device__ __forceinline__ void tmem_ld16x2(uint32_t a0, uint32_t a1, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, "
+        "%29, %30, %31}, [%33];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(a0), "r"(a1)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
     uint32_t r[16];
     asm volatile(
@@ -670,12 +688,15 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                 tc_fence_after();
                 const int t = row;
                 const float et = __expf(cum[t]);
-                float acc[kPT], gv[kPT];
-                tmem_ld16(tmem + lane_base + kColY + kPT * qc, acc);
-                if (carry) {
-                    tmem_ld16(tmem + lane_base + kColCG + kPT * qc, gv);   // C G_hiᵀ
+                float acc[kPT];
+                {   // Y and C G_hiᵀ in one TMEM round trip, then C G_loᵀ
+                    float yg[2 * kPT];
+                    tmem_ld16x2(tmem + lane_base + kColY + kPT * qc, tmem + lane_base + kColCG + kPT * qc, yg);
 #pragma unroll
-                    for (int j = 0; j < kPT; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
+                    for (int j = 0; j < kPT; ++j) acc[j] = carry ? fmaf(et, yg[kPT + j], yg[j]) : yg[j];
+                }
+                if (carry) {
+                    float gv[kPT];
                     tmem_ld16(tmem + lane_base + kColCG + 64 + kPT * qc, gv);   // C G_loᵀ
 #pragma unroll
                     for (int j = 0; j < kPT; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
