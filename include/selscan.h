@@ -85,9 +85,8 @@ typedef struct ss_dims {
  *                   ss_step does not use it.
  *   workspace_bytes its size.
  *   timeout_iters   bound on the polls of one cross-chunk wait (0: library
- *                   default, about one second); for ss_ssd_fwd with d_state
- *                   128, the bound on one wait in microseconds (0: two
- *                   seconds).  When it runs out the call records
+ *                   default, about one second); for ss_ssd_fwd, the bound on
+ *                   one wait in microseconds (0: two seconds).  When it runs out the call records
  *                   SS_ERR_TIMEOUT and finishes without hanging.
  *   chunk_len       timesteps per time chunk; 0 lets the library choose.  Any
  *                   positive value is accepted (it is rounded up to a multiple
@@ -119,8 +118,8 @@ enum {
     SS_TEST_DROP_CARRY = 1u << 30  /* TEST ONLY: the first chunk of batch 0, channel block 0 never
                                       publishes its carry, so its successor's bounded wait runs out
                                       (exercises SS_ERR_TIMEOUT without a hang); in ss_ssd_fwd
-                                      (d_state 128) the first CTA never signals its first C Bᵀ
-                                      product, so its compute warps' wait runs out */
+                                      the first CTA never signals its first C Bᵀ product, so its
+                                      compute warps' wait runs out */
 };
 
 /* ss_fwd -- selective-scan forward pass over [batch, seqlen] tokens.
@@ -253,15 +252,15 @@ typedef struct ss_ssd_dims {
  *   B, C         [batch, seqlen, d_state] bf16
  *   final_state  [batch, nheads, headdim, d_state] fp32 or NULL
  *   flags        SS_DELTA_SOFTPLUS, SS_SYNC_CHECK (bf16 only; SS_BF16 ignored);
- *                SS_TEST_DROP_CARRY for tests (d_state 128)
+ *                SS_TEST_DROP_CARRY for tests
  *   launch       stream; workspace (optional, see below); chunk_len > 0
  *                fixes the segment length (rounded up to whole chunks),
- *                0 lets the library choose; timeout_iters (d_state 128) the
- *                bound on one wait in microseconds, 0 for two seconds
- * Computed chunk by chunk as dense bf16 products with fp32 accumulation on
- * the tensor cores, the carried state fp32 on chip: d_state 128 in 128-step
- * chunks with tcgen05 MMAs (TMEM accumulators, TMA-staged tiles), d_state 64
- * in 64-step chunks with warp-level MMAs.  With a workspace of at least
+ *                0 lets the library choose; timeout_iters the bound on one
+ *                wait in microseconds, 0 for two seconds
+ * Computed chunk by chunk (128 steps) as dense bf16 products with fp32
+ * accumulation on the tensor cores -- tcgen05 MMAs, TMEM accumulators,
+ * TMA-staged tiles -- the carried state fp32 on chip; d_state 64 runs the
+ * same kernel with B, C and the state padded to 128 with zeros.  With a workspace of at least
  * ss_ssd_fwd_workspace_bytes(dims, flags) bytes (16-byte aligned; the call
  * owns it until its work on the stream is done) the library may also cut
  * each sequence into up to 8 segments run in parallel, when batch x heads
@@ -270,7 +269,7 @@ typedef struct ss_ssd_dims {
  * pass runs the segments from those (results equal to the unsplit scan up
  * to rounding).  A NULL workspace never splits; a smaller one is
  * SS_ERR_WORKSPACE.  The workspace's first word is a status word the call
- * clears: the d_state 128 kernels bound every wait (2 s) and record
+ * clears: the kernels bound every wait (2 s) and record
  * SS_ERR_TIMEOUT there if one runs out; with SS_SYNC_CHECK the call
  * synchronises the stream and returns that word.
  * Errors: SS_ERR_INVALID_ARG for NULL/misaligned pointers or sizes,

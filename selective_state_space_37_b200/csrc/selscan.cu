@@ -231,8 +231,8 @@ SsdLayout ssd_layout(const ss_ssd_dims* d) {
     return w;
 }
 
-// SELSCAN_SSD_MMA_SYNC=1 builds the d_state 128 scan on the warp-level
-// mma.sync kernel of ssd.cuh instead of the tcgen05 one (comparisons).
+// SELSCAN_SSD_MMA_SYNC=1 builds the SSD scan on the warp-level mma.sync
+// kernel of ssd.cuh instead of the tcgen05 one (comparisons).
 #ifndef SELSCAN_SSD_MMA_SYNC
 #define SELSCAN_SSD_MMA_SYNC 0
 #endif
@@ -302,9 +302,10 @@ int launch_ssd_tc(const tc::Params& base_p, const SsdParams& fold_p, const void*
         const cuuint64_t sx[3] = {static_cast<cuuint64_t>(tc::kP * 2), static_cast<cuuint64_t>(H * tc::kP * 2),
                                   static_cast<cuuint64_t>(L * H * tc::kP * 2)};
         const cuuint32_t bx[4] = {64, 1, static_cast<cuuint32_t>(tc::kQ), 1};
-        const cuuint64_t db[3] = {static_cast<cuuint64_t>(tc::kN), static_cast<cuuint64_t>(L),
+        const int64_t N = p.n;   // 128, or 64 (one 64-wide box per row)
+        const cuuint64_t db[3] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(L),
                                   static_cast<cuuint64_t>(batch)};
-        const cuuint64_t sb[2] = {static_cast<cuuint64_t>(tc::kN * 2), static_cast<cuuint64_t>(L * tc::kN * 2)};
+        const cuuint64_t sb[2] = {static_cast<cuuint64_t>(N * 2), static_cast<cuuint64_t>(L * N * 2)};
         const cuuint32_t bb[3] = {64, static_cast<cuuint32_t>(tc::kQ), 1};
         if (!make_map_sw128(&mx, x, 4, dx, sx, bx) || !make_map_sw128(&mb, B, 3, db, sb, bb) ||
             !make_map_sw128(&mc, C, 3, db, sb, bb) || !make_map_sw128(&my, p.y, 4, dx, sx, bx))
@@ -314,9 +315,10 @@ int launch_ssd_tc(const tc::Params& base_p, const SsdParams& fold_p, const void*
         kstate<<<static_cast<unsigned>(items * (nseg - 1)), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
         SsdParams f = fold_p;
         f.nseg = nseg;
-        const int64_t total = items * kSsdP * tc::kN;
+        const int64_t total = items * kSsdP * p.n;
         const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), 4096);
-        ss_ssd_fold_kernel<tc::kN><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(f);
+        if (p.n == tc::kN) ss_ssd_fold_kernel<tc::kN><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(f);
+        else ss_ssd_fold_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(f);
     }
     kmain<<<static_cast<unsigned>(items * nseg), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
@@ -1057,11 +1059,11 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
     p.softplus = (flags & SS_DELTA_SOFTPLUS) ? 1 : 0;
     const int64_t items = batch * H;
     int rc;
-    if (dims->d_state == 128 && !SELSCAN_SSD_MMA_SYNC) {
+    if (!SELSCAN_SSD_MMA_SYNC) {
         if (L == 0) {   // no steps: the final state is zero
             if (final_state &&
-                cudaMemsetAsync(final_state, 0, static_cast<size_t>(items * kSsdP * 128) * sizeof(float), stream) !=
-                    cudaSuccess)
+                cudaMemsetAsync(final_state, 0, static_cast<size_t>(items * kSsdP * dims->d_state) * sizeof(float),
+                                stream) != cudaSuccess)
                 return SS_ERR_CUDA;
             rc = SS_OK;
         } else {
@@ -1070,6 +1072,7 @@ int ss_ssd_fwd(const void* x, const void* dt, const float* dt_bias, const float*
             q.rec = p.rec; q.esum = p.esum;
             q.status = have_ws ? static_cast<uint32_t*>(launch->workspace) : nullptr;
             q.L = L; q.batch = p.batch; q.H = p.H; q.softplus = p.softplus;
+            q.n = static_cast<int>(dims->d_state);
             q.test_drop = (flags & SS_TEST_DROP_CARRY) ? 1 : 0;
             q.wait_ns = launch->timeout_iters ? static_cast<uint64_t>(launch->timeout_iters) * 1000ull : kTmaWaitNs;
             q.drain_ns = kTmaWaitNs;

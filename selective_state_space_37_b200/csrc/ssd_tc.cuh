@@ -110,6 +110,7 @@ struct Params {
     uint32_t* status;          // error word or null
     int64_t L;
     int batch, H, nseg, cseg;  // cseg: chunks of kQ steps per segment
+    int n;                     // d_state: 128, or 64 (B, C and the state padded to 128 with zeros)
     int softplus;
     int test_drop;             // test only: CTA 0 never signals its first C Bᵀ (a wait runs out)
     uint64_t wait_ns;          // bound on one hand-over wait
@@ -325,6 +326,13 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
         tmem_alloc(tmem_slot, kTmemCols);
         tmem_relinquish();
     }
+    if (p.n < kN) {   // d_state 64: B and C keep their second 64-column block at zero (TMA fills the first)
+        for (int i = tid; i < 2 * 1024; i += kThreads) {
+            const uint32_t blk = (i < 1024) ? kOffB + 16384u : kOffC + 16384u;
+            sts128(base + blk + static_cast<uint32_t>(i & 1023) * 16u, make_uint4(0, 0, 0, 0));
+        }
+        fence_proxy_async_smem();   // before the MMAs read them (ordered by the barrier below)
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -347,15 +355,16 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                 mbar_arrive_expect_tx(bar, kQ * kP * 2);
                 tma_load_4d(base + ((ci & 1) ? kOffX1 : kOffX0), &tm_x, 0, h, chunk_t0(ci), b, bar);
             };
+            const bool two = p.n == kN;   // B and C rows of 128 states: two 64-wide boxes
             auto issue_b = [&](int ci) {
-                mbar_arrive_expect_tx(b_full, 2 * kQ * 64 * 2);
+                mbar_arrive_expect_tx(b_full, (two ? 2 : 1) * kQ * 64 * 2);
                 tma_load_3d_u(base + kOffB, &tm_B, 0, chunk_t0(ci), b, b_full);
-                tma_load_3d_u(base + kOffB + 16384, &tm_B, 64, chunk_t0(ci), b, b_full);
+                if (two) tma_load_3d_u(base + kOffB + 16384, &tm_B, 64, chunk_t0(ci), b, b_full);
             };
             auto issue_c = [&](int ci) {
-                mbar_arrive_expect_tx(c_full, 2 * kQ * 64 * 2);
+                mbar_arrive_expect_tx(c_full, (two ? 2 : 1) * kQ * 64 * 2);
                 tma_load_3d_u(base + kOffC, &tm_C, 0, chunk_t0(ci), b, c_full);
-                tma_load_3d_u(base + kOffC + 16384, &tm_C, 64, chunk_t0(ci), b, c_full);
+                if (two) tma_load_3d_u(base + kOffC + 16384, &tm_C, 64, chunk_t0(ci), b, c_full);
             };
             auto pw_wait = [&](uint64_t* bar, uint32_t parity) {
                 if (mbar_wait_bounded(bar, parity, lim)) return true;
@@ -524,10 +533,12 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
         const float Dh = p.D ? p.D[h] : 0.0f;
         // Carried state: thread (n, qc) holds G[16 qc .. 16 qc + 15, n] (fp32).
         // Entering a segment > 0 of the main pass it is the folded record, else zero.
+        // (d_state 64: rows n >= 64 stay zero -- their B and C columns are zero)
         float G[kPT];
-        const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kP * kN : nullptr;
+        const int nn = p.n;
+        const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kP * nn : nullptr;
 #pragma unroll
-        for (int q = 0; q < kPT; ++q) G[q] = gin ? gin[(kPT * qc + q) * kN + row] : 0.0f;
+        for (int q = 0; q < kPT; ++q) G[q] = (gin && row < nn) ? gin[(kPT * qc + q) * nn + row] : 0.0f;
         auto store_g = [&]() {   // bf16 hi / lo copies of G: row n, chunks 2 qc, 2 qc + 1 of the [n][p] tiles
 #pragma unroll
             for (int c = 0; c < kXC; ++c) {
@@ -731,11 +742,11 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
         // outputs of the state: the segment's G_out (state pass) or the final state
         if (ok) {
             float* out = nullptr;
-            if (STATE) out = p.rec + (bh * (p.nseg - 1) + sg) * kP * kN;
-            else if (p.final_state && sg == p.nseg - 1) out = p.final_state + bh * kP * kN;
-            if (out) {
+            if (STATE) out = p.rec + (bh * (p.nseg - 1) + sg) * kP * nn;
+            else if (p.final_state && sg == p.nseg - 1) out = p.final_state + bh * kP * nn;
+            if (out && row < nn) {
 #pragma unroll
-                for (int q2 = 0; q2 < kPT; ++q2) out[(kPT * qc + q2) * kN + row] = G[q2];
+                for (int q2 = 0; q2 < kPT; ++q2) out[(kPT * qc + q2) * nn + row] = G[q2];
             }
             if (STATE && tid == 0) p.esum[bh * p.nseg + sg] = esum;
         }

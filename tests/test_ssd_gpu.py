@@ -1,8 +1,9 @@
 """GPU parity of ss_ssd_fwd (multi-head scalar-decay scan, tensor cores)
 against oracle.ssd (fp64 recurrence, pinned in test_oracle_ssd_pins.py).
 Bound: max|y - y_ref| <= 2e-2 · max|y_ref| and the same for the final state
--- the kernel rounds the decay-weighted C Bᵀ, the scaled B and the carried
-state's copy to bf16 (2^-9 relative each) before the tensor-core products."""
+-- the products' operands are bf16 (the masked C Bᵀ, X̃ and the carried
+state's hi/lo pair round to 2^-9 relative each), accumulation fp32.  Both
+d_state 64 (padded) and 128 run the tcgen05 kernel."""
 import ctypes
 
 import numpy as np
