@@ -522,7 +522,7 @@ def ss_ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, *, softplus=True, y=None, f
     or None.  Returns (y [batch, L, nheads, 64] bf16, final_state
     [batch, nheads, 64, d_state] fp32 or None).  split=False runs every
     sequence whole (no workspace); chunk_len > 0 fixes the segment length;
-    timeout_iters (d_state 128) bounds one wait in microseconds (0: two
+    timeout_iters bounds one wait in microseconds (0: two
     seconds); extra_flags adds raw SS_* flags (SS_TEST_DROP_CARRY in tests)."""
     batch, L, H, P = x.shape
     N = B.shape[-1]
