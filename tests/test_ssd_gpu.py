@@ -82,7 +82,7 @@ def test_ssd_full_size_sampled_heads():
     torch.cuda.empty_cache()
 
 
-# Forced time segments (the segment length rounds up to whole 64-step
+# Forced time segments (the segment length rounds up to whole 128-step
 # chunks): 2 .. 8 segments, ragged last chunk and segment, both state widths;
 # the state pass, the fold and the main pass must carry the state exactly.
 SEGS = [((2, 1000, 3, 128), 128), ((1, 333, 2, 64), 64), ((3, 700, 2, 128), 200), ((1, 4096, 1, 64), 512)]
@@ -95,6 +95,52 @@ def test_ssd_time_segments(shape, seg):
     y, st, yr, sr = run_and_ref(inp, chunk_len=seg)
     assert rel_max_err(to_f64(y), yr) <= TOL
     assert rel_max_err(to_f64(st), sr) <= TOL
+
+
+# Chunk boundaries of the 128-step chunks: one step short, exact, one over,
+# two chunks, three chunks and one step; both state widths (64 is padded).
+EDGES = [(L, N) for L in (127, 128, 129, 256, 385) for N in (64, 128)]
+
+
+@pytest.mark.parametrize("L,N", EDGES, ids=[f"L{l}_N{n}" for l, n in EDGES])
+def test_ssd_chunk_boundaries(L, N):
+    inp = ssd_inputs(1, L, 2, N, seed=900 + L + N, device=DEV)
+    y, st, yr, sr = run_and_ref(inp)
+    assert rel_max_err(to_f64(y), yr) <= TOL
+    assert rel_max_err(to_f64(st), sr) <= TOL
+
+
+def test_ssd_extreme_decays():
+    """Three heads: a fast decay with large steps (A = -30, Δ around 5, so
+    e^{cum} underflows within a few steps and the mask's factored decays
+    underflow with it), a near-zero decay rate and no decay at all (A = 0: the
+    state sums every input of the sequence)."""
+    inp = ssd_inputs(2, 300, 3, 128, seed=41, device=DEV)
+    inp["A"] = torch.tensor([-30.0, -1e-3, 0.0], dtype=torch.float32, device=DEV)
+    inp["dt_bias"] = torch.tensor([5.0, -2.0, -3.0], dtype=torch.float32, device=DEV)
+    y, st, yr, sr = run_and_ref(inp)
+    for h in range(3):
+        assert rel_max_err(to_f64(y[:, :, h]), yr[:, :, h]) <= TOL, h
+        assert rel_max_err(to_f64(st[:, h]), sr[:, h]) <= TOL, h
+
+
+def test_ssd_full_size_sampled_heads_dstate64():
+    """The padded d_state 64 path at the 2.7B layer's size (batch 4, L 8192,
+    80 heads), sampled (batch, head) pairs against the oracle."""
+    b, L, H, N = 4, 8192, 80, 64
+    inp = ssd_inputs(b, L, H, N, seed=13, device=DEV)
+    y, st = ss.ss_ssd_fwd(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], D=inp["D"], dt_bias=inp["dt_bias"],
+                          sync_check=True)
+    rng = np.random.default_rng(9)
+    picks = [(int(rng.integers(b)), int(h)) for h in rng.choice(H, size=4, replace=False)]
+    for bi, h in picks:
+        yr, sr = oracle.ssd(to_f64(inp["x"][bi:bi + 1, :, h:h + 1]), to_f64(inp["dt"][bi:bi + 1, :, h:h + 1]),
+                            to_f64(inp["A"][h:h + 1]), to_f64(inp["B"][bi:bi + 1]), to_f64(inp["C"][bi:bi + 1]),
+                            D=to_f64(inp["D"][h:h + 1]), dt_bias=to_f64(inp["dt_bias"][h:h + 1]))
+        assert rel_max_err(to_f64(y[bi:bi + 1, :, h:h + 1]), yr) <= TOL, (bi, h)
+        assert rel_max_err(to_f64(st[bi:bi + 1, h:h + 1]), sr) <= TOL, (bi, h)
+    del inp, y, st
+    torch.cuda.empty_cache()
 
 
 def test_ssd_split_matches_whole():
