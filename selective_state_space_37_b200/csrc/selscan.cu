@@ -268,32 +268,57 @@ int launch_ssd_tc(const tc::Params& base_p, const SsdParams& fold_p, const void*
     if (set_smem_limit(kmain, tc::kSmemBytes, attr_main, dev) != SS_OK ||
         set_smem_limit(kstate, tc::kSmemBytes, attr_state, dev) != SS_OK)
         return SS_ERR_CUDA;
-    int nseg = 1, cseg = static_cast<int>(nchunks);
-    if (have_ws) {
+    // Plan: items 0 .. n_whole - 1 run whole; the others are cut into nseg segments of cseg chunks
+    // (a state pass over the first nseg - 1, a fold, then every segment from its exact entering state).
+    int64_t n_whole = items, nseg = 1, cseg = nchunks;
+    if (have_ws && nchunks > 1) {
         const int64_t slots = sm_count_of_current_device();
-        if (chunk_len > 0) {
+        if (chunk_len > 0) {   // forced segment length: every item is cut
             int64_t cs = std::max<int64_t>(1, ceil_div(chunk_len, tc::kQ));
             if (ceil_div(nchunks, cs) > kmax) cs = ceil_div(nchunks, kmax);
-            cseg = static_cast<int>(cs);
-            nseg = static_cast<int>(ceil_div(nchunks, cs));
+            cseg = cs;
+            nseg = ceil_div(nchunks, cs);
+            n_whole = nseg > 1 ? 0 : items;
         } else {
-            double best = 0.0;
-            for (int64_t k = 1; k <= kmax; ++k) {
+            // Cost in chunk-times of the busiest SM (one CTA per SM): every item whole; every item cut into
+            // k segments; or only the items of the last, partly filled wave cut, so that their segments
+            // fill that wave.  Cut items add a state pass over k - 1 segments (about half the work of a
+            // chunk per chunk) and 10 % for the extra launches.
+            const int64_t waves = items / slots, tail = items - waves * slots;
+            auto cut_cost = [&](int64_t n, int64_t k, int64_t cs) {
+                return 1.1 * static_cast<double>(ceil_div(n * k, slots) * cs +
+                                                 ceil_div(n * (k - 1), slots) * cs / 2.0);
+            };
+            double best = static_cast<double>(ceil_div(items, slots) * nchunks);
+            for (int64_t k = 2; k <= kmax; ++k) {
                 const int64_t cs = ceil_div(nchunks, k);
                 if (ceil_div(nchunks, cs) != k) continue;
-                double cost = static_cast<double>(ceil_div(items * k, slots) * cs);
-                if (k > 1) cost = 1.1 * (cost + 0.5 * static_cast<double>(ceil_div(items * (k - 1), slots) * cs));
-                if (k == 1 || cost < best - 1e-9) {
-                    best = cost;
-                    nseg = static_cast<int>(k);
-                    cseg = static_cast<int>(cs);
+                const double every = cut_cost(items, k, cs);
+                if (every < best - 1e-9) {
+                    best = every;
+                    n_whole = 0;
+                    nseg = k;
+                    cseg = cs;
+                }
+                if (waves >= 1 && tail > 0) {
+                    const double last = static_cast<double>(waves * nchunks) + cut_cost(tail, k, cs);
+                    if (last < best - 1e-9) {
+                        best = last;
+                        n_whole = items - tail;
+                        nseg = k;
+                        cseg = cs;
+                    }
                 }
             }
         }
     }
-    p.nseg = nseg;
-    p.cseg = cseg;
-    if (items * nseg >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    const int64_t n_cut = nseg > 1 ? items - n_whole : 0;
+    if (nseg == 1) n_whole = items;
+    const int64_t grid = n_whole + n_cut * nseg;
+    if (grid >= (int64_t(1) << 31)) return SS_ERR_INVALID_ARG;
+    p.n_whole = static_cast<int>(n_whole);
+    p.nseg = static_cast<int>(nseg);
+    p.cseg = static_cast<int>(cseg);
     const int64_t H = p.H, batch = p.batch;
     CUtensorMap mx, mb, mc, my;
     {
@@ -311,16 +336,18 @@ int launch_ssd_tc(const tc::Params& base_p, const SsdParams& fold_p, const void*
             !make_map_sw128(&mc, C, 3, db, sb, bb) || !make_map_sw128(&my, p.y, 4, dx, sx, bx))
             return SS_ERR_CUDA;
     }
-    if (nseg > 1) {
-        kstate<<<static_cast<unsigned>(items * (nseg - 1)), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
-        SsdParams f = fold_p;
-        f.nseg = nseg;
-        const int64_t total = items * kSsdP * p.n;
+    if (n_cut > 0) {
+        kstate<<<static_cast<unsigned>(n_cut * (nseg - 1)), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
+        SsdParams f = fold_p;   // the fold runs over the cut items' records (their ranks as one batch row)
+        f.batch = 1;
+        f.H = static_cast<int>(n_cut);
+        f.nseg = static_cast<int>(nseg);
+        const int64_t total = n_cut * kSsdP * p.n;
         const int64_t blocks = std::min<int64_t>(ceil_div(total, 256), 4096);
         if (p.n == tc::kN) ss_ssd_fold_kernel<tc::kN><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(f);
         else ss_ssd_fold_kernel<64><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(f);
     }
-    kmain<<<static_cast<unsigned>(items * nseg), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
+    kmain<<<static_cast<unsigned>(grid), tc::kThreads, tc::kSmemBytes, stream>>>(p, mx, mb, mc, my);
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 

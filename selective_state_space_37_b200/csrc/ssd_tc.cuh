@@ -109,7 +109,9 @@ struct Params {
     float* esum;               // [batch, H, nseg]
     uint32_t* status;          // error word or null
     int64_t L;
-    int batch, H, nseg, cseg;  // cseg: chunks of kQ steps per segment
+    int batch, H;
+    int n_whole;               // (batch, head) sequences 0 .. n_whole - 1 run whole, one CTA each; the
+    int nseg, cseg;            // others are cut into nseg segments of cseg chunks of kQ steps
     int n;                     // d_state: 128, or 64 (B, C and the state padded to 128 with zeros)
     int softplus;
     int test_drop;             // test only: CTA 0 never signals its first C Bᵀ (a wait runs out)
@@ -274,8 +276,10 @@ __device__ __forceinline__ bool cw_any(bool pred) {
 }
 __device__ __forceinline__ void cw_sync() { asm volatile("bar.sync 1, 512;" ::: "memory"); }
 
-// Grid: one CTA per (segment k, batch b, head h), blockIdx.x = (k * batch + b) * H + h;
-// STATE runs segments 0 .. nseg - 2 only (G_out from zero, no outputs).
+// Grid: sequences are items i = b * H + h.  Main pass: CTAs 0 .. n_whole - 1 run items 0 .. n_whole - 1
+// whole; CTA n_whole + j runs segment j % nseg of item n_whole + j / nseg.  STATE: CTA j runs segment
+// j % (nseg - 1) of item n_whole + j / (nseg - 1) (segments 0 .. nseg - 2: G_out from zero, no outputs).
+// Segment records are indexed by the split item's rank r = i - n_whole.
 template <bool STATE>
 __global__ void __launch_bounds__(kThreads, 1)
 ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tm_x,
@@ -309,12 +313,27 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
     int* xw_slot = reinterpret_cast<int*>(gbase + kOffBar + 132);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int h = blockIdx.x % p.H;
-    const int b = (blockIdx.x / p.H) % p.batch;
-    const int sg = blockIdx.x / (p.H * p.batch);
+    int item, sg, nseg_i;
+    if (STATE) {
+        item = p.n_whole + static_cast<int>(blockIdx.x) / (p.nseg - 1);
+        sg = static_cast<int>(blockIdx.x) % (p.nseg - 1);
+        nseg_i = p.nseg;
+    } else if (static_cast<int>(blockIdx.x) < p.n_whole) {
+        item = static_cast<int>(blockIdx.x);
+        sg = 0;
+        nseg_i = 1;
+    } else {
+        const int j = static_cast<int>(blockIdx.x) - p.n_whole;
+        item = p.n_whole + j / p.nseg;
+        sg = j % p.nseg;
+        nseg_i = p.nseg;
+    }
+    const int64_t rk = item - p.n_whole;   // rank among the split items (records, Σ Δ A)
+    const int h = item % p.H;
+    const int b = item / p.H;
     const int64_t bh = static_cast<int64_t>(b) * p.H + h;
-    const int64_t seg_t0 = static_cast<int64_t>(sg) * p.cseg * kQ;
-    const int64_t seg_t1 = min(seg_t0 + static_cast<int64_t>(p.cseg) * kQ, p.L);
+    const int64_t seg_t0 = nseg_i == 1 ? 0 : static_cast<int64_t>(sg) * p.cseg * kQ;
+    const int64_t seg_t1 = nseg_i == 1 ? p.L : min(seg_t0 + static_cast<int64_t>(p.cseg) * kQ, p.L);
     const int nchunk = static_cast<int>((seg_t1 - seg_t0 + kQ - 1) / kQ);
     const uint64_t lim = p.wait_ns;
 
@@ -536,7 +555,7 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
         // (d_state 64: rows n >= 64 stay zero -- their B and C columns are zero)
         float G[kPT];
         const int nn = p.n;
-        const float* gin = (!STATE && sg > 0) ? p.rec + (bh * (p.nseg - 1) + (sg - 1)) * kP * nn : nullptr;
+        const float* gin = (!STATE && sg > 0) ? p.rec + (rk * (p.nseg - 1) + (sg - 1)) * kP * nn : nullptr;
 #pragma unroll
         for (int q = 0; q < kPT; ++q) G[q] = (gin && row < nn) ? gin[(kPT * qc + q) * nn + row] : 0.0f;
         auto store_g = [&]() {   // bf16 hi / lo copies of G: row n, chunks 2 qc, 2 qc + 1 of the [n][p] tiles
@@ -742,13 +761,13 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
         // outputs of the state: the segment's G_out (state pass) or the final state
         if (ok) {
             float* out = nullptr;
-            if (STATE) out = p.rec + (bh * (p.nseg - 1) + sg) * kP * nn;
-            else if (p.final_state && sg == p.nseg - 1) out = p.final_state + bh * kP * nn;
+            if (STATE) out = p.rec + (rk * (p.nseg - 1) + sg) * kP * nn;
+            else if (p.final_state && sg == nseg_i - 1) out = p.final_state + bh * kP * nn;
             if (out && row < nn) {
 #pragma unroll
                 for (int q2 = 0; q2 < kPT; ++q2) out[(kPT * qc + q2) * nn + row] = G[q2];
             }
-            if (STATE && tid == 0) p.esum[bh * p.nseg + sg] = esum;
+            if (STATE && tid == 0) p.esum[rk * p.nseg + sg] = esum;
         }
         if (tid == 0) {
             if (!STATE) bulk_wait0();

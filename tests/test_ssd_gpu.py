@@ -72,6 +72,7 @@ def test_ssd_full_size_sampled_heads():
                           sync_check=True)
     rng = np.random.default_rng(5)
     picks = [(int(rng.integers(b)), int(h)) for h in rng.choice(H, size=6, replace=False)]
+    picks.append((b - 1, H - 1))   # the last sequence: on 148 SMs it is among those cut into segments
     for bi, h in picks:
         yr, sr = oracle.ssd(to_f64(inp["x"][bi:bi + 1, :, h:h + 1]), to_f64(inp["dt"][bi:bi + 1, :, h:h + 1]),
                             to_f64(inp["A"][h:h + 1]), to_f64(inp["B"][bi:bi + 1]), to_f64(inp["C"][bi:bi + 1]),
