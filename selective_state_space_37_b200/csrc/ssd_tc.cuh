@@ -15,13 +15,13 @@
 // with G the P x N state entering the chunk.
 //
 // One CTA walks the chunks of one (b, h) in order, its warps specialised:
-//   warp 8 (producer, one thread): TMA loads of the x, B, C tiles and every
+//   warp 16 (producer, one thread): TMA loads of the x, B, C tiles and every
 //     MMA (bf16 operands, fp32 accumulation, M = 128):
 //       S   = C Bᵀ              128 x 128, K = N  -> TMEM columns [0, 128)
 //       CG  = C [G_hi | G_lo]ᵀ  128 x 128, K = N  -> TMEM columns [128, 256)
 //       ΔGᵀ = Bᵀ X̃              128 x 64,  K = Q  -> TMEM columns [320, 384)
 //       Y   = Mm X              128 x 64,  K = Q  -> TMEM columns [256, 320)
-//   warp 9: Δ, the prefix of Δ A and the decay factors, a chunk ahead into
+//   warp 17: Δ, the prefix of Δ A and the decay factors, a chunk ahead into
 //     a double buffer;
 //   warps 0..15 (compute): four threads per TMEM lane (one time step t, or
 //     one state index n), each on a quarter of the lane's columns: X̃ from x,
