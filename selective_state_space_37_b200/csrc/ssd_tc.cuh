@@ -37,10 +37,14 @@
 // wait that runs out records SS error -4 in the status word and the CTA
 // winds down (copies in flight drained, MMAs completed, TMEM released).
 //
-// Time segments: when batch x heads leaves SMs idle, each sequence is cut into
+// d_state 64 runs the same kernel with the second 64-column block of the B
+// and C tiles held at zero, so the state rows n >= 64 stay zero.
+//
+// Time segments: sequences that would leave SMs idle -- those of the last,
+// partly filled wave, or all of them when there are few -- are cut into
 // segments of whole chunks with an exact carry (state pass from G = 0 keeping
 // only G_out and Σ Δ A, the fold of ssd.cuh, then the main pass from each
-// segment's entering state).
+// segment's entering state); the host chooses the plan.
 #pragma once
 
 #include "common.cuh"
