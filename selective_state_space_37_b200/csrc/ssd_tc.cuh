@@ -18,7 +18,7 @@
 //   warp 16 (producer, one thread): TMA loads of the x, B, C tiles and every
 //     MMA (bf16 operands, fp32 accumulation, M = 128):
 //       S   = C Bᵀ              128 x 128, K = N  -> TMEM columns [0, 128)
-//       CG  = C [G_hi | G_lo]ᵀ  128 x 128, K = N  -> TMEM columns [128, 256)
+//       CG  = C G_hiᵀ + C G_loᵀ  128 x 64, K = N  -> TMEM columns [128, 192)
 //       ΔGᵀ = Bᵀ X̃              128 x 64,  K = Q  -> TMEM columns [320, 384)
 //       Y   = Mm X              128 x 64,  K = Q  -> TMEM columns [256, 320)
 //   warp 17: Δ, the prefix of Δ A and the decay factors, a chunk ahead into
@@ -33,7 +33,7 @@
 // update, and B and C of the next chunk load as soon as their last MMA is
 // done.  The carried state G stays fp32 in registers (the four threads of row
 // n hold G[:, n]); the product with C reads it as two bf16 terms G_hi + G_lo,
-// so it is not rounded to bf16 before the readout.  Every wait is bounded: a
+// accumulated into one tile, so it is not rounded to bf16 before the readout.  Every wait is bounded: a
 // wait that runs out records SS error -4 in the status word and the CTA
 // winds down (copies in flight drained, MMAs completed, TMEM released).
 //
@@ -69,7 +69,7 @@ constexpr int kPrefixWarp = kComputeWarps + 1;     // the Δ prefix, a chunk ahe
 constexpr int kThreads = kComputeThreads + 64;
 static_assert(kComputeThreads == 512 && kSB == 1 && kXC == 2, "the barriers and splits below assume 4 threads per row");
 constexpr uint32_t kTmemCols = 512;   // allocation (power of two >= the 384 columns used)
-constexpr uint32_t kColS = 0, kColCG = 128, kColY = 256, kColG = 320;
+constexpr uint32_t kColS = 0, kColCG = 128, kColY = 256, kColG = 320;   // CG: 64 columns
 
 // Instruction descriptors (kind::f16, bf16 x bf16 -> fp32, M = 128): bit 4 D
 // format f32, bits 7/10 A/B format bf16, bit 15/16 A/B major (1: MN-major),
@@ -431,14 +431,15 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                     issue_x(ci + 1);
                     ++x_issued;
                 }
-                if (!STATE) {   // CG = C [G_hi | G_lo]ᵀ: N = 128 over two MN blocks 16 KB apart
+                if (!STATE) {   // CG = C G_hiᵀ + C G_loᵀ, both accumulated into the same 64 columns
                     tc_fence_after();
                     if (carry) {
 #pragma unroll
                         for (int k = 0; k < kN / 16; ++k) {
                             const uint32_t aoff = (k >> 2) * 16384u + (k & 3) * 32u;
-                            umma(tmem + kColCG, sdesc(base + kOffC + aoff, 16, 1024),
-                                 sdesc(base + kOffGh + k * 2048u, 16384, 1024), kIdesc_128x128_KMN, k > 0);
+                            const uint64_t ad = sdesc(base + kOffC + aoff, 16, 1024);
+                            umma(tmem + kColCG, ad, sdesc(base + kOffGh + k * 2048u, 0, 1024), kIdesc_128x64_KMN, k > 0);
+                            umma(tmem + kColCG, ad, sdesc(base + kOffGl + k * 2048u, 0, 1024), kIdesc_128x64_KMN, 1);
                         }
                     }
                     umma_commit(cg_done);
@@ -723,17 +724,11 @@ ss_ssd_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ CUten
                 const int t = row;
                 const float et = __expf(cum[t]);
                 float acc[kPT];
-                {   // Y and C G_hiᵀ in one TMEM round trip, then C G_loᵀ
+                {   // Y and C Gᵀ in one TMEM round trip
                     float yg[2 * kPT];
                     tmem_ld16x2(tmem + lane_base + kColY + kPT * qc, tmem + lane_base + kColCG + kPT * qc, yg);
 #pragma unroll
                     for (int j = 0; j < kPT; ++j) acc[j] = carry ? fmaf(et, yg[kPT + j], yg[j]) : yg[j];
-                }
-                if (carry) {
-                    float gv[kPT];
-                    tmem_ld16(tmem + lane_base + kColCG + 64 + kPT * qc, gv);   // C G_loᵀ
-#pragma unroll
-                    for (int j = 0; j < kPT; ++j) acc[j] = fmaf(et, gv[j], acc[j]);
                 }
                 uint4 xv[kXC];
 #pragma unroll
