@@ -150,6 +150,7 @@ struct ChanParams {
     float Av[kHalf];   // raw A of this thread's states 8p .. 8p+7
     float a;           // A[ch, 0]; on the structured path A[ch, n] = a (n + 1)
     float ab;          // a (8p + 1): exponent factor of this half's first decay
+    float kq;          // 8p + 1: the power of r of this half's first decay
     float bias_s;      // bias in the softplus input's scale
     float Dv;
     uint32_t sp_mask;  // all ones: Δ goes through softplus
@@ -211,15 +212,16 @@ __device__ __forceinline__ float half_dot(const f32x2 (&Cp)[4], const f32x2 (&H)
     return lo + hi;
 }
 
-// One state update of this thread's half for one timestep.
+// One state update of this thread's half for one timestep.  Structured A:
+// lam is λ a (r = 2^(λ a)); otherwise λ.
 template <bool FAST, bool STRUCT, bool TRACK>
 __device__ __forceinline__ void half_update(float lam, float du, const f32x2 (&Bp)[4], f32x2 (&H)[4],
                                             f32x2 (&PP)[4], float& R, const ChanParams& cp) {
     const f32x2 DU = pk2(du, du);
     if (STRUCT) {
-        const float r = ex2_approx(lam * cp.a);
+        const float r = ex2_approx(lam);
         f32x2 Q[4];
-        half_ladder(ex2_approx(lam * cp.ab), r, Q);
+        half_ladder(ex2_approx(lam * cp.kq), r, Q);
 #pragma unroll
         for (int m = 0; m < 4; ++m) H[m] = fma2(Q[m], H[m], mul2(DU, Bp[m]));
         if (TRACK) R *= r;
@@ -235,23 +237,27 @@ __device__ __forceinline__ void half_update(float lam, float du, const f32x2 (&B
 
 // A group of NSTEP (even) timesteps of the scan, rows j0 .. j0+NSTEP-1.
 // us/dts/zs point at this channel's column of the tile (row 0); yrow at this
-// channel's output for row 0 of the tile.
-template <typename IO, bool FAST, bool STRUCT, bool TRACK, int NSTEP, bool CONV>
+// channel's output for row 0 of the tile.  FULL: softplus and gate both on
+// (known at compile time).
+template <typename IO, bool FAST, bool STRUCT, bool TRACK, int NSTEP, bool CONV, bool FULL>
 __device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* __restrict__ dts,
                                            const IO* __restrict__ zs, const float* __restrict__ bc, int j0,
                                            f32x2 (&H)[4], f32x2 (&PP)[4], float& R, const ChanParams& cp,
                                            IO* __restrict__ yrow, int64_t d) {
     constexpr int NH = NSTEP / 2;
-    // Phase A: this thread prepares steps j0 + 2i + p.
+    const uint32_t spm = FULL ? 0xffffffffu : cp.sp_mask;
+    const uint32_t zm = FULL ? 0xffffffffu : cp.z_mask;
+    // Phase A: this thread prepares steps j0 + 2i + p (λ a on the structured path).
     float lo[NH], dlo[NH], su[NH], g[NH];
 #pragma unroll
     for (int i = 0; i < NH; ++i) {
         const int row = (j0 + 2 * i + cp.p) * kCB;
         const float uu = u_at<IO, FAST, CONV>(us, j0 + 2 * i + cp.p, cp);
-        lo[i] = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
-        dlo[i] = lo[i] * uu;
+        const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, spm);
+        lo[i] = STRUCT ? lam * cp.a : lam;
+        dlo[i] = lam * uu;
         su[i] = cp.Dv * uu;
-        g[i] = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+        g[i] = blend(zm, gate_of<FAST>(to_f32(zs[row])), 1.0f);
     }
     float lam[NSTEP], du[NSTEP];
 #pragma unroll
@@ -283,18 +289,18 @@ __device__ __forceinline__ void scan_group(const IO* __restrict__ us, const IO* 
 }
 
 // One timestep of the scan (ragged tails); both threads prepare it.
-template <typename IO, bool FAST, bool STRUCT, bool TRACK, bool CONV>
+template <typename IO, bool FAST, bool STRUCT, bool TRACK, bool CONV, bool FULL>
 __device__ __forceinline__ void scan_one(const IO* __restrict__ us, const IO* __restrict__ dts,
                                          const IO* __restrict__ zs, const float* __restrict__ bc, int j,
                                          f32x2 (&H)[4], f32x2 (&PP)[4], float& R, const ChanParams& cp,
                                          IO* __restrict__ yrow, int64_t d) {
     const int row = j * kCB;
     const float uu = u_at<IO, FAST, CONV>(us, j, cp);
-    const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
-    const float g = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+    const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, FULL ? 0xffffffffu : cp.sp_mask);
+    const float g = blend(FULL ? 0xffffffffu : cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
     f32x2 Bp[4], Cp[4];
     load_bc(bc + j * 2 * kN, cp.p, Bp, Cp);
-    half_update<FAST, STRUCT, TRACK>(lam, lam * uu, Bp, H, PP, R, cp);
+    half_update<FAST, STRUCT, TRACK>(STRUCT ? lam * cp.a : lam, lam * uu, Bp, H, PP, R, cp);
     const float part = half_dot(Cp, H);
     const float yv = (part + partner(part) + cp.Dv * uu) * g;
     if (cp.valid && cp.p == 0) yrow[static_cast<int64_t>(j) * d] = from_f32<IO>(yv);
@@ -336,7 +342,7 @@ __device__ __forceinline__ float half_corr(float lam, const f32x2 (&Cp)[4], cons
 }
 
 // A group of NSTEP (even) timesteps of the fix-up pass.
-template <typename IO, bool FAST, bool STRUCT, int NSTEP>
+template <typename IO, bool FAST, bool STRUCT, int NSTEP, bool FULL>
 __device__ __forceinline__ void fix_group(const IO* __restrict__ ys, const IO* __restrict__ dts,
                                           const IO* __restrict__ zs, const float* __restrict__ bc, int j0,
                                           const f32x2 (&H0)[4], f32x2 (&PQ)[4], float& Rq, const ChanParams& cp,
@@ -346,8 +352,8 @@ __device__ __forceinline__ void fix_group(const IO* __restrict__ ys, const IO* _
 #pragma unroll
     for (int i = 0; i < NH; ++i) {
         const int row = (j0 + 2 * i + cp.p) * kCB;
-        lo[i] = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
-        g[i] = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+        lo[i] = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, FULL ? 0xffffffffu : cp.sp_mask);
+        g[i] = blend(FULL ? 0xffffffffu : cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
         yo[i] = to_f32(ys[row]);
     }
     float lam[NSTEP];
@@ -373,14 +379,14 @@ __device__ __forceinline__ void fix_group(const IO* __restrict__ ys, const IO* _
     }
 }
 
-template <typename IO, bool FAST, bool STRUCT>
+template <typename IO, bool FAST, bool STRUCT, bool FULL>
 __device__ __forceinline__ void fix_one(const IO* __restrict__ ys, const IO* __restrict__ dts,
                                         const IO* __restrict__ zs, const float* __restrict__ bc, int j,
                                         const f32x2 (&H0)[4], f32x2 (&PQ)[4], float& Rq, const ChanParams& cp,
                                         IO* __restrict__ yrow, int64_t d) {
     const int row = j * kCB;
-    const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, cp.sp_mask);
-    const float g = blend(cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
+    const float lam = lam_of<FAST>(to_f32(dts[row]), cp.bias_s, FULL ? 0xffffffffu : cp.sp_mask);
+    const float g = blend(FULL ? 0xffffffffu : cp.z_mask, gate_of<FAST>(to_f32(zs[row])), 1.0f);
     f32x2 Cp[4];
     load_c(bc + j * 2 * kN, cp.p, Cp);
     const float part = half_corr<FAST, STRUCT>(lam, Cp, H0, PQ, Rq, cp);
@@ -481,7 +487,7 @@ struct ItemCtx {
 
 // The scan (and, for a provisional chunk, look-back and fix-up) of one item,
 // specialised on the decay form and on whether the entry state is known.
-template <typename IO, bool USE_TMA, int STAGES, int G, bool UNROLL, bool STRUCT, bool EXACT, bool CONV>
+template <typename IO, bool USE_TMA, int STAGES, int G, bool UNROLL, bool STRUCT, bool EXACT, bool CONV, bool FULL>
 __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it, const ChanParams& cp,
                                          f32x2 (&H)[4]) {
     constexpr bool FAST = std::is_same<IO, __nv_bfloat16>::value;
@@ -511,12 +517,12 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
         if (UNROLL && nt == kTT) {
 #pragma unroll
             for (int gi = 0; gi < kTT / G; ++gi)
-                scan_group<IO, FAST, STRUCT, TRACK, G, CONV>(us, dts, zs, bc, gi * G, H, PP, R, cp, yrow, d);
+                scan_group<IO, FAST, STRUCT, TRACK, G, CONV, FULL>(us, dts, zs, bc, gi * G, H, PP, R, cp, yrow, d);
         } else {
             int j0 = 0;
             for (; j0 + G <= nt; j0 += G)
-                scan_group<IO, FAST, STRUCT, TRACK, G, CONV>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
-            for (; j0 < nt; ++j0) scan_one<IO, FAST, STRUCT, TRACK, CONV>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+                scan_group<IO, FAST, STRUCT, TRACK, G, CONV, FULL>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
+            for (; j0 < nt; ++j0) scan_one<IO, FAST, STRUCT, TRACK, CONV, FULL>(us, dts, zs, bc, j0, H, PP, R, cp, yrow, d);
         }
         t += nt;
     }
@@ -655,16 +661,17 @@ __device__ __forceinline__ void run_item(const ItemCtx<IO, USE_TMA, STAGES>& it,
             const float* bc = &S.bc[s][0][0];
             IO* yrow = ybase + (t - it.t_begin) * d;
             int j0 = 0;
-            for (; j0 + G <= nt; j0 += G) fix_group<IO, FAST, STRUCT, G>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
-            for (; j0 < nt; ++j0)           fix_one<IO, FAST, STRUCT>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
+            for (; j0 + G <= nt; j0 += G) fix_group<IO, FAST, STRUCT, G, FULL>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
+            for (; j0 < nt; ++j0)           fix_one<IO, FAST, STRUCT, FULL>(ys, dts, zs, bc, j0, H0, PQ, Rq, cp, yrow, d);
             t += nt;
         }
     }
 }
 
 // MINB resident CTAs per SM, groups of G steps, whole tiles unrolled or not;
-// CONV: u comes from the causal conv1d + SiLU prologue over x.
-template <typename IO, bool USE_TMA, int STAGES, int MINB, int G, bool UNROLL, bool CONV>
+// CONV: u comes from the causal conv1d + SiLU prologue over x; FULL: the
+// softplus and the gate are both on (the host launches it only then).
+template <typename IO, bool USE_TMA, int STAGES, int MINB, int G, bool UNROLL, bool CONV, bool FULL>
 __global__ void __launch_bounds__(kNT, MINB)
 ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_u,
               const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ CUtensorMap tm_z,
@@ -726,6 +733,7 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
     const int all_struct = __syncthreads_and(structured ? 1 : 0);
     const bool use_struct = FAST && all_struct && !(p.pflags & kPfForceGeneral);
     cp.ab = cp.a * static_cast<float>(hp + 1);
+    cp.kq = static_cast<float>(hp + 1);
     cp.Dv = (cp.valid && (p.pflags & kPfHasD)) ? __ldg(p.D + ch) : 0.f;
     const float biasv = (cp.valid && (p.pflags & kPfHasBias)) ? __ldg(p.bias + ch) : 0.f;
     cp.bias_s = FAST ? biasv * kLog2e : biasv;
@@ -774,11 +782,11 @@ ss_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUten
 
     static_assert(G % 2 == 0 && kTT % G == 0, "groups hold an even number of steps and tile a tile");
     if (use_struct) {
-        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, true, true, CONV>(it, cp, H);
-        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, true, false, CONV>(it, cp, H);
+        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, true, true, CONV, FULL>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, true, false, CONV, FULL>(it, cp, H);
     } else {
-        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, false, true, CONV>(it, cp, H);
-        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, false, false, CONV>(it, cp, H);
+        if (exact) run_item<IO, USE_TMA, STAGES, G, UNROLL, false, true, CONV, FULL>(it, cp, H);
+        else       run_item<IO, USE_TMA, STAGES, G, UNROLL, false, false, CONV, FULL>(it, cp, H);
     }
 }
 

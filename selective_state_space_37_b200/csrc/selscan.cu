@@ -181,9 +181,9 @@ bool make_map(CUtensorMap* m, const void* base, bool bf16, uint64_t inner, uint6
     return r == CUDA_SUCCESS;
 }
 
-template <typename IO, bool TMA, int STAGES, int MINB, int G, bool UNROLL, bool CONV>
+template <typename IO, bool TMA, int STAGES, int MINB, int G, bool UNROLL, bool CONV, bool FULL = false>
 int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
-    auto kern = ss_fwd_kernel<IO, TMA, STAGES, MINB, G, UNROLL, CONV>;
+    auto kern = ss_fwd_kernel<IO, TMA, STAGES, MINB, G, UNROLL, CONV, FULL>;
     const size_t smem = sizeof(FwdSmem<IO, STAGES>);
     static std::atomic<bool> attr_set[kMaxDevices];
     int dev = 0;
@@ -193,17 +193,24 @@ int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaS
     return cudaGetLastError() == cudaSuccess ? SS_OK : SS_ERR_CUDA;
 }
 
-// Forward-kernel instantiation for the variant, element type, TMA use and
-// the conv prologue.
+// Forward-kernel instantiation for the variant, element type, TMA use, the
+// conv prologue and (bf16) whether the softplus and the gate are both on.
+template <bool CONV, bool FULL>
+int launch_bf16(bool tma, Variant v, const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
+    if (v == kNarrow)
+        return tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 4, false, CONV, FULL>(p, items, maps, stream)
+                   : launch_fwd<__nv_bfloat16, false, 1, 2, 4, false, CONV, FULL>(p, items, maps, stream);
+    return tma ? launch_fwd<__nv_bfloat16, true, 4, 1, 8, true, CONV, FULL>(p, items, maps, stream)
+               : launch_fwd<__nv_bfloat16, false, 1, 1, 8, true, CONV, FULL>(p, items, maps, stream);
+}
+
 template <bool CONV>
 int launch_variant(bool bf16, bool tma, Variant v, const FwdParams& p, int64_t items, const CUtensorMap* maps,
                    cudaStream_t stream) {
     if (bf16) {
-        if (v == kNarrow)
-            return tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 4, false, CONV>(p, items, maps, stream)
-                       : launch_fwd<__nv_bfloat16, false, 1, 2, 4, false, CONV>(p, items, maps, stream);
-        return tma ? launch_fwd<__nv_bfloat16, true, 4, 1, 8, true, CONV>(p, items, maps, stream)
-                   : launch_fwd<__nv_bfloat16, false, 1, 1, 8, true, CONV>(p, items, maps, stream);
+        const bool full = (p.pflags & kPfSoftplus) && (p.pflags & kPfHasZ);
+        return full ? launch_bf16<CONV, true>(tma, v, p, items, maps, stream)
+                    : launch_bf16<CONV, false>(tma, v, p, items, maps, stream);
     }
     return tma ? launch_fwd<float, true, 2, 1, 8, false, CONV>(p, items, maps, stream)
                : launch_fwd<float, false, 1, 1, 8, false, CONV>(p, items, maps, stream);
