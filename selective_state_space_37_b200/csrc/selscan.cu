@@ -67,9 +67,9 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // scheduler), a 4-stage tile ring, groups of 8 steps with whole tiles
 // unrolled -- fastest when every SM can work on channels whose entry state is
 // known.  Narrow: two resident CTAs per SM (four warps per scheduler, <= 128
-// registers), a 3-stage ring, groups of 4 -- better latency hiding when a
-// problem has few channel blocks, so that almost every time chunk is
-// provisional anyway.
+// registers), a 3-stage ring, groups of 8 with the 32-step tile unrolled --
+// better latency hiding when a problem has few channel blocks, so that almost
+// every time chunk is provisional anyway.
 enum Variant { kWide = 0, kNarrow = 1 };
 constexpr int kCtasPerSm[2] = {1, 2};
 // Items per resident CTA slot the automatic chunking aims for (load balance:
@@ -198,7 +198,7 @@ int launch_fwd(const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaS
 template <bool CONV, bool FULL>
 int launch_bf16(bool tma, Variant v, const FwdParams& p, int64_t items, const CUtensorMap* maps, cudaStream_t stream) {
     if (v == kNarrow)
-        return tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 4, false, CONV, FULL>(p, items, maps, stream)
+        return tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 8, true, CONV, FULL>(p, items, maps, stream)
                    : launch_fwd<__nv_bfloat16, false, 1, 2, 4, false, CONV, FULL>(p, items, maps, stream);
     return tma ? launch_fwd<__nv_bfloat16, true, 4, 1, 8, true, CONV, FULL>(p, items, maps, stream)
                : launch_fwd<__nv_bfloat16, false, 1, 1, 8, true, CONV, FULL>(p, items, maps, stream);
