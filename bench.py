@@ -38,7 +38,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 # device code of the forward kernel (the profile's traffic figure is used only
 # while these files are unchanged)
 KERNEL_SOURCES = ["selective_state_space_37_b200/csrc/fwd.cuh",
-                  "selective_state_space_37_b200/csrc/common.cuh"]
+                  "selective_state_space_37_b200/csrc/common.cuh",
+                  "selective_state_space_37_b200/csrc/selscan.cu"]   # launch shapes
 
 
 def parse_args():
