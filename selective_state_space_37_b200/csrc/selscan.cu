@@ -64,7 +64,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Forward-kernel variants.  Wide: one resident CTA per SM (two warps per
-// scheduler), a 4-stage tile ring, groups of 4 steps with whole tiles
+// scheduler), a 2-stage tile ring, groups of 4 steps with whole tiles
 // unrolled -- fastest when every SM can work on channels whose entry state is
 // known.  Narrow: two resident CTAs per SM (four warps per scheduler, <= 128
 // registers), a 3-stage ring, groups of 8 with the 32-step tile unrolled --
@@ -200,7 +200,7 @@ int launch_bf16(bool tma, Variant v, const FwdParams& p, int64_t items, const CU
     if (v == kNarrow)
         return tma ? launch_fwd<__nv_bfloat16, true, 3, 2, 8, true, CONV, FULL>(p, items, maps, stream)
                    : launch_fwd<__nv_bfloat16, false, 1, 2, 4, false, CONV, FULL>(p, items, maps, stream);
-    return tma ? launch_fwd<__nv_bfloat16, true, 4, 1, 4, true, CONV, FULL>(p, items, maps, stream)
+    return tma ? launch_fwd<__nv_bfloat16, true, 2, 1, 4, true, CONV, FULL>(p, items, maps, stream)
                : launch_fwd<__nv_bfloat16, false, 1, 1, 8, true, CONV, FULL>(p, items, maps, stream);
 }
 
