@@ -132,11 +132,12 @@ def aggregate_value(world, per_rank_bytes, steps, ms_max):
 # structured-A path, counted from its source (both threads of a channel pair):
 # 3 decay-exponent arguments (λ·a once, by the thread that prepares the step;
 # λa·(8p+1) in each thread), 16 ladder products for the 16 decays, 16 Δu·B
-# products, 16 state FMAs, 16 readout products, 6 pair-sum reductions, and 9
-# scalar operations of the step's own (softplus argument, 1 + 2^y, Δu, D u,
-# two for the gate, three for the output).  ncu's FMA-pipe activity on the
-# 2.8B-shaped layer (49 %) agrees with this count.
-FP32_OPS_PER_CH_TS = 82
+# products, 16 state FMAs, 16 readout products, 2 lane-pair sums of the
+# readout (one per thread), and 9 scalar operations of the step's own
+# (softplus argument, 1 + 2^y, Δu, D u, two for the gate, three for the
+# output).  ncu's FMA-pipe activity on the 2.8B-shaped layer (48 %) agrees
+# with this count.
+FP32_OPS_PER_CH_TS = 78
 
 
 def alu_roofline(torch, device, ch_ts_per_s, clock_summary):

@@ -201,14 +201,15 @@ __device__ __forceinline__ void load_c(const float* __restrict__ bcrow, int p, f
     Cp[0] = pk2(c0.x, c0.y); Cp[1] = pk2(c0.z, c0.w); Cp[2] = pk2(c1.x, c1.y); Cp[3] = pk2(c1.z, c1.w);
 }
 
-// This thread's half of the readout Σ_n C_n h_n.
+// This thread's half of the readout Σ_n C_n h_n: one chain of packed
+// products (even and odd states), then the two lanes' sum.
 __device__ __forceinline__ float half_dot(const f32x2 (&Cp)[4], const f32x2 (&H)[4]) {
-    f32x2 a0 = mul2(Cp[0], H[0]);
-    f32x2 a1 = mul2(Cp[1], H[1]);
-    a0 = fma2(Cp[2], H[2], a0);
-    a1 = fma2(Cp[3], H[3], a1);
+    f32x2 a = mul2(Cp[0], H[0]);
+    a = fma2(Cp[1], H[1], a);
+    a = fma2(Cp[2], H[2], a);
+    a = fma2(Cp[3], H[3], a);
     float lo, hi;
-    upk2(add2(a0, a1), lo, hi);
+    upk2(a, lo, hi);
     return lo + hi;
 }
 
