@@ -49,6 +49,18 @@ def test_fwd_conv_bf16(shape, chunk):
     check(inp, w, cb, y, st)
 
 
+@pytest.mark.parametrize("shape", [(38, 100, 512), (2, 200, 200)], ids=["wide", "narrow"])
+def test_fwd_conv_bf16_no_gate(shape):
+    """Without the gate the prologue runs in the kernel that is not
+    specialised for softplus and gate both on."""
+    b, L, d = shape
+    inp = fwd_inputs(b, L, d, 16, "bf16", 640 + d, DEV, gate=False, D_kind="normal")
+    w, cb = conv_params(d, 640 + d, DEV, bias="normal")
+    for chunk in (0, 64):
+        y, st = run(inp, w, cb, chunk_len=chunk)
+        check(inp, w, cb, y, st)
+
+
 @pytest.mark.parametrize("chunk", [0, 64])
 def test_fwd_conv_fp32(chunk):
     inp = fwd_inputs(2, 130, 64, 16, "fp32", 71, DEV, gate=True, D_kind="normal")

@@ -78,6 +78,19 @@ def test_wide_variant_shapes(shape):
         check_full(inp, y, st, precisions=("f32",))
 
 
+@pytest.mark.parametrize("gate,softplus", [(False, True), (True, False), (False, False)],
+                         ids=["no_gate", "no_softplus", "neither"])
+def test_wide_variant_options(gate, softplus):
+    """The one-CTA-per-SM variant with the gate or the softplus off: the
+    kernel instantiated for both on is not the one that runs here."""
+    inp = fwd_inputs(38, 100, 512, 16, "bf16", 61, DEV, gate=gate, D_kind="normal", bias=softplus)
+    if not softplus:
+        inp["delta"] = (inp["delta"].float().abs() * 0.1).to(torch.bfloat16)
+    for chunk in (0, 64):
+        y, st = run(inp, chunk_len=chunk, softplus=softplus, sync_check=True)
+        check_full(inp, y, st, precisions=("f32",), softplus=softplus)
+
+
 @pytest.mark.parametrize("shape", [(2, 130, 64), (1, 70, 96), (2, 200, 30)])
 @pytest.mark.parametrize("chunk", [0, 64])
 def test_small_fp32(shape, chunk):
